@@ -1,0 +1,319 @@
+/*
+ * oracle.c -- plain, slow, fp64 CPU oracle of training-free block-sparse
+ * self-attention for video DiTs.  TEST INFRASTRUCTURE ONLY: the tests, the
+ * smoke check and the bench's CPU-baseline leg call it; the product path never
+ * does.  It shares no code, header or table with the CUDA library.
+ *
+ * What it computes follows the SubBlock router description on the page
+ * "MiniMax-H3 on 8xH200 benchmark" (news.paixiangai.cn), section "How SubBlock
+ * sparse attention works": queries and keys are cut into 64-token blocks, a
+ * light pooling step scores every key block for every query block and head, the
+ * top-scoring key blocks are kept and their indices handed to an exact
+ * block-sparse attention; `sparsity` is the fraction of key blocks dropped.
+ * The scoring is taken in its one-sub-block form: the score of key block J for
+ * query block I is mean(q over I) . mean(k over J) / sqrt(D).  The kept count
+ * is ceil((1 - s) * nKV) with ties broken towards the lower block index.
+ *
+ * Every function is the definition written out with plain loops, in fp64,
+ * in token order.  Inputs are bf16 bit patterns, widened exactly.
+ *
+ * Layouts: q, k, v are [B, H, Npad, D] row-major bf16; valid_len[b] is the
+ * number of real tokens of sample b (rows >= valid_len[b] are padding).
+ * Blocks: nB_b = ceil(valid_len[b] / block); block I holds tokens
+ * [I*block, min((I+1)*block, valid_len[b])).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+static double bf16_to_f64(uint16_t bits) {
+    uint32_t u = ((uint32_t)bits) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+static int n_blocks_of(int len, int block) { return (len + block - 1) / block; }
+
+/* Kept-count rule: clamp(ceil((1 - s) * n - 1e-9), 1, n), evaluated in fp64.
+ * The 1e-9 absorbs representation error such as (1 - 0.7) * 10 = 3.0000000000000004. */
+int32_t oracle_keep_count(int32_t n, double sparsity) {
+    if (n <= 0) return 0;
+    double x = ceil((1.0 - sparsity) * (double)n - 1e-9);
+    if (x < 1.0) x = 1.0;
+    if (x > (double)n) x = (double)n;
+    return (int32_t)x;
+}
+
+/* Mean of each block over its valid tokens.  out: [B, H, nBmax, D] with
+ * nBmax = Npad / block; blocks at or past nB_b are written as 0. */
+void oracle_pool(const uint16_t* x, int B, int H, int Npad, int D,
+                 const int32_t* valid_len, int block, double* out) {
+    int nBmax = Npad / block;
+#pragma omp parallel for collapse(2) schedule(dynamic)
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H; ++h) {
+            const uint16_t* xs = x + ((size_t)b * H + h) * (size_t)Npad * D;
+            int L = valid_len[b];
+            for (int I = 0; I < nBmax; ++I) {
+                double* o = out + (((size_t)b * H + h) * nBmax + I) * D;
+                int n0 = I * block, n1 = n0 + block < L ? n0 + block : L;
+                for (int d = 0; d < D; ++d) {
+                    double s = 0.0;
+                    for (int n = n0; n < n1; ++n) s += bf16_to_f64(xs[(size_t)n * D + d]);
+                    o[d] = (n1 > n0) ? s / (double)(n1 - n0) : 0.0;
+                }
+            }
+        }
+}
+
+/* Block scores S[b,h,I,J] = sum_d qbar[I,d] * kbar[J,d] * (1/sqrt(D)) for
+ * I, J < nB_b; entries outside that square are NAN.  S: [B, H, nBmax, nBmax]. */
+void oracle_scores(const double* qbar, const double* kbar, int B, int H, int nBmax, int D,
+                   const int32_t* valid_len, int block, double* S) {
+    double inv = 1.0 / sqrt((double)D);
+#pragma omp parallel for collapse(2) schedule(dynamic)
+    for (int b = 0; b < B; ++b) {
+        for (int h = 0; h < H; ++h) {
+            int nB = n_blocks_of(valid_len[b], block);
+            const double* qb = qbar + ((size_t)b * H + h) * nBmax * D;
+            const double* kb = kbar + ((size_t)b * H + h) * nBmax * D;
+            double* Sb = S + ((size_t)b * H + h) * nBmax * nBmax;
+            for (int I = 0; I < nBmax; ++I)
+                for (int J = 0; J < nBmax; ++J) {
+                    if (I >= nB || J >= nB) { Sb[(size_t)I * nBmax + J] = NAN; continue; }
+                    double s = 0.0;
+                    for (int d = 0; d < D; ++d) s += qb[(size_t)I * D + d] * kb[(size_t)J * D + d];
+                    Sb[(size_t)I * nBmax + J] = s * inv;
+                }
+        }
+    }
+}
+
+typedef struct { double score; int32_t index; } scored_block;
+
+/* Order: higher score first; equal scores -> lower block index first.  This is a
+ * total order, so the sort result does not depend on the sort's stability. */
+static int by_score_desc_index_asc(const void* pa, const void* pb) {
+    const scored_block* a = (const scored_block*)pa;
+    const scored_block* b = (const scored_block*)pb;
+    if (a->score > b->score) return -1;
+    if (a->score < b->score) return 1;
+    return (a->index > b->index) - (a->index < b->index);
+}
+
+static int int_asc(const void* pa, const void* pb) {
+    int32_t a = *(const int32_t*)pa, b = *(const int32_t*)pb;
+    return (a > b) - (a < b);
+}
+
+/* Top-k routing over precomputed scores S ([B,H,nBmax,nBmax], see oracle_scores).
+ * For each (b, h) and query block I < nB_b keep the k_b = keep(nB_b, s) best key
+ * blocks, written ascending to kv_idx[b,h,I,0..k_b) ([B,H,nBmax,kmax], unused
+ * tail entries = -1) with kv_cnt[b,h,I] = k_b; query blocks past nB_b get 0.
+ * Returns 0, or -1 when some k_b exceeds kmax. */
+int oracle_topk(const double* S, int B, int H, int nBmax, const int32_t* valid_len,
+                int block, double sparsity, int kmax, int32_t* kv_idx, int32_t* kv_cnt) {
+    int status = 0;
+    for (int b = 0; b < B; ++b)
+        if (oracle_keep_count(n_blocks_of(valid_len[b], block), sparsity) > kmax) status = -1;
+#pragma omp parallel
+    {
+        scored_block* row = (scored_block*)malloc(sizeof(scored_block) * (size_t)(nBmax > 0 ? nBmax : 1));
+#pragma omp for collapse(2) schedule(dynamic)
+        for (int b = 0; b < B; ++b)
+            for (int h = 0; h < H; ++h) {
+                int nB = n_blocks_of(valid_len[b], block);
+                int k = oracle_keep_count(nB, sparsity);
+                if (k > kmax) k = kmax;
+                for (int I = 0; I < nBmax; ++I) {
+                    size_t r = ((size_t)b * H + h) * nBmax + I;
+                    int32_t* idx = kv_idx + r * kmax;
+                    for (int t = 0; t < kmax; ++t) idx[t] = -1;
+                    if (I >= nB) { kv_cnt[r] = 0; continue; }
+                    for (int J = 0; J < nB; ++J) {
+                        row[J].score = S[r * nBmax + J];
+                        row[J].index = J;
+                    }
+                    qsort(row, (size_t)nB, sizeof(scored_block), by_score_desc_index_asc);
+                    for (int t = 0; t < k; ++t) idx[t] = row[t].index;
+                    qsort(idx, (size_t)k, sizeof(int32_t), int_asc);
+                    kv_cnt[r] = k;
+                }
+            }
+        free(row);
+    }
+    return status;
+}
+
+/* Whole selection: pool Q and K, score, route.  pooled_q / pooled_k / scores may
+ * be NULL; when given they receive the intermediate fp64 values. */
+int oracle_select(const uint16_t* q, const uint16_t* k, int B, int H, int Npad, int D,
+                  const int32_t* valid_len, int block, double sparsity, int kmax,
+                  int32_t* kv_idx, int32_t* kv_cnt,
+                  double* pooled_q, double* pooled_k, double* scores) {
+    int nBmax = Npad / block;
+    size_t np_ = (size_t)B * H * nBmax * D, ns = (size_t)B * H * nBmax * nBmax;
+    double* pq = pooled_q ? pooled_q : (double*)malloc(sizeof(double) * np_);
+    double* pk = pooled_k ? pooled_k : (double*)malloc(sizeof(double) * np_);
+    double* S = scores ? scores : (double*)malloc(sizeof(double) * ns);
+    oracle_pool(q, B, H, Npad, D, valid_len, block, pq);
+    oracle_pool(k, B, H, Npad, D, valid_len, block, pk);
+    oracle_scores(pq, pk, B, H, nBmax, D, valid_len, block, S);
+    int st = oracle_topk(S, B, H, nBmax, valid_len, block, sparsity, kmax, kv_idx, kv_cnt);
+    if (!pooled_q) free(pq);
+    if (!pooled_k) free(pk);
+    if (!scores) free(S);
+    return st;
+}
+
+/* Softmax attention of one query row over an explicit token list.
+ * logits_j = scale * sum_d q_d k_jd;  m = max_j logits_j;  p_j = exp(logits_j - m);
+ * Z = sum_j p_j;  o = sum_j p_j v_j / Z;  lse = m + log(Z).  An empty list gives
+ * o = 0 and lse = -inf.  buf holds the logits (n_tok entries). */
+static void attend_row(const uint16_t* qrow, const uint16_t* ks, const uint16_t* vs, int D,
+                       const int32_t* tok, int n_tok, double scale, double* buf,
+                       double* orow, double* lse, double* probs_out) {
+    for (int d = 0; d < D; ++d) orow[d] = 0.0;
+    if (n_tok == 0) { *lse = -INFINITY; return; }
+    double m = -INFINITY;
+    for (int t = 0; t < n_tok; ++t) {
+        const uint16_t* kr = ks + (size_t)tok[t] * D;
+        double s = 0.0;
+        for (int d = 0; d < D; ++d) s += bf16_to_f64(qrow[d]) * bf16_to_f64(kr[d]);
+        buf[t] = scale * s;
+        if (buf[t] > m) m = buf[t];
+    }
+    double Z = 0.0;
+    for (int t = 0; t < n_tok; ++t) { buf[t] = exp(buf[t] - m); Z += buf[t]; }
+    for (int t = 0; t < n_tok; ++t) {
+        const uint16_t* vr = vs + (size_t)tok[t] * D;
+        double w = buf[t] / Z;
+        if (probs_out) probs_out[tok[t]] = w;
+        for (int d = 0; d < D; ++d) orow[d] += w * bf16_to_f64(vr[d]);
+    }
+    *lse = m + log(Z);
+}
+
+/* Valid tokens of the kept blocks of one routing row, ascending.  Returns the
+ * count, or -1 if a block index is outside [0, nB_b). */
+static int kept_tokens(const int32_t* idx, int cnt, int nB, int L, int block, int32_t* tok) {
+    int n = 0;
+    for (int t = 0; t < cnt; ++t) {
+        int J = idx[t];
+        if (J < 0 || J >= nB) return -1;
+        for (int j = J * block; j < (J + 1) * block && j < L; ++j) tok[n++] = j;
+    }
+    return n;
+}
+
+/* Block-sparse attention with an external routing (kv_idx [B,H,nBmax,kmax],
+ * kv_cnt [B,H,nBmax]); nBmax = Npad / block.  For every valid query row i of
+ * query block I the row attends to the valid tokens of the blocks kv_idx[b,h,I,
+ * 0..kv_cnt).  Rows past valid_len[b] get o = 0 and lse = -inf.
+ * qblocks (NULL = all) restricts the work to the listed query blocks of every
+ * (b, h); rows outside them are left untouched.  scale <= 0 means 1/sqrt(D).
+ * o: [B,H,Npad,D] fp64, lse: [B,H,Npad] fp64.  Returns 0, or -1 on a routing
+ * entry outside the sample's blocks. */
+int oracle_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                     int B, int H, int Npad, int D, const int32_t* valid_len, int block,
+                     const int32_t* kv_idx, const int32_t* kv_cnt, int kmax, double scale,
+                     const int32_t* qblocks, int n_qblocks, double* o, double* lse) {
+    int nBmax = Npad / block;
+    int nq = qblocks ? n_qblocks : nBmax;
+    if (scale <= 0.0) scale = 1.0 / sqrt((double)D);
+    int status = 0;
+#pragma omp parallel
+    {
+        int32_t* tok = (int32_t*)malloc(sizeof(int32_t) * (size_t)Npad);
+        double* buf = (double*)malloc(sizeof(double) * (size_t)Npad);
+#pragma omp for collapse(3) schedule(dynamic)
+        for (int b = 0; b < B; ++b)
+            for (int h = 0; h < H; ++h)
+                for (int qi = 0; qi < nq; ++qi) {
+                    int I = qblocks ? qblocks[qi] : qi;
+                    int L = valid_len[b], nB = n_blocks_of(L, block);
+                    size_t bh = (size_t)b * H + h;
+                    const uint16_t* ks = k + bh * (size_t)Npad * D;
+                    const uint16_t* vs = v + bh * (size_t)Npad * D;
+                    size_t r = bh * nBmax + I;
+                    int n = kept_tokens(kv_idx + r * kmax, kv_cnt[r], nB, L, block, tok);
+                    if (n < 0) {
+#pragma omp atomic write
+                        status = -1;
+                        n = 0;
+                    }
+                    for (int i = I * block; i < (I + 1) * block; ++i) {
+                        double* orow = o + (bh * Npad + i) * D;
+                        double* l = lse + bh * Npad + i;
+                        if (i >= L) {
+                            for (int d = 0; d < D; ++d) orow[d] = 0.0;
+                            *l = -INFINITY;
+                            continue;
+                        }
+                        attend_row(q + (bh * Npad + i) * D, ks, vs, D, tok, n, scale, buf,
+                                   orow, l, NULL);
+                    }
+                }
+        free(tok);
+        free(buf);
+    }
+    return status;
+}
+
+/* Dense softmax attention over all valid tokens of the sample (no routing). */
+void oracle_dense(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                  int B, int H, int Npad, int D, const int32_t* valid_len, double scale,
+                  double* o, double* lse) {
+    if (scale <= 0.0) scale = 1.0 / sqrt((double)D);
+#pragma omp parallel
+    {
+        int32_t* tok = (int32_t*)malloc(sizeof(int32_t) * (size_t)Npad);
+        double* buf = (double*)malloc(sizeof(double) * (size_t)Npad);
+#pragma omp for collapse(3) schedule(dynamic)
+        for (int b = 0; b < B; ++b)
+            for (int h = 0; h < H; ++h)
+                for (int i = 0; i < Npad; ++i) {
+                    int L = valid_len[b];
+                    size_t bh = (size_t)b * H + h;
+                    double* orow = o + (bh * Npad + i) * D;
+                    double* l = lse + bh * Npad + i;
+                    if (i >= L) {
+                        for (int d = 0; d < D; ++d) orow[d] = 0.0;
+                        *l = -INFINITY;
+                        continue;
+                    }
+                    for (int j = 0; j < L; ++j) tok[j] = j;
+                    attend_row(q + (bh * Npad + i) * D, k + bh * (size_t)Npad * D,
+                               v + bh * (size_t)Npad * D, D, tok, L, scale, buf, orow, l, NULL);
+                }
+        free(tok);
+        free(buf);
+    }
+}
+
+/* Probability row of query row i of (b, h) under a routing: probs[j] for
+ * j in [0, Npad), zero outside the kept valid tokens.  Returns 0 or -1. */
+int oracle_probs(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                 int B, int H, int Npad, int D, const int32_t* valid_len, int block,
+                 const int32_t* kv_idx, const int32_t* kv_cnt, int kmax, double scale,
+                 int b, int h, int i, double* probs) {
+    (void)B;
+    int nBmax = Npad / block, L = valid_len[b], nB = n_blocks_of(L, block);
+    if (scale <= 0.0) scale = 1.0 / sqrt((double)D);
+    for (int j = 0; j < Npad; ++j) probs[j] = 0.0;
+    if (i >= L) return 0;
+    size_t bh = (size_t)b * H + h, r = bh * nBmax + i / block;
+    int32_t* tok = (int32_t*)malloc(sizeof(int32_t) * (size_t)Npad);
+    double* buf = (double*)malloc(sizeof(double) * (size_t)Npad);
+    double* orow = (double*)malloc(sizeof(double) * (size_t)D);
+    double lse;
+    int n = kept_tokens(kv_idx + r * kmax, kv_cnt[r], nB, L, block, tok);
+    int st = 0;
+    if (n < 0) st = -1;
+    else attend_row(q + (bh * Npad + i) * D, k + bh * (size_t)Npad * D, v + bh * (size_t)Npad * D,
+                    D, tok, n, scale, buf, orow, &lse, probs);
+    free(tok); free(buf); free(orow);
+    return st;
+}

@@ -1,0 +1,10 @@
+"""Seeded synthetic inputs shared by the oracle tests, the GPU tests and the bench.
+
+This package holds no arithmetic of the attention method itself: it only draws the
+Q, K, V fields, rounds them to bf16 and lays them out as padded [B, H, Npad, D]
+arrays with a per-sample valid length.
+"""
+from .synth import CONFIGS, Workload, make_workload, make_custom, bf16_bits_to_f32, f64_to_bf16_bits
+
+__all__ = ["CONFIGS", "Workload", "make_workload", "make_custom",
+           "bf16_bits_to_f32", "f64_to_bf16_bits"]
