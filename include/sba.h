@@ -1,0 +1,132 @@
+/*
+ * sba.h -- C ABI of the B200 (sm_100a) block-sparse self-attention library.
+ *
+ * The operation is training-free block-sparse self-attention over the token
+ * sequence of a video diffusion transformer, as the SubBlock router is described
+ * on the page "MiniMax-H3 on 8xH200 benchmark" (news.paixiangai.cn), section
+ * "How SubBlock sparse attention works": the sequence is cut into 64-token query
+ * and key blocks, a light pooling step scores each key block for each query
+ * block and head, the best key blocks are kept and their indices passed to an
+ * exact block-sparse attention kernel that never forms the full attention
+ * matrix; `sparsity` is the fraction of key blocks dropped (0.75 keeps about a
+ * quarter).  This library takes the one-sub-block form of that score:
+ *
+ *   qbar[I] = mean of q over the valid tokens of block I (same for kbar)
+ *   score[I][J] = qbar[I] . kbar[J] / sqrt(D)
+ *   kept(I) = the keep(nB, s) = clamp(ceil((1 - s) * nB - 1e-9), 1, nB) key
+ *             blocks of highest score, equal scores going to the lower index
+ *   o_i = sum_{j in kept tokens} softmax_j(scale * q_i . k_j) v_j   (non-causal)
+ *
+ * Conventions shared by every call:
+ *   - q, k, v, o: bf16, [B, H, Npad, D] contiguous row-major, device memory,
+ *     base addresses 16-byte aligned.  D is 64 or 128.  Npad % block == 0.
+ *   - valid_len: device int32 [B] with 1 <= valid_len[b] <= Npad, or NULL
+ *     (every sample is Npad long).  Rows n >= valid_len[b] are padding: they are
+ *     never read as keys or values, and their outputs are written as 0 (o) and
+ *     -inf (lse).  nB_b = ceil(valid_len[b] / block).
+ *   - block must be 64.
+ *   - Routing: kv_idx int32 [B, H, Npad/block, kmax] and kv_cnt int32
+ *     [B, H, Npad/block]; row (b, h, I) lists kv_cnt key-block indices in
+ *     ascending order in its first kv_cnt entries (later entries unspecified);
+ *     query blocks I >= nB_b have kv_cnt = 0.
+ *   - stream: a cudaStream_t (NULL = legacy default stream).  Every call is
+ *     asynchronous on that stream; the library never synchronises except in
+ *     sba_get_device_status.
+ *   - Ownership: the caller allocates and frees every buffer passed in.  The
+ *     library keeps only a small per-device cache of TMA tensor descriptors.
+ *   - Errors: argument checks run on the host before any launch and return an
+ *     sba_status without touching device memory.  A failed launch returns
+ *     SBA_ERR_CUDA.  Faults detected inside a kernel (a wait that gave up, a
+ *     routing entry outside [0, nB_b)) set a device-side error word that
+ *     sba_get_device_status reports.
+ */
+#ifndef SBA_H_
+#define SBA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SBA_OK = 0,
+    SBA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, sparsity outside [0,1), kmax too small */
+    SBA_ERR_UNSUPPORTED = 2,   /* D not 64/128, block not 64, Npad beyond SBA_MAX_NPAD */
+    SBA_ERR_ALIGNMENT = 3,     /* a device pointer not 16-byte aligned */
+    SBA_ERR_CUDA = 4,          /* a CUDA runtime or driver call failed */
+    SBA_ERR_TIMEOUT = 5,       /* a kernel wait gave up (reported by sba_get_device_status) */
+    SBA_ERR_DEVICE_FLAG = 6    /* a kernel found a bad routing entry (sba_get_device_status) */
+} sba_status;
+
+/* Largest padded sequence length a call accepts (4096 blocks of 64 tokens). */
+#define SBA_MAX_NPAD 262144
+
+/* Kept key blocks per query block for n_blocks candidate blocks at sparsity s:
+ * clamp(ceil((1 - s) * n_blocks - 1e-9), 1, n_blocks), evaluated in fp64; 0 when
+ * n_blocks <= 0.  Pure host function. */
+int32_t sba_keep_count(int32_t n_blocks, double sparsity);
+
+/* Bytes of device workspace sba_pool_select needs for this shape (0 on bad
+ * arguments).  The workspace holds the pooled Q and K block means. */
+size_t sba_pool_select_workspace_size(int B, int H, int Npad, int D, int block);
+
+/* Routing step: pool Q and K per block, score every key block for every query
+ * block, keep the best keep(nB_b, sparsity) blocks per (b, h, I).
+ *   q, k        bf16 [B, H, Npad, D] (read only)
+ *   valid_len   int32 [B] device, or NULL
+ *   sparsity    in [0, 1)
+ *   kmax        row capacity of kv_idx; must be >= sba_keep_count(Npad/block, s)
+ *   kv_idx      int32 [B, H, Npad/block, kmax] (written)
+ *   kv_cnt      int32 [B, H, Npad/block] (written)
+ *   workspace   device buffer of at least sba_pool_select_workspace_size bytes,
+ *               16-byte aligned; contents on entry are ignored
+ * The kept set equals the exact (real-number) top-k of the scores except where
+ * two scores differ by less than the fp64 rounding of their evaluation. */
+sba_status sba_pool_select(const void* q, const void* k, int B, int H, int Npad, int D,
+                           const int32_t* valid_len, int block, double sparsity, int kmax,
+                           int32_t* kv_idx, int32_t* kv_cnt,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/* Block means of x as fp64 values [B, H, Npad/block, D] (inspection helper;
+ * blocks past nB_b are written as 0).  `out` is device memory. */
+sba_status sba_block_means(const void* x, int B, int H, int Npad, int D,
+                           const int32_t* valid_len, int block, double* out, void* stream);
+
+/* Exact attention over the routed key blocks.
+ *   o      bf16 [B, H, Npad, D] (written; padding rows written as 0)
+ *   lse    fp32 [B, H, Npad] natural-log log-sum-exp of the scaled logits, or
+ *          NULL; padding rows and rows with no kept token get -inf
+ *   softmax_scale  multiplier of q.k; <= 0 selects 1/sqrt(D)
+ * A query row whose routing row is empty gets o = 0, lse = -inf. */
+sba_status sba_attention(const void* q, const void* k, const void* v, void* o, float* lse,
+                         int B, int H, int Npad, int D, const int32_t* valid_len, int block,
+                         const int32_t* kv_idx, const int32_t* kv_cnt, int kmax,
+                         float softmax_scale, void* stream);
+
+/* Dense attention over all valid tokens of each sample (the sparsity = 0 case
+ * without a routing), same layouts as sba_attention. */
+sba_status sba_dense_attention(const void* q, const void* k, const void* v, void* o, float* lse,
+                               int B, int H, int Npad, int D, const int32_t* valid_len,
+                               float softmax_scale, void* stream);
+
+/* Synchronises `stream`, returns and clears the device-side error word of the
+ * current device: SBA_OK, SBA_ERR_TIMEOUT or SBA_ERR_DEVICE_FLAG (or
+ * SBA_ERR_CUDA if the synchronisation itself failed). */
+sba_status sba_get_device_status(void* stream);
+
+/* Limit, in GPU clock cycles, of every wait inside the attention kernel
+ * (default about 2^32 cycles, i.e. seconds).  A wait that reaches it gives up,
+ * sets SBA_ERR_TIMEOUT and lets the kernel exit cleanly.  0 restores the
+ * default.  Meant for tests of the timeout path. */
+void sba_set_wait_limit(uint64_t cycles);
+
+/* Static description of a status code. */
+const char* sba_strerror(sba_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SBA_H_ */

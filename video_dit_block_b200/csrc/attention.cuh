@@ -1,0 +1,400 @@
+// attention.cuh -- exact softmax attention over routed 64-token key blocks, sm_100a.
+//
+// The computation is the block-sparse stage of the SubBlock router on the page
+// "MiniMax-H3 on 8xH200 benchmark" (news.paixiangai.cn), section "How SubBlock
+// sparse attention works": each query block attends, exactly, to the tokens of
+// its kept key blocks only, and the full attention matrix is never formed.
+//
+// Tiling.  A CTA owns two adjacent 64-row query blocks I0 = 2p, I1 = 2p + 1 of
+// one (b, h): a 128-row Q tile, the full-rate M of a single-CTA tcgen05.mma.
+// It walks the ascending union of the two kept lists; a key block kept by only
+// one of the two is masked to -inf for the other half's rows.
+//
+// Warp roles (192 threads):
+//   warps 0-3  softmax + epilogue; thread t owns query row t = TMEM lane t
+//   warp 4     builds the union list, then issues TMA loads (Q once, K/V per block)
+//   warp 5     allocates TMEM and issues the MMAs (one elected lane)
+// Per key block j:  S_j = Q K_j^T  (M=128, N=64, K=D) into TMEM buffer j%2;
+//                   softmax reads S_j, writes P_j (bf16) to shared memory;
+//                   O += P_j V_j (M=128, N=D, K=64) into the TMEM accumulator.
+// The MMA warp issues S_{j+1} before PV_j so the tensor core works on the next
+// scores while the softmax warps exponentiate.  The running max is only moved
+// when it grows by more than 8 (log2 units); O is then rescaled in TMEM.
+//
+// Every wait is bounded: on expiry the CTA records SBA_ERR_TIMEOUT, unwinds all
+// roles, drains its own TMA loads and MMAs and frees its TMEM.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+
+namespace sba {
+
+constexpr int kMaxBlocks = 4096;  // SBA_MAX_NPAD / 64
+
+struct AttnParams {
+    __nv_bfloat16* o;
+    float* lse;
+    const int32_t* valid_len;
+    const int32_t* kv_idx;
+    const int32_t* kv_cnt;
+    int H;
+    int Npad;
+    int kmax;
+    int dense;
+    float scale_log2;  // softmax scale * log2(e)
+    unsigned long long wait_limit;
+};
+
+template <int D, int NS>
+struct AttnSmem {
+    static constexpr int kQBytes = 128 * D * 2;
+    static constexpr int kKVBytes = 64 * D * 2;
+    static constexpr int kPBytes = 128 * 64 * 2;
+    static constexpr int kQ = 0;
+    static constexpr int kK = kQ + kQBytes;
+    static constexpr int kV = kK + NS * kKVBytes;
+    static constexpr int kP = kV + NS * kKVBytes;
+    static constexpr int kBars = kP + 2 * kPBytes;
+    // barriers: q_full, k_full[NS], v_full[NS], kv_empty[NS], s_full[2], p_full[2],
+    //           pv_done[2], drain
+    static constexpr int kNumBars = 1 + 3 * NS + 7;
+    static constexpr int kCtl = kBars + kNumBars * 8;      // tmem base, abort, n_union, pad
+    static constexpr int kBitmap = kCtl + 16;              // uint32 [2][kMaxBlocks/32]
+    static constexpr int kList = kBitmap + 2 * (kMaxBlocks / 32) * 4;  // uint16 [kMaxBlocks]
+    static constexpr int kTotal = kList + kMaxBlocks * 2;
+    static constexpr int kAlloc = kTotal + 1024;            // slack for 1024-byte alignment
+};
+
+__device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, uint64_t limit) {
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if ((uint64_t)(clock64() - t0) > limit) return false;
+    }
+    return true;
+}
+
+template <int D, int NS>
+__global__ void __launch_bounds__(192, 1)
+    attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+    using SM = AttnSmem<D, NS>;
+    constexpr int NCH = D / 64;                 // 128-byte column chunks per row
+    constexpr uint32_t kIdescS = idesc_bf16_f32(128, 64, 0, 0);
+    constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, 0, 1);
+    constexpr uint32_t kTmemCols = 256;         // S[2] at 0 / 64, O at 128
+
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* sm = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const uint32_t sQ = smem_u32(sm + SM::kQ);
+    const uint32_t sK = smem_u32(sm + SM::kK);
+    const uint32_t sV = smem_u32(sm + SM::kV);
+    const uint32_t sP = smem_u32(sm + SM::kP);
+    unsigned char* sPg = sm + SM::kP;
+    const uint32_t bars = smem_u32(sm + SM::kBars);
+    const uint32_t bar_q = bars;
+    auto bar_kf = [&](int s) { return bars + 8u * (1 + s); };
+    auto bar_vf = [&](int s) { return bars + 8u * (1 + NS + s); };
+    auto bar_ke = [&](int s) { return bars + 8u * (1 + 2 * NS + s); };
+    auto bar_sf = [&](int s) { return bars + 8u * (1 + 3 * NS + s); };
+    auto bar_pf = [&](int s) { return bars + 8u * (3 + 3 * NS + s); };
+    auto bar_pv = [&](int s) { return bars + 8u * (5 + 3 * NS + s); };
+    const uint32_t bar_drain = bars + 8u * (7 + 3 * NS);
+    uint32_t* ctl = reinterpret_cast<uint32_t*>(sm + SM::kCtl);
+    volatile uint32_t* abort_flag = ctl + 1;
+    uint32_t* bm = reinterpret_cast<uint32_t*>(sm + SM::kBitmap);
+    uint16_t* ulist = reinterpret_cast<uint16_t*>(sm + SM::kList);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int h = blockIdx.y, b = blockIdx.z;
+    const int bh = b * p.H + h;
+    const int nQ = p.Npad / 64;
+    const int I0 = 2 * blockIdx.x;
+    const int L = p.valid_len ? p.valid_len[b] : p.Npad;
+    const int nB = (L + 63) / 64;
+    const int W = (nB + 31) / 32;
+
+    if (tid == 0) {
+        mbar_init(bar_q, 1);
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(bar_kf(s), 1);
+            mbar_init(bar_vf(s), 1);
+            mbar_init(bar_ke(s), 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar_sf(s), 1);
+            mbar_init(bar_pf(s), 128);
+            mbar_init(bar_pv(s), 1);
+        }
+        mbar_init(bar_drain, 1);
+        *abort_flag = 0u;
+        fence_barrier_init();
+    }
+    if (warp == 5) tmem_alloc(smem_u32(ctl), kTmemCols);
+    if (warp == 4) {
+        // union of the two kept lists as a bitmap per half, then an ascending list
+        for (int w = lane; w < W; w += 32) {
+            uint32_t full = 0;
+            if (p.dense) full = (w * 32 + 32 <= nB) ? 0xffffffffu : ((1u << (nB - w * 32)) - 1u);
+            bm[w] = (p.dense && I0 < nB) ? full : 0u;
+            bm[kMaxBlocks / 32 + w] = (p.dense && I0 + 1 < nB) ? full : 0u;
+        }
+        __syncwarp();
+        if (!p.dense) {
+            for (int half = 0; half < 2; ++half) {
+                const int I = I0 + half;
+                if (I >= nQ) continue;
+                const size_t row = (size_t)bh * nQ + I;
+                int cnt = p.kv_cnt[row];
+                if (cnt < 0 || cnt > p.kmax) {
+                    raise_device_error(kErrBadRouting);
+                    cnt = cnt < 0 ? 0 : p.kmax;
+                }
+                const int32_t* lst = p.kv_idx + row * p.kmax;
+                for (int t = lane; t < cnt; t += 32) {
+                    const int J = lst[t];
+                    if (J >= 0 && J < nB)
+                        atomicOr(&bm[half * (kMaxBlocks / 32) + (J >> 5)], 1u << (J & 31));
+                    else
+                        raise_device_error(kErrBadRouting);
+                }
+            }
+        }
+        __syncwarp();
+        int base = 0;
+        for (int w0 = 0; w0 < W; w0 += 32) {
+            const int w = w0 + lane;
+            const uint32_t u = w < W ? (bm[w] | bm[kMaxBlocks / 32 + w]) : 0u;
+            const int c = __popc(u);
+            int incl = c;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += v;
+            }
+            int pos = base + incl - c;
+            uint32_t bits = u;
+            while (bits) {
+                const int bit = __ffs(bits) - 1;
+                bits &= bits - 1;
+                ulist[pos++] = static_cast<uint16_t>(w * 32 + bit);
+            }
+            base += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) ctl[2] = static_cast<uint32_t>(base);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ctl[0];
+    const int n = static_cast<int>(ctl[2]);
+    const uint64_t lim = p.wait_limit;
+
+    if (warp == 4) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0 && n > 0) {
+            tma_prefetch_desc(&tmQ);
+            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmV);
+            mbar_arrive_expect_tx(bar_q, SM::kQBytes);
+            for (int c = 0; c < NCH; ++c)
+                tma_load_3d(sQ + c * (128 * 128), &tmQ, bar_q, c * 64, I0 * 64, bh);
+            int issued = 0;
+            for (int j = 0; j < n; ++j) {
+                const int st = j % NS;
+                if (j >= NS && !wait_bounded(bar_ke(st), ((j / NS) - 1) & 1, abort_flag, lim)) break;
+                const int J = ulist[j];
+                mbar_arrive_expect_tx(bar_kf(st), SM::kKVBytes);
+                for (int c = 0; c < NCH; ++c)
+                    tma_load_3d(sK + st * SM::kKVBytes + c * (64 * 128), &tmK, bar_kf(st), c * 64,
+                                J * 64, bh);
+                mbar_arrive_expect_tx(bar_vf(st), SM::kKVBytes);
+                for (int c = 0; c < NCH; ++c)
+                    tma_load_3d(sV + st * SM::kKVBytes + c * (64 * 128), &tmV, bar_vf(st), c * 64,
+                                J * 64, bh);
+                issued = j + 1;
+            }
+            if (*abort_flag) {
+                // let this CTA's own copies land before the CTA exits
+                wait_drain(bar_q, 0, lim);
+                for (int j = issued > NS ? issued - NS : 0; j < issued; ++j) {
+                    wait_drain(bar_kf(j % NS), (j / NS) & 1, lim);
+                    wait_drain(bar_vf(j % NS), (j / NS) & 1, lim);
+                }
+            }
+        }
+    } else if (warp == 5) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0 && n > 0) {
+            bool ok = wait_bounded(bar_q, 0, abort_flag, lim);
+            tc_fence_after();
+            for (int j = 0; ok && j <= n; ++j) {
+                if (j < n) {
+                    const int st = j % NS;
+                    if (!wait_bounded(bar_kf(st), (j / NS) & 1, abort_flag, lim)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t dS = tmem + (j & 1) * 64;
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint64_t a = smem_desc_sw128(sQ + (kk / 4) * (128 * 128) + (kk % 4) * 32, 16, 1024);
+                        const uint64_t bd = smem_desc_sw128(
+                            sK + st * SM::kKVBytes + (kk / 4) * (64 * 128) + (kk % 4) * 32, 16, 1024);
+                        mma_bf16_ss(dS, a, bd, kIdescS, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(bar_sf(j & 1));
+                }
+                if (j >= 1) {
+                    const int jj = j - 1, st = jj % NS;
+                    if (!wait_bounded(bar_pf(jj & 1), (jj >> 1) & 1, abort_flag, lim)) { ok = false; break; }
+                    if (!wait_bounded(bar_vf(st), (jj / NS) & 1, abort_flag, lim)) { ok = false; break; }
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t a = smem_desc_sw128(sP + (jj & 1) * SM::kPBytes + kk * 32, 16, 1024);
+                        const uint64_t bd = smem_desc_sw128(sV + st * SM::kKVBytes + kk * (16 * 128),
+                                                            64 * 128, 1024);
+                        mma_bf16_ss(tmem + 128, a, bd, kIdescPV, (jj > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    mma_commit(bar_pv(jj & 1));
+                    mma_commit(bar_ke(st));
+                }
+            }
+            if (!ok) {
+                // every MMA this thread issued must finish before TMEM is freed
+                mma_commit(bar_drain);
+                wait_drain(bar_drain, 0, lim);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ softmax warps
+        const int r = tid;                      // query row of the tile = TMEM lane
+        const int half = r >> 6;
+        const int tok = (I0 + half) * 64 + (r & 63);
+        const uint32_t* bmh = bm + half * (kMaxBlocks / 32);
+        const uint32_t tl = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+        const float sc = p.scale_log2;
+        float m = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int j = 0; j < n; ++j) {
+            const int J = ulist[j];
+            const bool kept = (bmh[J >> 5] >> (J & 31)) & 1u;
+            int ncol = kept ? L - J * 64 : 0;
+            ncol = ncol > 64 ? 64 : ncol;
+            if (!warp_wait_bounded(bar_sf(j & 1), (j >> 1) & 1, abort_flag, lim)) { ok = false; break; }
+            tc_fence_after();
+            float x[64];
+            {
+                uint32_t a[32], c[32];
+                tmem_ld32(tl + (j & 1) * 64, a);
+                tmem_ld32(tl + (j & 1) * 64 + 32, c);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    x[i] = i < ncol ? __uint_as_float(a[i]) * sc : -INFINITY;
+                    x[32 + i] = 32 + i < ncol ? __uint_as_float(c[i]) * sc : -INFINITY;
+                }
+            }
+            float mloc = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < 64; ++i) mloc = fmaxf(mloc, x[i]);
+            const float m_new = fmaxf(m, mloc);
+            const bool grow = m_new > m + 8.f;
+            if (j > 0 && __any_sync(0xffffffffu, grow)) {
+                // O accumulates P V with the running max; move it and rescale O, l.
+                if (!warp_wait_bounded(bar_pv((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag, lim)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const float alpha = (m_new == -INFINITY) ? 1.f : ex2_approx(m - m_new);
+#pragma unroll
+                for (int ch = 0; ch < D / 32; ++ch) {
+                    uint32_t o[32];
+                    tmem_ld32(tl + 128 + ch * 32, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                    tmem_st32(tl + 128 + ch * 32, o);
+                }
+                tmem_wait_st();
+                l *= alpha;
+                m = m_new;
+            } else if (grow || j == 0) {
+                m = m_new;
+            }
+            const float mref = (m == -INFINITY) ? 0.f : m;
+            float rs = 0.f;
+            uint32_t pk[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const float p0 = ex2_approx(x[2 * i] - mref);
+                const float p1 = ex2_approx(x[2 * i + 1] - mref);
+                rs += p0 + p1;
+                __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+                pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+            }
+            l += rs;
+            // P buffer j%2 is free once PV(j-2) has completed
+            if (j >= 2 && !warp_wait_bounded(bar_pv(j & 1), ((j - 2) >> 1) & 1, abort_flag, lim)) {
+                ok = false;
+                break;
+            }
+            unsigned char* prow = sPg + (j & 1) * SM::kPBytes + r * 128;
+#pragma unroll
+            for (int c16 = 0; c16 < 8; ++c16)
+                *reinterpret_cast<uint4*>(prow + ((c16 ^ (r & 7)) << 4)) =
+                    make_uint4(pk[4 * c16], pk[4 * c16 + 1], pk[4 * c16 + 2], pk[4 * c16 + 3]);
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(bar_pf(j & 1));
+        }
+
+        // ------------------------------------------------------------ epilogue
+        if (ok && n > 0) ok = warp_wait_bounded(bar_pv((n - 1) & 1), ((n - 1) >> 1) & 1, abort_flag, lim);
+        tc_fence_after();
+        const bool in_range = tok < p.Npad && (I0 + half) < nQ;
+        const bool valid = tok < L && l > 0.f;
+        __nv_bfloat16* orow = p.o + ((size_t)bh * p.Npad + tok) * D;
+        if (ok) {
+            const float inv_l = valid ? 1.f / l : 0.f;
+#pragma unroll
+            for (int ch = 0; ch < D / 32; ++ch) {
+                uint32_t o[32];
+                if (n > 0) {
+                    tmem_ld32(tl + 128 + ch * 32, o);
+                    tmem_wait_ld();
+                }
+                if (in_range) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float o0 = (n > 0 && valid) ? __uint_as_float(o[2 * i]) * inv_l : 0.f;
+                        const float o1 = (n > 0 && valid) ? __uint_as_float(o[2 * i + 1]) * inv_l : 0.f;
+                        __nv_bfloat162 h2 = __floats2bfloat162_rn(o0, o1);
+                        pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+                    }
+                    uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4)
+                        dst[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+                }
+            }
+            if (in_range && p.lse)
+                p.lse[(size_t)bh * p.Npad + tok] =
+                    valid ? (m + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
+        }
+    }
+
+    // ---------------------------------------------------------------- teardown
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace sba

@@ -1,0 +1,246 @@
+// sba.cu -- host side of the C ABI declared in include/sba.h: argument checks,
+// TMA tensor-map encoding, launches and the device status word.  The whole
+// library is this one translation unit (kernels come from the .cuh files).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/sba.h"
+#include "attention.cuh"
+#include "common.cuh"
+#include "select.cuh"
+
+namespace {
+
+constexpr uint64_t kDefaultWaitLimit = 1ull << 32;  // clock cycles, ~2 s at 2 GHz
+uint64_t g_wait_limit = kDefaultWaitLimit;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+sba_status check_shape(int B, int H, int Npad, int D, int block) {
+    if (B <= 0 || H <= 0 || Npad <= 0) return SBA_ERR_INVALID_ARG;
+    if (B > 65535 || H > 65535) return SBA_ERR_UNSUPPORTED;
+    if (D != 64 && D != 128) return SBA_ERR_UNSUPPORTED;
+    if (block != 64) return SBA_ERR_UNSUPPORTED;
+    if (Npad % block != 0) return SBA_ERR_INVALID_ARG;
+    if (Npad > SBA_MAX_NPAD) return SBA_ERR_UNSUPPORTED;
+    return SBA_OK;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// [B*H, Npad, D] bf16 viewed as a 3-D tensor; box = 64 columns (128 B) x rows x 1,
+// 128-byte swizzle (the canonical K-major / MN-major SW128 operand layout).
+bool make_map(CUtensorMap* map, const void* base, int BH, int Npad, int D, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Npad, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Npad * D * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int D, int NS>
+sba_status launch_attention(const void* q, const void* k, const void* v, void* o, float* lse,
+                            int B, int H, int Npad, const int32_t* valid_len,
+                            const int32_t* kv_idx, const int32_t* kv_cnt, int kmax, int dense,
+                            float softmax_scale, cudaStream_t stream) {
+    using SM = sba::AttnSmem<D, NS>;
+    CUtensorMap tq, tk, tv;
+    const int BH = B * H;
+    if (!make_map(&tq, q, BH, Npad, D, 128) || !make_map(&tk, k, BH, Npad, D, 64) ||
+        !make_map(&tv, v, BH, Npad, D, 64))
+        return SBA_ERR_CUDA;
+    if (cudaFuncSetAttribute(sba::attn_kernel<D, NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SM::kAlloc) != cudaSuccess)
+        return SBA_ERR_CUDA;
+    sba::AttnParams p;
+    p.o = static_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.valid_len = valid_len;
+    p.kv_idx = kv_idx;
+    p.kv_cnt = kv_cnt;
+    p.H = H;
+    p.Npad = Npad;
+    p.kmax = kmax;
+    p.dense = dense;
+    const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)D);
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.wait_limit = g_wait_limit;
+    dim3 grid((Npad / 64 + 1) / 2, H, B);
+    sba::attn_kernel<D, NS><<<grid, 192, SM::kAlloc, stream>>>(tq, tk, tv, p);
+    return cudaGetLastError() == cudaSuccess ? SBA_OK : SBA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t sba_keep_count(int32_t n_blocks, double sparsity) {
+    return sba::keep_count(n_blocks, sparsity);
+}
+
+size_t sba_pool_select_workspace_size(int B, int H, int Npad, int D, int block) {
+    if (check_shape(B, H, Npad, D, block) != SBA_OK) return 0;
+    return sba::select_workspace_bytes((size_t)B * H, (size_t)Npad / block, (size_t)D);
+}
+
+sba_status sba_pool_select(const void* q, const void* k, int B, int H, int Npad, int D,
+                           const int32_t* valid_len, int block, double sparsity, int kmax,
+                           int32_t* kv_idx, int32_t* kv_cnt, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+    sba_status st = check_shape(B, H, Npad, D, block);
+    if (st != SBA_OK) return st;
+    if (!q || !k || !kv_idx || !kv_cnt || !workspace) return SBA_ERR_INVALID_ARG;
+    if (!(sparsity >= 0.0 && sparsity < 1.0)) return SBA_ERR_INVALID_ARG;
+    const int nB = Npad / block;
+    if (kmax < sba::keep_count(nB, sparsity)) return SBA_ERR_INVALID_ARG;
+    if (workspace_bytes < sba::select_workspace_bytes((size_t)B * H, nB, D)) return SBA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(workspace) || !aligned16(valid_len))
+        return SBA_ERR_ALIGNMENT;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t BH = (size_t)B * H;
+    sba::SelectWorkspace ws = sba::carve_select_workspace(workspace, BH, nB, D);
+    const long long groups = (long long)BH * nB;
+    const int gpc = 256 / (D / 8);  // block groups per CTA
+    const unsigned pool_grid = (unsigned)((groups + gpc - 1) / gpc);
+    // largest tile of query blocks whose score rows fit in shared memory
+    int TQ = 32;
+    while (TQ > 8 && sba::score_select_smem(D, TQ, nB) > 227 * 1024) TQ /= 2;
+    const size_t smem = sba::score_select_smem(D, TQ, nB);
+    if (smem > 227 * 1024) return SBA_ERR_UNSUPPORTED;
+    dim3 sgrid((nB + TQ - 1) / TQ, (unsigned)BH);
+    if (D == 128) {
+        sba::pool_kernel<128><<<pool_grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(q), valid_len, H, Npad,
+                                                        ws.qmean64, ws.qmean32, ws.qnorm, groups);
+        sba::pool_kernel<128><<<pool_grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(k), valid_len, H, Npad,
+                                                        ws.kmean64, ws.kmean32, ws.knorm, groups);
+        if (cudaFuncSetAttribute(sba::score_select_kernel<128>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+            return SBA_ERR_CUDA;
+        sba::score_select_kernel<128><<<sgrid, 256, smem, s>>>(ws, valid_len, H, Npad, sparsity, kmax,
+                                                               TQ, kv_idx, kv_cnt);
+    } else {
+        sba::pool_kernel<64><<<pool_grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(q), valid_len, H, Npad,
+                                                       ws.qmean64, ws.qmean32, ws.qnorm, groups);
+        sba::pool_kernel<64><<<pool_grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(k), valid_len, H, Npad,
+                                                       ws.kmean64, ws.kmean32, ws.knorm, groups);
+        if (cudaFuncSetAttribute(sba::score_select_kernel<64>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+            return SBA_ERR_CUDA;
+        sba::score_select_kernel<64><<<sgrid, 256, smem, s>>>(ws, valid_len, H, Npad, sparsity, kmax,
+                                                              TQ, kv_idx, kv_cnt);
+    }
+    return cudaGetLastError() == cudaSuccess ? SBA_OK : SBA_ERR_CUDA;
+}
+
+sba_status sba_block_means(const void* x, int B, int H, int Npad, int D, const int32_t* valid_len,
+                           int block, double* out, void* stream) {
+    sba_status st = check_shape(B, H, Npad, D, block);
+    if (st != SBA_OK) return st;
+    if (!x || !out) return SBA_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(out) || !aligned16(valid_len)) return SBA_ERR_ALIGNMENT;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const long long groups = (long long)B * H * (Npad / block);
+    const int gpc = 256 / (D / 8);
+    const unsigned grid = (unsigned)((groups + gpc - 1) / gpc);
+    if (D == 128)
+        sba::pool_kernel<128><<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), valid_len, H,
+                                                   Npad, out, nullptr, nullptr, groups);
+    else
+        sba::pool_kernel<64><<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), valid_len, H,
+                                                  Npad, out, nullptr, nullptr, groups);
+    return cudaGetLastError() == cudaSuccess ? SBA_OK : SBA_ERR_CUDA;
+}
+
+static sba_status attention_common(const void* q, const void* k, const void* v, void* o, float* lse,
+                                   int B, int H, int Npad, int D, const int32_t* valid_len,
+                                   int block, const int32_t* kv_idx, const int32_t* kv_cnt,
+                                   int kmax, int dense, float softmax_scale, void* stream) {
+    sba_status st = check_shape(B, H, Npad, D, block);
+    if (st != SBA_OK) return st;
+    if (!q || !k || !v || !o) return SBA_ERR_INVALID_ARG;
+    if (!dense && (!kv_idx || !kv_cnt || kmax <= 0)) return SBA_ERR_INVALID_ARG;
+    if (!std::isfinite(softmax_scale)) return SBA_ERR_INVALID_ARG;
+    if ((long long)B * H * Npad > (1ll << 31)) return SBA_ERR_UNSUPPORTED;  // 3-D TMA row index
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(valid_len) ||
+        (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) ||
+        (kv_idx && (reinterpret_cast<uintptr_t>(kv_idx) & 3u)) ||
+        (kv_cnt && (reinterpret_cast<uintptr_t>(kv_cnt) & 3u)))
+        return SBA_ERR_ALIGNMENT;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (D == 128)
+        return launch_attention<128, 4>(q, k, v, o, lse, B, H, Npad, valid_len, kv_idx, kv_cnt, kmax,
+                                        dense, softmax_scale, s);
+    return launch_attention<64, 4>(q, k, v, o, lse, B, H, Npad, valid_len, kv_idx, kv_cnt, kmax, dense,
+                                   softmax_scale, s);
+}
+
+sba_status sba_attention(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                         int H, int Npad, int D, const int32_t* valid_len, int block,
+                         const int32_t* kv_idx, const int32_t* kv_cnt, int kmax,
+                         float softmax_scale, void* stream) {
+    return attention_common(q, k, v, o, lse, B, H, Npad, D, valid_len, block, kv_idx, kv_cnt, kmax,
+                            0, softmax_scale, stream);
+}
+
+sba_status sba_dense_attention(const void* q, const void* k, const void* v, void* o, float* lse,
+                               int B, int H, int Npad, int D, const int32_t* valid_len,
+                               float softmax_scale, void* stream) {
+    return attention_common(q, k, v, o, lse, B, H, Npad, D, valid_len, 64, nullptr, nullptr, 0, 1,
+                            softmax_scale, stream);
+}
+
+sba_status sba_get_device_status(void* stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SBA_ERR_CUDA;
+    int word = 0;
+    const int zero = 0;
+    if (cudaMemcpyFromSymbol(&word, sba::g_device_error, sizeof(int)) != cudaSuccess) return SBA_ERR_CUDA;
+    if (cudaMemcpyToSymbol(sba::g_device_error, &zero, sizeof(int)) != cudaSuccess) return SBA_ERR_CUDA;
+    if (word == sba::kErrTimeout) return SBA_ERR_TIMEOUT;
+    if (word != 0) return SBA_ERR_DEVICE_FLAG;
+    return SBA_OK;
+}
+
+void sba_set_wait_limit(uint64_t cycles) { g_wait_limit = cycles ? cycles : kDefaultWaitLimit; }
+
+const char* sba_strerror(sba_status status) {
+    switch (status) {
+        case SBA_OK: return "ok";
+        case SBA_ERR_INVALID_ARG: return "invalid argument";
+        case SBA_ERR_UNSUPPORTED: return "unsupported shape or parameter";
+        case SBA_ERR_ALIGNMENT: return "misaligned device pointer";
+        case SBA_ERR_CUDA: return "CUDA call failed";
+        case SBA_ERR_TIMEOUT: return "a kernel wait gave up";
+        case SBA_ERR_DEVICE_FLAG: return "a kernel found an invalid routing entry";
+    }
+    return "unknown status";
+}
+
+}  // extern "C"

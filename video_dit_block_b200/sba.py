@@ -1,0 +1,184 @@
+"""Python binding of the C ABI in include/sba.h (argument marshalling only).
+
+Every function takes torch CUDA tensors, allocates outputs with torch (device
+memory and streams are PyTorch's job here), and calls the CUDA library through
+ctypes.  There is no fallback: if libsba.so is missing or a tensor is not on a
+CUDA device, the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from .build import LIB
+
+SBA_OK = 0
+_STATUS = {0: "SBA_OK", 1: "SBA_ERR_INVALID_ARG", 2: "SBA_ERR_UNSUPPORTED", 3: "SBA_ERR_ALIGNMENT",
+           4: "SBA_ERR_CUDA", 5: "SBA_ERR_TIMEOUT", 6: "SBA_ERR_DEVICE_FLAG"}
+MAX_NPAD = 262144
+BLOCK = 64
+
+
+class SbaError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {_STATUS.get(code, code)} ({_lib.sba_strerror(code).decode()})")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libsba.so; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB):
+            raise RuntimeError(f"CUDA library not built: {LIB} is missing "
+                               "(run `python -m video_dit_block_b200.build`)")
+        L = ctypes.CDLL(LIB)
+        vp, i32, f64, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_double, ctypes.c_float, ctypes.c_size_t
+        L.sba_keep_count.restype = ctypes.c_int32
+        L.sba_keep_count.argtypes = [ctypes.c_int32, f64]
+        L.sba_pool_select_workspace_size.restype = sz
+        L.sba_pool_select_workspace_size.argtypes = [i32, i32, i32, i32, i32]
+        L.sba_pool_select.restype = i32
+        L.sba_pool_select.argtypes = [vp, vp, i32, i32, i32, i32, vp, i32, f64, i32, vp, vp, vp, sz, vp]
+        L.sba_block_means.restype = i32
+        L.sba_block_means.argtypes = [vp, i32, i32, i32, i32, vp, i32, vp, vp]
+        L.sba_attention.restype = i32
+        L.sba_attention.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, i32, vp, vp, i32, f32, vp]
+        L.sba_dense_attention.restype = i32
+        L.sba_dense_attention.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, f32, vp]
+        L.sba_get_device_status.restype = i32
+        L.sba_get_device_status.argtypes = [vp]
+        L.sba_set_wait_limit.restype = None
+        L.sba_set_wait_limit.argtypes = [ctypes.c_uint64]
+        L.sba_strerror.restype = ctypes.c_char_p
+        L.sba_strerror.argtypes = [i32]
+        _lib = L
+    return _lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(code, what):
+    if code != SBA_OK:
+        raise SbaError(code, what)
+
+
+def _qkv(*ts):
+    for t in ts:
+        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.dim() == 4 and t.is_contiguous()):
+            raise ValueError("expected contiguous bf16 CUDA tensors [B, H, Npad, D]")
+    return ts[0].shape
+
+
+def _valid_len(valid_len, device):
+    if valid_len is None:
+        return None
+    if not (valid_len.is_cuda and valid_len.dtype == torch.int32 and valid_len.is_contiguous()):
+        raise ValueError("valid_len must be a contiguous int32 CUDA tensor [B]")
+    return valid_len
+
+
+def keep_count(n_blocks: int, sparsity: float) -> int:
+    return int(lib().sba_keep_count(int(n_blocks), float(sparsity)))
+
+
+def kmax_for(Npad: int, sparsity: float, block: int = BLOCK) -> int:
+    """Row capacity of kv_idx that every sample of padded length Npad fits in."""
+    return keep_count(Npad // block, sparsity)
+
+
+def workspace_size(B: int, H: int, Npad: int, D: int, block: int = BLOCK) -> int:
+    return int(lib().sba_pool_select_workspace_size(B, H, Npad, D, block))
+
+
+def pool_select(q, k, valid_len=None, sparsity: float = 0.0, kmax: int | None = None,
+                block: int = BLOCK, kv_idx=None, kv_cnt=None, workspace=None, stream=None):
+    """Routing: returns (kv_idx int32 [B,H,Npad/64,kmax], kv_cnt int32 [B,H,Npad/64])."""
+    B, H, Npad, D = _qkv(q, k)
+    vl = _valid_len(valid_len, q.device)
+    nB = Npad // block
+    if kmax is None:
+        kmax = kmax_for(Npad, sparsity, block)
+    if kv_idx is None:
+        kv_idx = torch.empty((B, H, nB, kmax), dtype=torch.int32, device=q.device)
+    if kv_cnt is None:
+        kv_cnt = torch.empty((B, H, nB), dtype=torch.int32, device=q.device)
+    wsz = workspace_size(B, H, Npad, D, block)
+    if workspace is None:
+        workspace = torch.empty(wsz, dtype=torch.uint8, device=q.device)
+    _check(lib().sba_pool_select(_ptr(q), _ptr(k), B, H, Npad, D, _ptr(vl), block, float(sparsity),
+                                 int(kmax), _ptr(kv_idx), _ptr(kv_cnt), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream(stream)),
+           "sba_pool_select")
+    return kv_idx, kv_cnt
+
+
+def block_means(x, valid_len=None, block: int = BLOCK, stream=None):
+    """fp64 block means [B, H, Npad/64, D]."""
+    B, H, Npad, D = _qkv(x)
+    out = torch.empty((B, H, Npad // block, D), dtype=torch.float64, device=x.device)
+    _check(lib().sba_block_means(_ptr(x), B, H, Npad, D, _ptr(_valid_len(valid_len, x.device)), block,
+                                 _ptr(out), _stream(stream)), "sba_block_means")
+    return out
+
+
+def attention(q, k, v, kv_idx, kv_cnt, valid_len=None, softmax_scale: float = 0.0, out=None,
+              lse=None, want_lse: bool = True, block: int = BLOCK, stream=None):
+    """Block-sparse attention under a routing.  Returns (o bf16, lse fp32 or None)."""
+    B, H, Npad, D = _qkv(q, k, v)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H, Npad), dtype=torch.float32, device=q.device)
+    if not (kv_idx.dtype == torch.int32 and kv_cnt.dtype == torch.int32 and kv_idx.is_contiguous()
+            and kv_cnt.is_contiguous() and kv_idx.is_cuda and kv_cnt.is_cuda):
+        raise ValueError("kv_idx / kv_cnt must be contiguous int32 CUDA tensors")
+    _check(lib().sba_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Npad, D,
+                               _ptr(_valid_len(valid_len, q.device)), block, _ptr(kv_idx),
+                               _ptr(kv_cnt), kv_idx.shape[-1], float(softmax_scale), _stream(stream)),
+           "sba_attention")
+    return out, lse
+
+
+def dense_attention(q, k, v, valid_len=None, softmax_scale: float = 0.0, out=None, lse=None,
+                    want_lse: bool = True, stream=None):
+    """Dense attention over each sample's valid tokens.  Returns (o bf16, lse fp32 or None)."""
+    B, H, Npad, D = _qkv(q, k, v)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H, Npad), dtype=torch.float32, device=q.device)
+    _check(lib().sba_dense_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Npad, D,
+                                     _ptr(_valid_len(valid_len, q.device)), float(softmax_scale),
+                                     _stream(stream)), "sba_dense_attention")
+    return out, lse
+
+
+def sparse_attention(q, k, v, valid_len=None, sparsity: float = 0.75, softmax_scale: float = 0.0,
+                     stream=None):
+    """The whole path: routing then block-sparse attention.  Returns (o, lse, kv_idx, kv_cnt)."""
+    kv_idx, kv_cnt = pool_select(q, k, valid_len, sparsity, stream=stream)
+    o, lse = attention(q, k, v, kv_idx, kv_cnt, valid_len, softmax_scale, stream=stream)
+    return o, lse, kv_idx, kv_cnt
+
+
+def device_status(stream=None) -> int:
+    """Synchronise the stream; return and clear the device-side error word (an SBA_* code)."""
+    return int(lib().sba_get_device_status(_stream(stream)))
+
+
+def set_wait_limit(cycles: int) -> None:
+    lib().sba_set_wait_limit(int(cycles))
