@@ -1,0 +1,357 @@
+#!/usr/bin/env python
+"""Benchmark of the block-sparse attention path on B200.
+
+One step = the whole path over one batch: sba_pool_select (pool, score, top-k) then
+sba_attention over the kept blocks.  Prints ONE JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+Metric: effective TFLOP/s on the kept blocks, counted as
+4 * D * sum_{b,h,I} c_I * sum_{J kept} c_J (c = valid tokens of a block), divided by
+the step time.  N > 1 runs one replica per GPU (every (b, h) is independent; there is
+no exchange inside the path), so scaling is weak and `value` sums all replicas.
+`--impl reference` times the fp64 CPU oracle on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "block-sparse attn effective TFLOP/s (kept blocks) and % of B200 bf16 peak"
+SPEC_BF16_TFLOPS = 2250.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", default="480p_dense")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kept_flops(kv_idx, kv_cnt, valid_len, D, block=64):
+    """4*D*sum_{b,h,I} c_I * sum_{J in kept(b,h,I)} c_J, exact for partial blocks."""
+    B, H, nQ, kmax = kv_idx.shape
+    total = 0
+    for b in range(B):
+        L = int(valid_len[b])
+        cI = np.clip(L - block * np.arange(nQ), 0, block).astype(np.int64)          # [nQ]
+        idx = kv_idx[b].astype(np.int64)                                               # [H,nQ,kmax]
+        live = np.arange(kmax)[None, None, :] < kv_cnt[b][:, :, None]
+        cJ = np.where(live, np.clip(L - block * idx, 0, block), 0)
+        total += int((cJ.sum(axis=2) * cI[None, :]).sum())
+    return 4 * D * total
+
+
+class ClockSampler:
+    """nvidia-smi every 200 ms while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=5)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def oracle_sample(w, target_s=10.0, seed=0):
+    """Time the fp64 oracle, as it stands, on a bounded sample of the workload: the
+    full routing of head (b=0, h=0) and the attention of a seeded subset of that head's
+    query blocks, sized to about `target_s` seconds.
+
+    Throughput: routing one head costs t_sel and serves that head's kept FLOPs f_head;
+    the sampled attention did f_sample kept FLOPs in t_attn.  So one kept FLOP costs
+    t_sel / f_head + t_attn / f_sample seconds of the oracle."""
+    import oracle
+    q1, k1, v1 = (np.ascontiguousarray(x[:1, :1]) for x in (w.q, w.k, w.v))
+    vl1 = np.ascontiguousarray(w.valid_len[:1])
+    t0 = time.perf_counter()
+    idx, cnt = oracle.select(q1, k1, vl1, w.sparsity)
+    t_sel = time.perf_counter() - t0
+    f_head = kept_flops(idx, cnt, vl1, w.D)
+    L = int(vl1[0])
+    nB0 = (L + 63) // 64
+    order = np.random.default_rng(seed).permutation(nB0).astype(np.int32)
+    t0 = time.perf_counter()
+    oracle.attention(q1, k1, v1, idx, cnt, vl1, qblocks=order[:1])
+    t_one = max(time.perf_counter() - t0, 1e-4)
+    n = int(max(1, min(nB0, target_s / t_one)))
+    t0 = time.perf_counter()
+    oracle.attention(q1, k1, v1, idx, cnt, vl1, qblocks=order[:n])
+    t_attn = time.perf_counter() - t0
+    sel = order[:n]
+    sub_cnt = np.zeros_like(cnt)
+    sub_cnt[:, :, sel] = cnt[:, :, sel]
+    f_sample = kept_flops(idx, sub_cnt, vl1, w.D) if n < nB0 else f_head
+    sec_per_flop = t_sel / f_head + t_attn / f_sample
+    return {"t_sel": t_sel, "t_attn": t_attn, "f_head": f_head, "f_sample": f_sample,
+            "n_qblocks": n, "value": 1.0 / sec_per_flop / 1e12}
+
+
+def cpu_baseline_from(sample, kind="oracle"):
+    return {"value": sample["value"], "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": kind,
+            "sample": (f"fp64 oracle on all host cores: routing of head (0,0) ({sample['t_sel']:.2f} s) "
+                       f"+ attention of {sample['n_qblocks']} seeded query blocks of that head "
+                       f"({sample['t_attn']:.2f} s); TFLOP/s = 1 / (t_route/F_head + t_attn/F_sample)")}
+
+
+def workload_config(w, extra=None):
+    c = {"workload": w.name, "B": w.B, "H": w.H, "D": w.D, "N": int(np.prod(w.grid)),
+         "Npad": w.Npad, "valid_len": [int(x) for x in w.valid_len], "block": 64,
+         "sparsity": w.sparsity, "grid_thw": list(w.grid), "parallelism": "replicas"}
+    c.update(extra or {})
+    return c
+
+
+def run_reference(args):
+    """The oracle as the reference arm, rank 0 only: every step is a bounded sample."""
+    from workloads import CONFIGS, make_workload
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    w = make_workload(args.config, heads=1)
+    per = []
+    target = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    for i in range(args.warmup + args.steps):
+        s = oracle_sample(w, target_s=target, seed=i)
+        if i >= args.warmup:
+            per.append(s)
+    value = statistics.mean(s["value"] for s in per)
+    t_step = statistics.mean(s["t_sel"] + s["t_attn"] for s in per)
+    cb = cpu_baseline_from(per[-1])
+    cb["value"] = value
+    cfg = workload_config(w, {"H": CONFIGS[args.config]["H"],
+                              "sample": "each step: oracle routing of head (0,0) + attention of a "
+                                        "seeded subset of its query blocks"})
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": t_step * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded smooth field + noise)",
+            "config": cfg, "cpu_baseline": cb,
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args):
+    import torch
+
+    import video_dit_block_b200 as sba
+    from workloads import make_workload
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+
+    w = make_workload(args.config)
+    t = lambda x: torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
+    q, k, v = t(w.q), t(w.k), t(w.v)
+    vl = torch.from_numpy(w.valid_len).to(dev)
+    B, H, Npad, D = q.shape
+    kmax = sba.kmax_for(Npad, w.sparsity)
+    kv_idx = torch.empty((B, H, Npad // 64, kmax), dtype=torch.int32, device=dev)
+    kv_cnt = torch.empty((B, H, Npad // 64), dtype=torch.int32, device=dev)
+    ws = torch.empty(sba.workspace_size(B, H, Npad, D), dtype=torch.uint8, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, Npad), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(qq=q, kk=k, vv=v):
+        sba.pool_select(qq, kk, vl, w.sparsity, kmax, kv_idx=kv_idx, kv_cnt=kv_cnt, workspace=ws,
+                        stream=stream)
+        sba.attention(qq, kk, vv, kv_idx, kv_cnt, vl, out=o, lse=lse, stream=stream)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    status = sba.device_status(stream)
+    if status != 0:
+        raise RuntimeError(f"device status {status} after warm-up")
+    f_step = kept_flops(kv_idx.cpu().numpy(), kv_cnt.cpu().numpy(), w.valid_len, D)
+
+    # ---- timed region: K steps, events on the launching stream
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    clocks = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    time.sleep(0.3)
+    for i in range(K):
+        ev[i][0].record(stream)
+        sba.pool_select(q, k, vl, w.sparsity, kmax, kv_idx=kv_idx, kv_cnt=kv_cnt, workspace=ws,
+                        stream=stream)
+        ev[i][1].record(stream)
+        sba.attention(q, k, v, kv_idx, kv_cnt, vl, out=o, lse=lse, stream=stream)
+        ev[i][2].record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    barrier()
+    total_ms = ev[0][0].elapsed_time(ev[-1][2])
+    sel_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    attn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    if sba.device_status(stream) != 0:
+        raise RuntimeError("device status error in the timed region")
+    vals = torch.tensor([total_ms, attn_ms, sel_ms], dtype=torch.float64, device=dev)
+    if dist is not None:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    total_ms, attn_ms, sel_ms = (float(x) for x in vals.cpu())
+    ms_step = total_ms / K
+    value = world * f_step / (ms_step * 1e-3) / 1e12
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        qh, kh, vh = (x.cpu().pin_memory() for x in (q, k, v))
+        vlh = vl.cpu().pin_memory()
+        oh = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        vld = torch.empty_like(vl)
+        Ke = max(2, K // 2)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(Ke):
+            qd.copy_(qh, non_blocking=True)
+            kd.copy_(kh, non_blocking=True)
+            vd.copy_(vh, non_blocking=True)
+            vld.copy_(vlh, non_blocking=True)
+            sba.pool_select(qd, kd, vld, w.sparsity, kmax, kv_idx=kv_idx, kv_cnt=kv_cnt, workspace=ws,
+                            stream=stream)
+            sba.attention(qd, kd, vd, kv_idx, kv_cnt, vld, out=o, lse=lse, stream=stream)
+            oh.copy_(o, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = torch.tensor([e0.elapsed_time(e1) / Ke], dtype=torch.float64, device=dev)
+        if dist is not None:
+            dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
+        e_ms = float(e_ms.item())
+        bi = 3 * q.numel() * 2 + vl.numel() * 4
+        e2e = {"value": world * f_step / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": e_ms, "h2d_bytes_per_step": bi, "d2h_bytes_per_step": o.numel() * 2}
+
+    if rank != 0:
+        if dist is not None:
+            dist.destroy_process_group()
+        return
+    peaks, src = load_peaks()
+    peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    achieved = f_step / (attn_ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded smooth field + noise, bf16; no weights involved)",
+        "config": workload_config(w, {
+            "l2": f"inputs {3 * q.numel() * 2 / 1e6:.0f} MB > 126 MB L2; no flush between steps",
+            "kmax": kmax}),
+        "pct_of_spec_bf16_peak": 100.0 * value / world / SPEC_BF16_TFLOPS,
+        "attn_ms": attn_ms, "select_ms": sel_ms, "kept_tflop_per_step": f_step / 1e12,
+        "roofline": {"bound": "tensor", "kernel": "attn_kernel<128,4>" if D == 128 else "attn_kernel<64,4>",
+                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_source": f"{src} bf16_tflops_sustained (kernel timed inside a seconds-long loop)",
+                     "traffic": None},
+        "gpu_launches": 4 * K,
+        "clocks": clk,
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_from(oracle_sample(w, target_s=15.0))
+    print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.warmup < 3:
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,115 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function declared
+in include/sba.h, and rejects bad arguments on the host before touching device memory."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sba.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from video_dit_block_b200 import build
+    build.build()
+    import video_dit_block_b200 as sba
+    return sba.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sba_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_path():
+    names = declared_functions()
+    for n in ("sba_pool_select", "sba_attention", "sba_dense_attention", "sba_keep_count",
+              "sba_get_device_status", "sba_strerror"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+@pytest.mark.parametrize("n", [1, 2, 3, 7, 10, 16, 100, 512, 841, 1182, 4096])
+@pytest.mark.parametrize("s", [0.0, 0.1, 0.3, 0.5, 0.7, 0.75, 0.8, 0.9, 0.95, 0.999])
+def test_keep_count_matches_oracle(lib, oracle_mod, n, s):
+    assert lib.sba_keep_count(n, s) == oracle_mod.keep_count(n, s)
+
+
+def test_strerror(lib):
+    for code in range(7):
+        assert lib.sba_strerror(code)
+    assert lib.sba_strerror(99) == b"unknown status"
+
+
+def test_workspace_size(lib):
+    assert lib.sba_pool_select_workspace_size(1, 24, 32768, 128, 64) > 0
+    assert lib.sba_pool_select_workspace_size(1, 24, 32768, 96, 64) == 0
+    assert lib.sba_pool_select_workspace_size(1, 24, 32760, 128, 64) == 0
+
+
+# Fake device pointers: every call below must fail validation before any CUDA call.
+A = ctypes.c_void_p(0x10000)       # 16-byte aligned
+MIS = ctypes.c_void_p(0x10008)     # 8-byte aligned only
+NULL = None
+S = None                           # stream
+
+
+def pool_select(lib, q=A, k=A, B=1, H=2, Npad=1024, D=64, vl=NULL, block=64, s=0.5, kmax=8,
+                idx=A, cnt=A, ws=A, wsb=1 << 30):
+    return lib.sba_pool_select(q, k, B, H, Npad, D, vl, block, s, kmax, idx, cnt, ws, wsb, S)
+
+
+def attention(lib, q=A, k=A, v=A, o=A, lse=A, B=1, H=2, Npad=1024, D=64, vl=NULL, block=64,
+              idx=A, cnt=A, kmax=8, scale=0.0):
+    return lib.sba_attention(q, k, v, o, lse, B, H, Npad, D, vl, block, idx, cnt, kmax, scale, S)
+
+
+@pytest.mark.parametrize("kwargs,code", [
+    (dict(q=NULL), 1), (dict(k=NULL), 1), (dict(idx=NULL), 1), (dict(cnt=NULL), 1), (dict(ws=NULL), 1),
+    (dict(B=0), 1), (dict(H=-1), 1), (dict(Npad=1000), 1), (dict(D=96), 2), (dict(block=32), 2),
+    (dict(Npad=262144 + 64), 2), (dict(s=1.0), 1), (dict(s=-0.1), 1), (dict(s=float("nan")), 1),
+    (dict(kmax=7), 1), (dict(wsb=16), 1), (dict(q=MIS), 3), (dict(vl=MIS), 3), (dict(ws=MIS), 3),
+])
+def test_pool_select_rejects(lib, kwargs, code):
+    assert pool_select(lib, **kwargs) == code
+
+
+@pytest.mark.parametrize("kwargs,code", [
+    (dict(q=NULL), 1), (dict(v=NULL), 1), (dict(o=NULL), 1), (dict(idx=NULL), 1), (dict(cnt=NULL), 1),
+    (dict(kmax=0), 1), (dict(D=32), 2), (dict(block=128), 2), (dict(Npad=100), 1),
+    (dict(scale=float("inf")), 1), (dict(scale=float("nan")), 1), (dict(o=MIS), 3),
+    (dict(lse=ctypes.c_void_p(0x10002)), 3), (dict(idx=ctypes.c_void_p(0x10002)), 3),
+])
+def test_attention_rejects(lib, kwargs, code):
+    assert attention(lib, **kwargs) == code
+
+
+def test_dense_attention_rejects(lib):
+    assert lib.sba_dense_attention(A, A, NULL, A, A, 1, 2, 1024, 64, NULL, 0.0, S) == 1
+    assert lib.sba_dense_attention(A, A, A, A, A, 1, 2, 1024, 80, NULL, 0.0, S) == 2
+    assert lib.sba_dense_attention(MIS, A, A, A, A, 1, 2, 1024, 64, NULL, 0.0, S) == 3
+
+
+def test_block_means_rejects(lib):
+    assert lib.sba_block_means(NULL, 1, 2, 1024, 64, NULL, 64, A, S) == 1
+    assert lib.sba_block_means(A, 1, 2, 1024, 64, NULL, 64, MIS, S) == 3
+    assert lib.sba_block_means(A, 1, 2, 1024, 48, NULL, 64, A, S) == 2
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+
+    import video_dit_block_b200 as sba
+    x = torch.zeros((1, 1, 64, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        sba.dense_attention(x, x, x)
+    with pytest.raises(ValueError):
+        sba.pool_select(x, x, None, 0.5)

@@ -68,7 +68,12 @@ struct AttnSmem {
     static constexpr int kAlloc = kTotal + 1024;            // slack for 1024-byte alignment
 };
 
-__device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, uint64_t limit) {
+// Drains after an abort wait for work that always completes on its own (this CTA's
+// TMA copies and MMAs), so their limit is fixed and generous, independent of the
+// wait limit the caller set.
+constexpr uint64_t kDrainLimit = 1ull << 32;
+
+__device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, uint64_t limit = kDrainLimit) {
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity)) {
         if ((uint64_t)(clock64() - t0) > limit) return false;
@@ -192,6 +197,7 @@ __global__ void __launch_bounds__(192, 1)
     const uint32_t tmem = ctl[0];
     const int n = static_cast<int>(ctl[2]);
     const uint64_t lim = p.wait_limit;
+    int issued = 0;  // K/V blocks whose loads the producer has issued
 
     if (warp == 4) {
         // ------------------------------------------------------------ TMA producer
@@ -202,7 +208,6 @@ __global__ void __launch_bounds__(192, 1)
             mbar_arrive_expect_tx(bar_q, SM::kQBytes);
             for (int c = 0; c < NCH; ++c)
                 tma_load_3d(sQ + c * (128 * 128), &tmQ, bar_q, c * 64, I0 * 64, bh);
-            int issued = 0;
             for (int j = 0; j < n; ++j) {
                 const int st = j % NS;
                 if (j >= NS && !wait_bounded(bar_ke(st), ((j / NS) - 1) & 1, abort_flag, lim)) break;
@@ -216,14 +221,6 @@ __global__ void __launch_bounds__(192, 1)
                     tma_load_3d(sV + st * SM::kKVBytes + c * (64 * 128), &tmV, bar_vf(st), c * 64,
                                 J * 64, bh);
                 issued = j + 1;
-            }
-            if (*abort_flag) {
-                // let this CTA's own copies land before the CTA exits
-                wait_drain(bar_q, 0, lim);
-                for (int j = issued > NS ? issued - NS : 0; j < issued; ++j) {
-                    wait_drain(bar_kf(j % NS), (j / NS) & 1, lim);
-                    wait_drain(bar_vf(j % NS), (j / NS) & 1, lim);
-                }
             }
         }
     } else if (warp == 5) {
@@ -261,11 +258,6 @@ __global__ void __launch_bounds__(192, 1)
                     mma_commit(bar_pv(jj & 1));
                     mma_commit(bar_ke(st));
                 }
-            }
-            if (!ok) {
-                // every MMA this thread issued must finish before TMEM is freed
-                mma_commit(bar_drain);
-                wait_drain(bar_drain, 0, lim);
             }
         }
     } else {
@@ -391,6 +383,22 @@ __global__ void __launch_bounds__(192, 1)
     // ---------------------------------------------------------------- teardown
     tc_fence_before();
     __syncthreads();
+    if (*abort_flag) {
+        // An aborted CTA still lets its own TMA copies land and its MMAs finish
+        // before it frees TMEM and exits.
+        if (warp == 4 && lane == 0 && n > 0) {
+            wait_drain(bar_q, 0);
+            for (int j = issued > NS ? issued - NS : 0; j < issued; ++j) {
+                wait_drain(bar_kf(j % NS), (j / NS) & 1);
+                wait_drain(bar_vf(j % NS), (j / NS) & 1);
+            }
+        }
+        if (warp == 5 && lane == 0) {
+            mma_commit(bar_drain);
+            wait_drain(bar_drain, 0);
+        }
+        __syncthreads();
+    }
     if (warp == 5) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);

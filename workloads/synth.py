@@ -25,8 +25,10 @@ Nothing here computes any part of the attention method.
 """
 from __future__ import annotations
 
+import concurrent.futures
 import dataclasses
 import math
+import os
 
 import numpy as np
 
@@ -88,25 +90,18 @@ class Workload:
 def f64_to_bf16_bits(x: np.ndarray) -> np.ndarray:
     """Round float64 values to bf16 with round-to-nearest-even, directly from the
     binary64 encoding (no intermediate float32 rounding).  Normal-range values only."""
-    x = np.ascontiguousarray(x, dtype=np.float64)
-    b = x.view(np.uint64)
+    b = np.ascontiguousarray(x, dtype=np.float64).view(np.uint64)
+    keep = b >> np.uint64(45)                       # sign | 11-bit exponent | 7 mantissa bits
     low = b & np.uint64((1 << 45) - 1)
-    keep = b >> np.uint64(45)
     half = np.uint64(1 << 44)
-    up = (low > half) | ((low == half) & ((keep & np.uint64(1)) == np.uint64(1)))
-    keep = keep + up.astype(np.uint64)
-    sign = (keep >> np.uint64(18)) & np.uint64(1)
-    exp = ((keep >> np.uint64(7)) & np.uint64(0x7FF)).astype(np.int64)
-    mant = keep & np.uint64(0x7F)
-    zero = (b & np.uint64(0x7FFFFFFFFFFFFFFF)) == np.uint64(0)
-    e16 = exp - 1023 + 127
-    bad = (~zero) & ((e16 < 1) | (e16 > 254))
-    if np.any(bad):
+    keep += (low > half) | ((low == half) & (keep & np.uint64(1)).astype(bool))
+    # re-bias the exponent (1023 -> 127) in the combined exponent|mantissa field
+    em = (keep & np.uint64(0x3FFFF)).astype(np.int64) - ((1023 - 127) << 7)
+    zero = (b << np.uint64(1)) == np.uint64(0)
+    if np.any(~zero & ((em < (1 << 7)) | (em > (254 << 7) + 127))):
         raise ValueError("value outside the bf16 normal range")
-    e16 = np.where(zero, 0, e16).astype(np.uint64)
-    mant = np.where(zero, np.uint64(0), mant)
-    out = (sign << np.uint64(15)) | (e16 << np.uint64(7)) | mant
-    return out.astype(np.uint16)
+    em[zero] = 0
+    return (((keep >> np.uint64(18)) << np.uint64(15)) | em.astype(np.uint64)).astype(np.uint16)
 
 
 def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
@@ -153,22 +148,25 @@ def _build(name, B, H, D, grid, sparsity, sigma, per_head_freq, drop_rate, seed,
     valid_len = np.array([len(r) for r in keep_rows], dtype=np.int32)
     Npad = BLOCK * int(math.ceil(valid_len.max() / BLOCK))
     pad_bits = f64_to_bf16_bits(np.array([pad_value]))[0]
-    out = {}
-    for ti, tname in enumerate(TENSORS):
-        arr = np.full((B, len(hsel), Npad, D), pad_bits, dtype=np.uint16)
-        for b in range(B):
-            shared = None
-            if not per_head_freq:
-                shared = _rng(seed, 1, ti, b).uniform(0.0, 3.0, size=(D, 8, 3))
-            for hi, h in enumerate(hsel):
-                fr = shared if shared is not None else \
-                    _rng(seed, 2, ti, b, h).uniform(0.0, 3.0, size=(D, 8, 3))
-                ph = _rng(seed, 3, ti, b, h).uniform(0.0, 2 * np.pi, size=(D, 8))
-                eps = _rng(seed, 4, ti, b, h).standard_normal((N, D), dtype=np.float32)
-                x = _field(grid, fr, ph) + sigma * eps.astype(np.float64)
-                rows = keep_rows[b]
-                arr[b, hi, :len(rows)] = f64_to_bf16_bits(x[rows])
-        out[tname] = arr
+    out = {t: np.full((B, len(hsel), Npad, D), pad_bits, dtype=np.uint16) for t in TENSORS}
+
+    def one(job):
+        ti, b, hi, h = job
+        if per_head_freq:
+            fr = _rng(seed, 2, ti, b, h).uniform(0.0, 3.0, size=(D, 8, 3))
+        else:
+            fr = _rng(seed, 1, ti, b).uniform(0.0, 3.0, size=(D, 8, 3))
+        ph = _rng(seed, 3, ti, b, h).uniform(0.0, 2 * np.pi, size=(D, 8))
+        eps = _rng(seed, 4, ti, b, h).standard_normal((N, D), dtype=np.float32)
+        x = _field(grid, fr, ph) + sigma * eps.astype(np.float64)
+        rows = keep_rows[b]
+        out[TENSORS[ti]][b, hi, :len(rows)] = f64_to_bf16_bits(x[rows])
+
+    jobs = [(ti, b, hi, h) for ti in range(3) for b in range(B) for hi, h in enumerate(hsel)]
+    # numpy releases the GIL in the heavy kernels: threads give real parallelism, and
+    # every job owns its own generators, so the result does not depend on scheduling.
+    with concurrent.futures.ThreadPoolExecutor(max_workers=min(len(jobs), os.cpu_count() or 1)) as ex:
+        list(ex.map(one, jobs))
     return Workload(name=name, q=out["q"], k=out["k"], v=out["v"], valid_len=valid_len,
                     sparsity=float(sparsity), grid=tuple(grid), seed=seed)
 
