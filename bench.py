@@ -327,7 +327,7 @@ def run_ours(args):
             "kmax": kmax}),
         "pct_of_spec_bf16_peak": 100.0 * value / world / SPEC_BF16_TFLOPS,
         "attn_ms": attn_ms, "select_ms": sel_ms, "kept_tflop_per_step": f_step / 1e12,
-        "roofline": {"bound": "tensor", "kernel": "attn_kernel<128,4>" if D == 128 else "attn_kernel<64,4>",
+        "roofline": {"bound": "tensor", "kernel": "attn_kernel<128,2>" if D == 128 else "attn_kernel<64,4>",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_source": f"{src} bf16_tflops_sustained (kernel timed inside a seconds-long loop)",
                      "traffic": None},

@@ -52,12 +52,10 @@ template <int D, int NS>
 struct AttnSmem {
     static constexpr int kQBytes = 128 * D * 2;
     static constexpr int kKVBytes = 64 * D * 2;
-    static constexpr int kPBytes = 128 * 64 * 2;
     static constexpr int kQ = 0;
     static constexpr int kK = kQ + kQBytes;
     static constexpr int kV = kK + NS * kKVBytes;
-    static constexpr int kP = kV + NS * kKVBytes;
-    static constexpr int kBars = kP + 2 * kPBytes;
+    static constexpr int kBars = kV + NS * kKVBytes;
     // barriers: q_full, k_full[NS], v_full[NS], kv_empty[NS], s_full[2], p_full[2],
     //           pv_done[2], drain
     static constexpr int kNumBars = 1 + 3 * NS + 7;
@@ -82,7 +80,7 @@ __device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, uint64
 }
 
 template <int D, int NS>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(192, 2)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
     using SM = AttnSmem<D, NS>;
@@ -97,8 +95,6 @@ __global__ void __launch_bounds__(192, 1)
     const uint32_t sQ = smem_u32(sm + SM::kQ);
     const uint32_t sK = smem_u32(sm + SM::kK);
     const uint32_t sV = smem_u32(sm + SM::kV);
-    const uint32_t sP = smem_u32(sm + SM::kP);
-    unsigned char* sPg = sm + SM::kP;
     const uint32_t bars = smem_u32(sm + SM::kBars);
     const uint32_t bar_q = bars;
     auto bar_kf = [&](int s) { return bars + 8u * (1 + s); };
@@ -250,10 +246,10 @@ __global__ void __launch_bounds__(192, 1)
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
-                        const uint64_t a = smem_desc_sw128(sP + (jj & 1) * SM::kPBytes + kk * 32, 16, 1024);
                         const uint64_t bd = smem_desc_sw128(sV + st * SM::kKVBytes + kk * (16 * 128),
                                                             64 * 128, 1024);
-                        mma_bf16_ss(tmem + 128, a, bd, kIdescPV, (jj > 0 || kk > 0) ? 1u : 0u);
+                        mma_bf16_ts(tmem + 128, tmem + (jj & 1) * 64 + kk * 8, bd, kIdescPV,
+                                    (jj > 0 || kk > 0) ? 1u : 0u);
                     }
                     mma_commit(bar_pv(jj & 1));
                     mma_commit(bar_ke(st));
@@ -277,25 +273,35 @@ __global__ void __launch_bounds__(192, 1)
             ncol = ncol > 64 ? 64 : ncol;
             if (!warp_wait_bounded(bar_sf(j & 1), (j >> 1) & 1, abort_flag, lim)) { ok = false; break; }
             tc_fence_after();
+            const uint32_t sbuf = tl + (j & 1) * 64;
             float x[64];
             {
                 uint32_t a[32], c[32];
-                tmem_ld32(tl + (j & 1) * 64, a);
-                tmem_ld32(tl + (j & 1) * 64 + 32, c);
+                tmem_ld32(sbuf, a);
+                tmem_ld32(sbuf + 32, c);
                 tmem_wait_ld();
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    x[i] = i < ncol ? __uint_as_float(a[i]) * sc : -INFINITY;
-                    x[32 + i] = 32 + i < ncol ? __uint_as_float(c[i]) * sc : -INFINITY;
+                    x[i] = __uint_as_float(a[i]);
+                    x[32 + i] = __uint_as_float(c[i]);
                 }
             }
-            float mloc = -INFINITY;
+            if (ncol < 64) {  // key block not kept by this row's query block, or ragged tail
 #pragma unroll
-            for (int i = 0; i < 64; ++i) mloc = fmaxf(mloc, x[i]);
-            const float m_new = fmaxf(m, mloc);
+                for (int i = 0; i < 64; ++i) x[i] = i < ncol ? x[i] : -INFINITY;
+            }
+            float mx0 = x[0], mx1 = x[1], mx2 = x[2], mx3 = x[3];
+#pragma unroll
+            for (int i = 4; i < 64; i += 4) {
+                mx0 = fmaxf(mx0, x[i]);
+                mx1 = fmaxf(mx1, x[i + 1]);
+                mx2 = fmaxf(mx2, x[i + 2]);
+                mx3 = fmaxf(mx3, x[i + 3]);
+            }
+            const float m_new = fmaxf(m, fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sc);
             const bool grow = m_new > m + 8.f;
             if (j > 0 && __any_sync(0xffffffffu, grow)) {
-                // O accumulates P V with the running max; move it and rescale O, l.
+                // O holds sum P V with the old running max: move the max, rescale O and l.
                 if (!warp_wait_bounded(bar_pv((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag, lim)) {
                     ok = false;
                     break;
@@ -311,35 +317,27 @@ __global__ void __launch_bounds__(192, 1)
                     for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
                     tmem_st32(tl + 128 + ch * 32, o);
                 }
-                tmem_wait_st();
                 l *= alpha;
                 m = m_new;
             } else if (grow || j == 0) {
                 m = m_new;
             }
-            const float mref = (m == -INFINITY) ? 0.f : m;
-            float rs = 0.f;
+            // p = 2^(s * scale * log2e - m), packed to bf16 pairs over the S columns just read
+            const float nm = (m == -INFINITY) ? 0.f : -m;
+            float rs0 = 0.f, rs1 = 0.f;
             uint32_t pk[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-                const float p0 = ex2_approx(x[2 * i] - mref);
-                const float p1 = ex2_approx(x[2 * i + 1] - mref);
-                rs += p0 + p1;
+                const float p0 = ex2_approx(fmaf(x[2 * i], sc, nm));
+                const float p1 = ex2_approx(fmaf(x[2 * i + 1], sc, nm));
+                rs0 += p0;
+                rs1 += p1;
                 __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
                 pk[i] = *reinterpret_cast<uint32_t*>(&h2);
             }
-            l += rs;
-            // P buffer j%2 is free once PV(j-2) has completed
-            if (j >= 2 && !warp_wait_bounded(bar_pv(j & 1), ((j - 2) >> 1) & 1, abort_flag, lim)) {
-                ok = false;
-                break;
-            }
-            unsigned char* prow = sPg + (j & 1) * SM::kPBytes + r * 128;
-#pragma unroll
-            for (int c16 = 0; c16 < 8; ++c16)
-                *reinterpret_cast<uint4*>(prow + ((c16 ^ (r & 7)) << 4)) =
-                    make_uint4(pk[4 * c16], pk[4 * c16 + 1], pk[4 * c16 + 2], pk[4 * c16 + 3]);
-            fence_proxy_async_smem();
+            l += rs0 + rs1;
+            tmem_st32(sbuf, pk);
+            tmem_wait_st();
             tc_fence_before();
             mbar_arrive(bar_pf(j & 1));
         }

@@ -196,7 +196,7 @@ static sba_status attention_common(const void* q, const void* k, const void* v, 
         return SBA_ERR_ALIGNMENT;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (D == 128)
-        return launch_attention<128, 4>(q, k, v, o, lse, B, H, Npad, valid_len, kv_idx, kv_cnt, kmax,
+        return launch_attention<128, 2>(q, k, v, o, lse, B, H, Npad, valid_len, kv_idx, kv_cnt, kmax,
                                         dense, softmax_scale, s);
     return launch_attention<64, 4>(q, k, v, o, lse, B, H, Npad, valid_len, kv_idx, kv_cnt, kmax, dense,
                                    softmax_scale, s);
