@@ -56,9 +56,9 @@ struct AttnSmem {
     static constexpr int kK = kQ + kQBytes;
     static constexpr int kV = kK + NS * kKVBytes;
     static constexpr int kBars = kV + NS * kKVBytes;
-    // barriers: q_full, k_full[NS], v_full[NS], kv_empty[NS], s_full[2], p_full[2],
-    //           pv_done[2], drain
-    static constexpr int kNumBars = 1 + 3 * NS + 7;
+    // barriers: q_full, k_full[NS], v_full[NS], k_empty[NS], v_empty[NS], s_full[2],
+    //           p_full[2], pv_done[2], drain
+    static constexpr int kNumBars = 1 + 4 * NS + 7;
     static constexpr int kCtl = kBars + kNumBars * 8;      // tmem base, abort, n_union, pad
     static constexpr int kBitmap = kCtl + 16;              // uint32 [2][kMaxBlocks/32]
     static constexpr int kList = kBitmap + 2 * (kMaxBlocks / 32) * 4;  // uint16 [kMaxBlocks]
@@ -100,10 +100,11 @@ __global__ void __launch_bounds__(192, 2)
     auto bar_kf = [&](int s) { return bars + 8u * (1 + s); };
     auto bar_vf = [&](int s) { return bars + 8u * (1 + NS + s); };
     auto bar_ke = [&](int s) { return bars + 8u * (1 + 2 * NS + s); };
-    auto bar_sf = [&](int s) { return bars + 8u * (1 + 3 * NS + s); };
-    auto bar_pf = [&](int s) { return bars + 8u * (3 + 3 * NS + s); };
-    auto bar_pv = [&](int s) { return bars + 8u * (5 + 3 * NS + s); };
-    const uint32_t bar_drain = bars + 8u * (7 + 3 * NS);
+    auto bar_ve = [&](int s) { return bars + 8u * (1 + 3 * NS + s); };
+    auto bar_sf = [&](int s) { return bars + 8u * (1 + 4 * NS + s); };
+    auto bar_pf = [&](int s) { return bars + 8u * (3 + 4 * NS + s); };
+    auto bar_pv = [&](int s) { return bars + 8u * (5 + 4 * NS + s); };
+    const uint32_t bar_drain = bars + 8u * (7 + 4 * NS);
     uint32_t* ctl = reinterpret_cast<uint32_t*>(sm + SM::kCtl);
     volatile uint32_t* abort_flag = ctl + 1;
     uint32_t* bm = reinterpret_cast<uint32_t*>(sm + SM::kBitmap);
@@ -124,6 +125,7 @@ __global__ void __launch_bounds__(192, 2)
             mbar_init(bar_kf(s), 1);
             mbar_init(bar_vf(s), 1);
             mbar_init(bar_ke(s), 1);
+            mbar_init(bar_ve(s), 1);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(bar_sf(s), 1);
@@ -193,7 +195,7 @@ __global__ void __launch_bounds__(192, 2)
     const uint32_t tmem = ctl[0];
     const int n = static_cast<int>(ctl[2]);
     const uint64_t lim = p.wait_limit;
-    int issued = 0;  // K/V blocks whose loads the producer has issued
+    int issued_k = 0, issued_v = 0;  // K / V blocks whose loads the producer has issued
 
     if (warp == 4) {
         // ------------------------------------------------------------ TMA producer
@@ -204,19 +206,29 @@ __global__ void __launch_bounds__(192, 2)
             mbar_arrive_expect_tx(bar_q, SM::kQBytes);
             for (int c = 0; c < NCH; ++c)
                 tma_load_3d(sQ + c * (128 * 128), &tmQ, bar_q, c * 64, I0 * 64, bh);
-            for (int j = 0; j < n; ++j) {
-                const int st = j % NS;
-                if (j >= NS && !wait_bounded(bar_ke(st), ((j / NS) - 1) & 1, abort_flag, lim)) break;
-                const int J = ulist[j];
-                mbar_arrive_expect_tx(bar_kf(st), SM::kKVBytes);
-                for (int c = 0; c < NCH; ++c)
-                    tma_load_3d(sK + st * SM::kKVBytes + c * (64 * 128), &tmK, bar_kf(st), c * 64,
-                                J * 64, bh);
-                mbar_arrive_expect_tx(bar_vf(st), SM::kKVBytes);
-                for (int c = 0; c < NCH; ++c)
-                    tma_load_3d(sV + st * SM::kKVBytes + c * (64 * 128), &tmV, bar_vf(st), c * 64,
-                                J * 64, bh);
-                issued = j + 1;
+            // K runs one block ahead of V: K(j) is released as soon as S(j) is done,
+            // V(j) only after PV(j).  Issue order K0, K1, V0, K2, V1, ...
+            for (int j = 0; j <= n; ++j) {
+                if (j < n) {
+                    const int st = j % NS;
+                    if (j >= NS && !wait_bounded(bar_ke(st), ((j / NS) - 1) & 1, abort_flag, lim)) break;
+                    const int J = ulist[j];
+                    mbar_arrive_expect_tx(bar_kf(st), SM::kKVBytes);
+                    for (int c = 0; c < NCH; ++c)
+                        tma_load_3d(sK + st * SM::kKVBytes + c * (64 * 128), &tmK, bar_kf(st), c * 64,
+                                    J * 64, bh);
+                    issued_k = j + 1;
+                }
+                if (j >= 1) {
+                    const int jv = j - 1, st = jv % NS;
+                    if (jv >= NS && !wait_bounded(bar_ve(st), ((jv / NS) - 1) & 1, abort_flag, lim)) break;
+                    const int J = ulist[jv];
+                    mbar_arrive_expect_tx(bar_vf(st), SM::kKVBytes);
+                    for (int c = 0; c < NCH; ++c)
+                        tma_load_3d(sV + st * SM::kKVBytes + c * (64 * 128), &tmV, bar_vf(st), c * 64,
+                                    J * 64, bh);
+                    issued_v = jv + 1;
+                }
             }
         }
     } else if (warp == 5) {
@@ -238,6 +250,7 @@ __global__ void __launch_bounds__(192, 2)
                         mma_bf16_ss(dS, a, bd, kIdescS, kk > 0 ? 1u : 0u);
                     }
                     mma_commit(bar_sf(j & 1));
+                    mma_commit(bar_ke(st));
                 }
                 if (j >= 1) {
                     const int jj = j - 1, st = jj % NS;
@@ -252,7 +265,7 @@ __global__ void __launch_bounds__(192, 2)
                                     (jj > 0 || kk > 0) ? 1u : 0u);
                     }
                     mma_commit(bar_pv(jj & 1));
-                    mma_commit(bar_ke(st));
+                    mma_commit(bar_ve(st));
                 }
             }
         }
@@ -386,10 +399,10 @@ __global__ void __launch_bounds__(192, 2)
         // before it frees TMEM and exits.
         if (warp == 4 && lane == 0 && n > 0) {
             wait_drain(bar_q, 0);
-            for (int j = issued > NS ? issued - NS : 0; j < issued; ++j) {
+            for (int j = issued_k > NS ? issued_k - NS : 0; j < issued_k; ++j)
                 wait_drain(bar_kf(j % NS), (j / NS) & 1);
+            for (int j = issued_v > NS ? issued_v - NS : 0; j < issued_v; ++j)
                 wait_drain(bar_vf(j % NS), (j / NS) & 1);
-            }
         }
         if (warp == 5 && lane == 0) {
             mma_commit(bar_drain);
