@@ -21,9 +21,9 @@
  *   - q, k, v, o: bf16, [B, H, Npad, D] contiguous row-major, device memory,
  *     base addresses 16-byte aligned.  D is 64 or 128.  Npad % block == 0.
  *   - valid_len: device int32 [B] with 1 <= valid_len[b] <= Npad, or NULL
- *     (every sample is Npad long).  Rows n >= valid_len[b] are padding: they are
- *     never read as keys or values, and their outputs are written as 0 (o) and
- *     -inf (lse).  nB_b = ceil(valid_len[b] / block).
+ *     (every sample is Npad long).  Rows n >= valid_len[b] are padding: as keys
+ *     and values they get zero weight (their contents must be finite), and their
+ *     outputs are written as 0 (o) and -inf (lse).  nB_b = ceil(valid_len[b] / block).
  *   - block must be 64.
  *   - Routing: kv_idx int32 [B, H, Npad/block, kmax] and kv_cnt int32
  *     [B, H, Npad/block]; row (b, h, I) lists kv_cnt key-block indices in
@@ -32,8 +32,9 @@
  *   - stream: a cudaStream_t (NULL = legacy default stream).  Every call is
  *     asynchronous on that stream; the library never synchronises except in
  *     sba_get_device_status.
+ *   - Inputs must be finite.
  *   - Ownership: the caller allocates and frees every buffer passed in.  The
- *     library keeps only a small per-device cache of TMA tensor descriptors.
+ *     library's only device state is one error word per device.
  *   - Errors: argument checks run on the host before any launch and return an
  *     sba_status without touching device memory.  A failed launch returns
  *     SBA_ERR_CUDA.  Faults detected inside a kernel (a wait that gave up, a

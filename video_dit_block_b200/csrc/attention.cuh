@@ -10,13 +10,19 @@
 // It walks the ascending union of the two kept lists; a key block kept by only
 // one of the two is masked to -inf for the other half's rows.
 //
-// Warp roles (192 threads):
-//   warps 0-3  softmax + epilogue; thread t owns query row t = TMEM lane t
-//   warp 4     builds the union list, then issues TMA loads (Q once, K/V per block)
-//   warp 5     allocates TMEM and issues the MMAs (one elected lane)
+// Warp roles (192 threads; two CTAs share an SM, so one CTA's MMAs run while the
+// other's softmax warps work):
+//   warps 0-3  softmax + epilogue; thread t owns query row t = TMEM lane t.  Warps
+//              0-1 serve query block I0, warps 2-3 query block I1, so "this key
+//              block is kept" is uniform over a warp and unkept blocks cost no
+//              exponentials (the warp writes P = 0)
+//   warp 4     builds the union list, then issues TMA loads: Q once, then K and V
+//              per key block in two rings; K(j) is freed when S(j) is done and V(j)
+//              when PV(j) is, and K is issued one block ahead of V
+//   warp 5     allocates TMEM (256 columns) and issues the MMAs (one elected lane)
 // Per key block j:  S_j = Q K_j^T  (M=128, N=64, K=D) into TMEM buffer j%2;
-//                   softmax reads S_j, writes P_j (bf16) to shared memory;
-//                   O += P_j V_j (M=128, N=D, K=64) into the TMEM accumulator.
+//                   softmax reads S_j and writes P_j (bf16) back over it;
+//                   O += P_j V_j (M=128, N=D, K=64), P read from TMEM.
 // The MMA warp issues S_{j+1} before PV_j so the tensor core works on the next
 // scores while the softmax warps exponentiate.  The running max is only moved
 // when it grows by more than 8 (log2 units); O is then rescaled in TMEM.
@@ -281,12 +287,23 @@ __global__ void __launch_bounds__(192, 2)
         bool ok = true;
         for (int j = 0; j < n; ++j) {
             const int J = ulist[j];
-            const bool kept = (bmh[J >> 5] >> (J & 31)) & 1u;
+            const bool kept = (bmh[J >> 5] >> (J & 31)) & 1u;  // uniform over the warp
             int ncol = kept ? L - J * 64 : 0;
             ncol = ncol > 64 ? 64 : ncol;
             if (!warp_wait_bounded(bar_sf(j & 1), (j >> 1) & 1, abort_flag, lim)) { ok = false; break; }
             tc_fence_after();
             const uint32_t sbuf = tl + (j & 1) * 64;
+            if (!kept) {
+                // the other query block of the tile keeps this key block: P = 0 for these rows
+                uint32_t z[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) z[i] = 0u;
+                tmem_st32(sbuf, z);
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar_pf(j & 1));
+                continue;
+            }
             float x[64];
             {
                 uint32_t a[32], c[32];
@@ -299,19 +316,18 @@ __global__ void __launch_bounds__(192, 2)
                     x[32 + i] = __uint_as_float(c[i]);
                 }
             }
-            if (ncol < 64) {  // key block not kept by this row's query block, or ragged tail
+            if (ncol < 64) {  // ragged tail block of the sample
 #pragma unroll
                 for (int i = 0; i < 64; ++i) x[i] = i < ncol ? x[i] : -INFINITY;
             }
-            float mx0 = x[0], mx1 = x[1], mx2 = x[2], mx3 = x[3];
+            float mx0 = x[0], mx1 = x[1];
 #pragma unroll
-            for (int i = 4; i < 64; i += 4) {
-                mx0 = fmaxf(mx0, x[i]);
-                mx1 = fmaxf(mx1, x[i + 1]);
-                mx2 = fmaxf(mx2, x[i + 2]);
-                mx3 = fmaxf(mx3, x[i + 3]);
+            for (int i = 2; i < 62; i += 4) {
+                mx0 = fmax3(mx0, x[i], x[i + 1]);
+                mx1 = fmax3(mx1, x[i + 2], x[i + 3]);
             }
-            const float m_new = fmaxf(m, fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sc);
+            mx0 = fmax3(mx0, x[62], x[63]);
+            const float m_new = fmaxf(m, fmaxf(mx0, mx1) * sc);
             const bool grow = m_new > m + 8.f;
             if (j > 0 && __any_sync(0xffffffffu, grow)) {
                 // O holds sum P V with the old running max: move the max, rescale O and l.
@@ -337,18 +353,25 @@ __global__ void __launch_bounds__(192, 2)
             }
             // p = 2^(s * scale * log2e - m), packed to bf16 pairs over the S columns just read
             const float nm = (m == -INFINITY) ? 0.f : -m;
-            float rs0 = 0.f, rs1 = 0.f;
+            const uint64_t sc2 = pack2(sc, sc), nm2 = pack2(nm, nm);
+            uint64_t acc0 = pack2(0.f, 0.f), acc1 = acc0;
             uint32_t pk[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-                const float p0 = ex2_approx(fmaf(x[2 * i], sc, nm));
-                const float p1 = ex2_approx(fmaf(x[2 * i + 1], sc, nm));
-                rs0 += p0;
-                rs1 += p1;
+                float y0, y1;
+                unpack2(ffma2(pack2(x[2 * i], x[2 * i + 1]), sc2, nm2), y0, y1);
+                const float p0 = ex2_approx(y0), p1 = ex2_approx(y1);
+                if (i & 1) acc1 = fadd2(acc1, pack2(p0, p1));
+                else acc0 = fadd2(acc0, pack2(p0, p1));
                 __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
                 pk[i] = *reinterpret_cast<uint32_t*>(&h2);
             }
-            l += rs0 + rs1;
+            {
+                float a0, a1, b0, b1;
+                unpack2(acc0, a0, a1);
+                unpack2(acc1, b0, b1);
+                l += (a0 + a1) + (b0 + b1);
+            }
             tmem_st32(sbuf, pk);
             tmem_wait_st();
             tc_fence_before();
