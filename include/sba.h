@@ -58,7 +58,8 @@ typedef enum {
     SBA_ERR_ALIGNMENT = 3,     /* a device pointer not 16-byte aligned */
     SBA_ERR_CUDA = 4,          /* a CUDA runtime or driver call failed */
     SBA_ERR_TIMEOUT = 5,       /* a kernel wait gave up (reported by sba_get_device_status) */
-    SBA_ERR_DEVICE_FLAG = 6    /* a kernel found a bad routing entry (sba_get_device_status) */
+    SBA_ERR_DEVICE_FLAG = 6,   /* a kernel found a bad routing entry (sba_get_device_status) */
+    SBA_ERR_SCRATCH_TOO_SMALL = 7  /* problem too large for sba_pool_select_noalloc's fixed scratch */
 } sba_status;
 
 /* Largest padded sequence length a call accepts (4096 blocks of 64 tokens). */
@@ -122,6 +123,38 @@ sba_status sba_get_device_status(void* stream);
  * sets SBA_ERR_TIMEOUT and lets the kernel exit cleanly.  0 restores the
  * default.  Meant for tests of the timeout path. */
 void sba_set_wait_limit(uint64_t cycles);
+
+/* Routing for callers that cannot allocate device memory.
+ *
+ * No counterpart on the pages: this is a library convenience.  Some callers may
+ * not call cudaMalloc at all -- for instance code that runs inside a host
+ * framework which owns every byte of device memory and hands the kernel no
+ * workspace, or a latency-critical path where an allocation (which can
+ * synchronise the device) is not allowed.  For them this entry point does what
+ * sba_pool_select does, with the same arguments apart from the workspace, using
+ * scratch that lives in a fixed array inside the library instead.
+ *
+ *   - The array holds sba_noalloc_scratch_bytes() bytes (16 MiB).  Every GPU that
+ *     loads the library keeps that much device memory for it until the process
+ *     exits.  A problem whose sba_pool_select_workspace_size() exceeds it is
+ *     rejected with SBA_ERR_SCRATCH_TOO_SMALL before anything is launched.
+ *   - Nothing is allocated or freed: the call makes no cudaMalloc/cudaFree and
+ *     calls no allocating library routine.
+ *   - The first call on a device looks up the array's device address (once per
+ *     device, under a lock) with cudaGetSymbolAddress; make that first call
+ *     before any stream capture.
+ *   - All calls on a device share the one array and it keeps whatever the last
+ *     call left in it.  That is harmless here, since every value a call reads
+ *     from it was written earlier in the same call, so nothing has to start at
+ *     zero.  But two calls whose kernels overlap on the GPU (different streams,
+ *     no ordering between them) race on the array and may return wrong
+ *     routings: serialise them. */
+sba_status sba_pool_select_noalloc(const void* q, const void* k, int B, int H, int Npad, int D,
+                                   const int32_t* valid_len, int block, double sparsity, int kmax,
+                                   int32_t* kv_idx, int32_t* kv_cnt, void* stream);
+
+/* Size in bytes of the fixed scratch array sba_pool_select_noalloc uses. */
+size_t sba_noalloc_scratch_bytes(void);
 
 /* Static description of a status code. */
 const char* sba_strerror(sba_status status);

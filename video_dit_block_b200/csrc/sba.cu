@@ -239,8 +239,53 @@ const char* sba_strerror(sba_status status) {
         case SBA_ERR_CUDA: return "CUDA call failed";
         case SBA_ERR_TIMEOUT: return "a kernel wait gave up";
         case SBA_ERR_DEVICE_FLAG: return "a kernel found an invalid routing entry";
+        case SBA_ERR_SCRATCH_TOO_SMALL: return "problem needs more scratch than the fixed no-allocation buffer holds";
     }
     return "unknown status";
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- routing without allocation
+// Scratch for sba_pool_select_noalloc: a fixed array in device memory that every
+// GPU loading this library holds until the process exits.  Its name is only a
+// host-side handle; the kernel gets the device address from cudaGetSymbolAddress.
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+void* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mutex;
+
+// Device address of the scratch array on the current device, resolved on first use.
+sba_status noalloc_scratch(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SBA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return SBA_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return SBA_OK;
+}
+}  // namespace
+
+extern "C" size_t sba_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
+
+extern "C" sba_status sba_pool_select_noalloc(const void* q, const void* k, int B, int H, int Npad,
+                                              int D, const int32_t* valid_len, int block,
+                                              double sparsity, int kmax, int32_t* kv_idx,
+                                              int32_t* kv_cnt, void* stream) {
+    sba_status st = check_shape(B, H, Npad, D, block);
+    if (st != SBA_OK) return st;
+    const size_t need = sba::select_workspace_bytes((size_t)B * H, (size_t)Npad / block, (size_t)D);
+    if (need > kNoAllocScratchBytes) return SBA_ERR_SCRATCH_TOO_SMALL;
+    void* scratch = nullptr;
+    st = noalloc_scratch(&scratch);
+    if (st != SBA_OK) return st;
+    return sba_pool_select(q, k, B, H, Npad, D, valid_len, block, sparsity, kmax, kv_idx, kv_cnt,
+                           scratch, kNoAllocScratchBytes, stream);
+}

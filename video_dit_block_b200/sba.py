@@ -16,7 +16,8 @@ from .build import LIB
 
 SBA_OK = 0
 _STATUS = {0: "SBA_OK", 1: "SBA_ERR_INVALID_ARG", 2: "SBA_ERR_UNSUPPORTED", 3: "SBA_ERR_ALIGNMENT",
-           4: "SBA_ERR_CUDA", 5: "SBA_ERR_TIMEOUT", 6: "SBA_ERR_DEVICE_FLAG"}
+           4: "SBA_ERR_CUDA", 5: "SBA_ERR_TIMEOUT", 6: "SBA_ERR_DEVICE_FLAG",
+           7: "SBA_ERR_SCRATCH_TOO_SMALL"}
 MAX_NPAD = 262144
 BLOCK = 64
 
@@ -55,6 +56,10 @@ def lib() -> ctypes.CDLL:
         L.sba_get_device_status.argtypes = [vp]
         L.sba_set_wait_limit.restype = None
         L.sba_set_wait_limit.argtypes = [ctypes.c_uint64]
+        L.sba_pool_select_noalloc.restype = i32
+        L.sba_pool_select_noalloc.argtypes = [vp, vp, i32, i32, i32, i32, vp, i32, f64, i32, vp, vp, vp]
+        L.sba_noalloc_scratch_bytes.restype = sz
+        L.sba_noalloc_scratch_bytes.argtypes = []
         L.sba_strerror.restype = ctypes.c_char_p
         L.sba_strerror.argtypes = [i32]
         _lib = L
