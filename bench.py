@@ -47,6 +47,20 @@ def parse():
     return ap.parse_args()
 
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one attention launch,
+# from the ncu capture summarised in profiles/attn_kernel_480p_dense.md, and the hash
+# of the kernel sources it was taken with.  Reported only while the sources match.
+ATTN_TRAFFIC = {"480p_dense": (636370688 + 190253568, "33c27d24287ca6f9")}
+KERNEL_SOURCES = ("video_dit_block_b200/csrc/attention.cuh", "video_dit_block_b200/csrc/ptx.cuh",
+                  "video_dit_block_b200/csrc/common.cuh")
+
+
+def kernel_source_hash():
+    import hashlib
+    data = b"".join(open(os.path.join(ROOT, f), "rb").read() for f in KERNEL_SOURCES)
+    return hashlib.sha256(data).hexdigest()[:16]
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -141,13 +155,15 @@ def oracle_sample(w, target_s=10.0, seed=0):
     L = int(vl1[0])
     nB0 = (L + 63) // 64
     order = np.random.default_rng(seed).permutation(nB0).astype(np.int32)
-    t0 = time.perf_counter()
-    oracle.attention(q1, k1, v1, idx, cnt, vl1, qblocks=order[:1])
-    t_one = max(time.perf_counter() - t0, 1e-4)
-    n = int(max(1, min(nB0, target_s / t_one)))
-    t0 = time.perf_counter()
-    oracle.attention(q1, k1, v1, idx, cnt, vl1, qblocks=order[:n])
-    t_attn = time.perf_counter() - t0
+    # grow the sample (doubling) until one run takes about target_s / 2 or covers the head
+    n, t_attn = 1, 0.0
+    while True:
+        t0 = time.perf_counter()
+        oracle.attention(q1, k1, v1, idx, cnt, vl1, qblocks=order[:n])
+        t_attn = time.perf_counter() - t0
+        if t_attn >= target_s / 2 or n >= nB0:
+            break
+        n = min(nB0, max(2 * n, int(n * target_s / 2 / max(t_attn, 1e-3))))
     sel = order[:n]
     sub_cnt = np.zeros_like(cnt)
     sub_cnt[:, :, sel] = cnt[:, :, sel]
@@ -315,6 +331,8 @@ def run_ours(args):
             dist.destroy_process_group()
         return
     peaks, src = load_peaks()
+    tr = ATTN_TRAFFIC.get(w.name)
+    traffic = tr[0] if tr is not None and tr[1] == kernel_source_hash() else None
     peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
     achieved = f_step / (attn_ms * 1e-3) / 1e12
     line = {
@@ -330,7 +348,7 @@ def run_ours(args):
         "roofline": {"bound": "tensor", "kernel": "attn_kernel<128,2>" if D == 128 else "attn_kernel<64,4>",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_source": f"{src} bf16_tflops_sustained (kernel timed inside a seconds-long loop)",
-                     "traffic": None},
+                     "traffic": traffic},
         "gpu_launches": 4 * K,
         "clocks": clk,
     }
