@@ -1,8 +1,9 @@
 #!/usr/bin/env python
 """Benchmark of the block-sparse attention path on B200.
 
-One step = the whole path over one batch: sba_pool_select (pool, score, top-k) then
-sba_attention over the kept blocks.  Prints ONE JSON line (rank 0).
+One step = the whole path over one batch: sba_pool_select (pool, score, top-k),
+sba_pair_query_blocks (which two query blocks share an attention tile) and
+sba_attention_paired over the kept blocks.  Prints ONE JSON line (rank 0).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
 
@@ -245,12 +246,22 @@ def run_ours(args):
     ws = torch.empty(sba.workspace_size(B, H, Npad, D), dtype=torch.uint8, device=dev)
     o = torch.empty_like(q)
     lse = torch.empty((B, H, Npad), dtype=torch.float32, device=dev)
+    nQ = Npad // 64
+    pair_order = torch.empty((B, H, 2 * ((nQ + 1) // 2)), dtype=torch.int32, device=dev)
+    pws = torch.empty(int(sba.lib().sba_pair_workspace_size(B, H, Npad, 64)), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step(qq=q, kk=k, vv=v):
-        sba.pool_select(qq, kk, vl, w.sparsity, kmax, kv_idx=kv_idx, kv_cnt=kv_cnt, workspace=ws,
+    def route(qq=q, kk=k, vll=vl):
+        sba.pool_select(qq, kk, vll, w.sparsity, kmax, kv_idx=kv_idx, kv_cnt=kv_cnt, workspace=ws,
                         stream=stream)
-        sba.attention(qq, kk, vv, kv_idx, kv_cnt, vl, out=o, lse=lse, stream=stream)
+        sba.pair_query_blocks(kv_idx, kv_cnt, vll, pair_order=pair_order, workspace=pws, stream=stream)
+
+    def attend(qq=q, kk=k, vv=v, vll=vl):
+        sba.attention_paired(qq, kk, vv, kv_idx, kv_cnt, pair_order, vll, out=o, lse=lse, stream=stream)
+
+    def step(qq=q, kk=k, vv=v):
+        route(qq, kk)
+        attend(qq, kk, vv)
 
     def barrier():
         if dist is not None:
@@ -274,10 +285,9 @@ def run_ours(args):
     time.sleep(0.3)
     for i in range(K):
         ev[i][0].record(stream)
-        sba.pool_select(q, k, vl, w.sparsity, kmax, kv_idx=kv_idx, kv_cnt=kv_cnt, workspace=ws,
-                        stream=stream)
+        route()
         ev[i][1].record(stream)
-        sba.attention(q, k, v, kv_idx, kv_cnt, vl, out=o, lse=lse, stream=stream)
+        attend()
         ev[i][2].record(stream)
     torch.cuda.synchronize(dev)
     clk = clocks.stop()
@@ -312,9 +322,8 @@ def run_ours(args):
             kd.copy_(kh, non_blocking=True)
             vd.copy_(vh, non_blocking=True)
             vld.copy_(vlh, non_blocking=True)
-            sba.pool_select(qd, kd, vld, w.sparsity, kmax, kv_idx=kv_idx, kv_cnt=kv_cnt, workspace=ws,
-                            stream=stream)
-            sba.attention(qd, kd, vd, kv_idx, kv_cnt, vld, out=o, lse=lse, stream=stream)
+            route(qd, kd, vld)
+            attend(qd, kd, vd, vld)
             oh.copy_(o, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize(dev)
@@ -349,7 +358,9 @@ def run_ours(args):
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_source": f"{src} bf16_tflops_sustained (kernel timed inside a seconds-long loop)",
                      "traffic": traffic},
-        "gpu_launches": 4 * K,
+        # per step: 2 pooling + 1 scoring/top-k, 10 pairing (bitmaps, 4 x propose/resolve,
+        # emit), 1 attention
+        "gpu_launches": 14 * K,
         "clocks": clk,
     }
     if e2e is not None:

@@ -107,6 +107,32 @@ sba_status sba_attention(const void* q, const void* k, const void* v, void* o, f
                          const int32_t* kv_idx, const int32_t* kv_cnt, int kmax,
                          float softmax_scale, void* stream);
 
+/* Pairing of query blocks into attention tiles (a performance choice only).
+ * The attention kernel processes two 64-row query blocks per 128-row tile over
+ * the union of their kept key blocks, so a key block kept by only one of the two
+ * is masked work for the other.  This pass picks, per (b, h), pairs whose kept
+ * lists overlap most: bitmaps of the kept sets, four rounds of mutual-best
+ * matching among query blocks at most 64 positions apart, the rest paired in
+ * order.  It never changes a result of sba_attention_paired, only its speed.
+ *   kv_idx, kv_cnt, kmax, valid_len  a routing as produced by sba_pool_select
+ *   pair_order  int32 [B, H, 2 * ceil(Npad/block / 2)] (written): tile t holds
+ *               query blocks pair_order[b,h,2t] and [2t+1]; every query block of
+ *               [0, Npad/block) appears once; a final unused slot is -1
+ *   workspace   device buffer of sba_pair_workspace_size() bytes, 16-byte aligned */
+size_t sba_pair_workspace_size(int B, int H, int Npad, int block);
+sba_status sba_pair_query_blocks(const int32_t* kv_idx, const int32_t* kv_cnt, int B, int H,
+                                 int Npad, int kmax, const int32_t* valid_len, int block,
+                                 int32_t* pair_order, void* workspace, size_t workspace_bytes,
+                                 void* stream);
+
+/* sba_attention with the tiles given by pair_order (see sba_pair_query_blocks);
+ * results equal sba_attention's up to the order of floating-point accumulation.
+ * pair_order must not be NULL; every query block must appear in it once. */
+sba_status sba_attention_paired(const void* q, const void* k, const void* v, void* o, float* lse,
+                                int B, int H, int Npad, int D, const int32_t* valid_len, int block,
+                                const int32_t* kv_idx, const int32_t* kv_cnt, int kmax,
+                                const int32_t* pair_order, float softmax_scale, void* stream);
+
 /* Dense attention over all valid tokens of each sample (the sparsity = 0 case
  * without a routing), same layouts as sba_attention. */
 sba_status sba_dense_attention(const void* q, const void* k, const void* v, void* o, float* lse,

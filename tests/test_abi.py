@@ -98,6 +98,17 @@ def test_dense_attention_rejects(lib):
     assert lib.sba_dense_attention(MIS, A, A, A, A, 1, 2, 1024, 64, NULL, 0.0, S) == 3
 
 
+def test_pairing_rejects(lib):
+    assert lib.sba_pair_workspace_size(1, 2, 1024, 64) > 0
+    assert lib.sba_pair_query_blocks(A, A, 1, 2, 1024, 8, NULL, 64, NULL, A, 1 << 30, S) == 1
+    assert lib.sba_pair_query_blocks(A, A, 1, 2, 1024, 8, NULL, 64, A, A, 16, S) == 1
+    assert lib.sba_pair_query_blocks(A, A, 1, 2, 1000, 8, NULL, 64, A, A, 1 << 30, S) == 1
+    assert lib.sba_pair_query_blocks(A, A, 1, 2, 1024, 8, NULL, 64, A, MIS, 1 << 30, S) == 3
+    assert lib.sba_attention_paired(A, A, A, A, A, 1, 2, 1024, 64, NULL, 64, A, A, 8, NULL, 0.0, S) == 1
+    assert lib.sba_attention_paired(A, A, A, A, A, 1, 2, 1024, 64, NULL, 64, A, A, 8,
+                                    ctypes.c_void_p(0x10002), 0.0, S) == 3
+
+
 def test_block_means_rejects(lib):
     assert lib.sba_block_means(NULL, 1, 2, 1024, 64, NULL, 64, A, S) == 1
     assert lib.sba_block_means(A, 1, 2, 1024, 64, NULL, 64, MIS, S) == 3

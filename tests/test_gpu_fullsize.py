@@ -22,8 +22,8 @@ def sba():
 def test_full_size_sampled(sba, oracle_mod, name):
     w = make_workload(name)
     q, k, v, vl = to_device(w, DEV)
-    idx, cnt = sba.pool_select(q, k, vl, w.sparsity)
-    o, lse = sba.attention(q, k, v, idx, cnt, vl)
+    # the bench's path: routing, tile pairing, paired attention
+    o, lse, idx, cnt = sba.sparse_attention(q, k, v, vl, w.sparsity)
     assert sba.device_status() == 0
     rng = np.random.default_rng(len(name))
     idx_h, cnt_h = idx.cpu().numpy(), cnt.cpu().numpy()

@@ -3,9 +3,9 @@
 The compute path is a C-ABI CUDA library (include/sba.h, csrc/); this package is its
 Python binding.  See `sba` for the calls.
 """
-from .sba import (SbaError, attention, block_means, dense_attention, device_status, keep_count,
-                  kmax_for, lib, pool_select, set_wait_limit, sparse_attention, workspace_size)
+from .sba import (SbaError, attention, attention_paired, block_means, dense_attention, device_status, keep_count,
+                  kmax_for, lib, pair_query_blocks, pool_select, set_wait_limit, sparse_attention, workspace_size)
 
-__all__ = ["SbaError", "attention", "block_means", "dense_attention", "device_status",
-           "keep_count", "kmax_for", "lib", "pool_select", "set_wait_limit", "sparse_attention",
+__all__ = ["SbaError", "attention", "attention_paired", "block_means", "dense_attention", "device_status",
+           "keep_count", "kmax_for", "lib", "pair_query_blocks", "pool_select", "set_wait_limit", "sparse_attention",
            "workspace_size"]

@@ -5,8 +5,10 @@
 // sparse attention works": each query block attends, exactly, to the tokens of
 // its kept key blocks only, and the full attention matrix is never formed.
 //
-// Tiling.  A CTA owns two adjacent 64-row query blocks I0 = 2p, I1 = 2p + 1 of
-// one (b, h): a 128-row Q tile, the full-rate M of a single-CTA tcgen05.mma.
+// Tiling.  A CTA owns two 64-row query blocks of one (b, h) -- by default the
+// adjacent I0 = 2p, I1 = 2p + 1, or the pair a routing-side pass chose for overlap
+// of their kept lists -- as a 128-row Q tile, the full-rate M of a single-CTA
+// tcgen05.mma.
 // It walks the ascending union of the two kept lists; a key block kept by only
 // one of the two is masked to -inf for the other half's rows.
 //
@@ -46,6 +48,7 @@ struct AttnParams {
     const int32_t* valid_len;
     const int32_t* kv_idx;
     const int32_t* kv_cnt;
+    const int32_t* pair_order;  // [B*H][2*ceil(nQ/2)] query blocks per tile, -1 = none; NULL = adjacent
     int H;
     int Npad;
     int kmax;
@@ -120,7 +123,13 @@ __global__ void __launch_bounds__(192, 2)
     const int h = blockIdx.y, b = blockIdx.z;
     const int bh = b * p.H + h;
     const int nQ = p.Npad / 64;
-    const int I0 = 2 * blockIdx.x;
+    // the tile's two query blocks; a slot outside [0, nQ) is empty
+    int qb[2] = {2 * (int)blockIdx.x, 2 * (int)blockIdx.x + 1};
+    if (p.pair_order) {
+        const int32_t* po = p.pair_order + (size_t)bh * (2 * gridDim.x) + 2 * blockIdx.x;
+        qb[0] = po[0];
+        qb[1] = po[1];
+    }
     const int L = p.valid_len ? p.valid_len[b] : p.Npad;
     const int nB = (L + 63) / 64;
     const int W = (nB + 31) / 32;
@@ -148,14 +157,14 @@ __global__ void __launch_bounds__(192, 2)
         for (int w = lane; w < W; w += 32) {
             uint32_t full = 0;
             if (p.dense) full = (w * 32 + 32 <= nB) ? 0xffffffffu : ((1u << (nB - w * 32)) - 1u);
-            bm[w] = (p.dense && I0 < nB) ? full : 0u;
-            bm[kMaxBlocks / 32 + w] = (p.dense && I0 + 1 < nB) ? full : 0u;
+            bm[w] = (p.dense && qb[0] >= 0 && qb[0] < nB) ? full : 0u;
+            bm[kMaxBlocks / 32 + w] = (p.dense && qb[1] >= 0 && qb[1] < nB) ? full : 0u;
         }
         __syncwarp();
         if (!p.dense) {
             for (int half = 0; half < 2; ++half) {
-                const int I = I0 + half;
-                if (I >= nQ) continue;
+                const int I = qb[half];
+                if (I < 0 || I >= nQ) continue;
                 const size_t row = (size_t)bh * nQ + I;
                 int cnt = p.kv_cnt[row];
                 if (cnt < 0 || cnt > p.kmax) {
@@ -209,9 +218,13 @@ __global__ void __launch_bounds__(192, 2)
             tma_prefetch_desc(&tmQ);
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
-            mbar_arrive_expect_tx(bar_q, SM::kQBytes);
-            for (int c = 0; c < NCH; ++c)
-                tma_load_3d(sQ + c * (128 * 128), &tmQ, bar_q, c * 64, I0 * 64, bh);
+            // Q: one 64-row box per query block of the tile (an empty slot's rows stay
+            // unloaded; its rows keep nothing, so they only ever multiply P = 0)
+            const bool q1 = qb[1] >= 0 && qb[1] < nQ;
+            mbar_arrive_expect_tx(bar_q, (q1 ? 2 : 1) * (64 * D * 2));
+            for (int h2 = 0; h2 < (q1 ? 2 : 1); ++h2)
+                for (int c = 0; c < NCH; ++c)
+                    tma_load_3d(sQ + c * (128 * 128) + h2 * (64 * 128), &tmQ, bar_q, c * 64, qb[h2] * 64, bh);
             // K runs one block ahead of V: K(j) is released as soon as S(j) is done,
             // V(j) only after PV(j).  Issue order K0, K1, V0, K2, V1, ...
             for (int j = 0; j <= n; ++j) {
@@ -279,7 +292,7 @@ __global__ void __launch_bounds__(192, 2)
         // ------------------------------------------------------------ softmax warps
         const int r = tid;                      // query row of the tile = TMEM lane
         const int half = r >> 6;
-        const int tok = (I0 + half) * 64 + (r & 63);
+        const int tok = qb[half] * 64 + (r & 63);
         const uint32_t* bmh = bm + half * (kMaxBlocks / 32);
         const uint32_t tl = tmem + (static_cast<uint32_t>(warp * 32) << 16);
         const float sc = p.scale_log2;
@@ -381,7 +394,7 @@ __global__ void __launch_bounds__(192, 2)
         // ------------------------------------------------------------ epilogue
         if (ok && n > 0) ok = warp_wait_bounded(bar_pv((n - 1) & 1), ((n - 1) >> 1) & 1, abort_flag, lim);
         tc_fence_after();
-        const bool in_range = tok < p.Npad && (I0 + half) < nQ;
+        const bool in_range = qb[half] >= 0 && qb[half] < nQ;
         const bool valid = tok < L && l > 0.f;
         __nv_bfloat16* orow = p.o + ((size_t)bh * p.Npad + tok) * D;
         if (ok) {

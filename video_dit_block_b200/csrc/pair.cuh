@@ -1,0 +1,220 @@
+// pair.cuh -- choose which two query blocks share a 128-row attention tile.
+//
+// The attention kernel runs two 64-row query blocks per tile over the union of
+// their kept key blocks; a key block kept by only one of them is masked work for
+// the other.  Pairing query blocks whose kept lists overlap most cuts that waste.
+// This pass is a heuristic on top of the routing and never changes any result,
+// only which query blocks share a tile:
+//   1. a bitmap of each query block's kept key blocks;
+//   2. a few rounds of mutual-best matching: every unmatched query block proposes
+//      the unmatched block within +-64 positions whose kept set overlaps its own
+//      most (ties: nearer, then lower), and mutual proposals are matched.  Overlaps
+//      are computed once; later rounds walk each block's 16 best candidates.  The
+//      window reaches the same position one frame later in the raster order of
+//      these latent grids (25-57 blocks per frame), where the kept sets are most
+//      alike;
+//   3. the tile list: matched pairs in order, then the leftovers two by two, then
+//      the blocks past the sample's valid length; an odd count leaves one slot -1.
+#pragma once
+#include <cstdint>
+
+#include "select.cuh"  // align256
+
+namespace sba {
+
+constexpr int kPairWindow = 64;  // a multiple of 32
+constexpr int kPairRounds = 4;
+
+constexpr int kPairCands = 16;  // candidates kept per query block after the overlap pass
+
+struct PairWorkspace {
+    uint32_t* bits;     // [BH][nQ][W] kept-set bitmaps, W = ceil(nQ / 32)
+    int32_t* proposal;  // [BH][nQ]
+    int32_t* partner;   // [BH][nQ], -1 = unmatched
+    int32_t* cand;      // [BH][nQ][kPairCands] best candidates in preference order, -1 = none
+};
+
+__host__ __device__ inline size_t pair_workspace_bytes(size_t BH, size_t nQ) {
+    const size_t W = (nQ + 31) / 32;
+    return align256(BH * nQ * W * 4) + 2 * align256(BH * nQ * 4) + align256(BH * nQ * kPairCands * 4);
+}
+
+__host__ __device__ inline PairWorkspace carve_pair_workspace(void* base, size_t BH, size_t nQ) {
+    const size_t W = (nQ + 31) / 32;
+    char* p = static_cast<char*>(base);
+    PairWorkspace w;
+    w.bits = reinterpret_cast<uint32_t*>(p);
+    p += align256(BH * nQ * W * 4);
+    w.proposal = reinterpret_cast<int32_t*>(p);
+    p += align256(BH * nQ * 4);
+    w.partner = reinterpret_cast<int32_t*>(p);
+    p += align256(BH * nQ * 4);
+    w.cand = reinterpret_cast<int32_t*>(p);
+    return w;
+}
+
+// One warp per routing row (bh, I): its kept-set bitmap (built in shared memory,
+// then written out word by word); partner reset to -1.
+__global__ void __launch_bounds__(256) pair_bitmap_kernel(PairWorkspace ws, const int32_t* __restrict__ kv_idx,
+                                                          const int32_t* __restrict__ kv_cnt, int nQ, int kmax,
+                                                          long long rows) {
+    extern __shared__ uint32_t srow[];  // [8 warps][W]
+    const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
+    const long long row = (long long)blockIdx.x * 8 + warp;
+    if (row >= rows) return;
+    const int W = (nQ + 31) / 32;
+    uint32_t* bm = srow + warp * W;
+    for (int w = lane; w < W; w += 32) bm[w] = 0u;
+    __syncwarp();
+    int cnt = kv_cnt[row];
+    cnt = cnt < 0 ? 0 : (cnt > kmax ? kmax : cnt);
+    const int32_t* lst = kv_idx + (size_t)row * kmax;
+    for (int t = lane; t < cnt; t += 32) {
+        const int J = lst[t];
+        if (J >= 0 && J < nQ) atomicOr(&bm[J >> 5], 1u << (J & 31));
+    }
+    __syncwarp();
+    uint32_t* out = ws.bits + (size_t)row * W;
+    for (int w = lane; w < W; w += 32) out[w] = bm[w];
+    if (lane == 0) ws.partner[row] = -1;
+}
+
+// A CTA of 8 warps proposes for 8 consecutive query blocks a0..a0+7 of one (b, h);
+// the bitmaps of their joint window [a0 - 64, a0 + 71] are staged in shared memory
+// once.  A query block that keeps every key block (dense routing) has the same
+// overlap with every candidate and proposes nothing, so it stays in order.
+constexpr int kPairWarps = 8;
+constexpr int kPairSpan = 2 * kPairWindow + kPairWarps;  // blocks staged per CTA
+
+__global__ void __launch_bounds__(256) pair_propose_kernel(PairWorkspace ws,
+                                                           const int32_t* __restrict__ kv_cnt,
+                                                           const int32_t* __restrict__ valid_len,
+                                                           int H, int nQ, int tiles_per_bh) {
+    extern __shared__ uint32_t sbits[];  // [kPairSpan][W]
+    const int bh = blockIdx.x / tiles_per_bh;
+    const int a0 = (blockIdx.x % tiles_per_bh) * kPairWarps;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
+    const int L = valid_len ? valid_len[bh / H] : nQ * 64;
+    const int nB = (L + 63) / 64;
+    const int W = (nQ + 31) / 32;
+    const uint32_t* gbits = ws.bits + (size_t)bh * nQ * W;
+    const int lo = a0 - kPairWindow;
+    for (int i = threadIdx.x; i < kPairSpan * W; i += blockDim.x) {
+        const int c = lo + i / W;
+        sbits[i] = (c >= 0 && c < nB) ? gbits[(size_t)c * W + (i % W)] : 0u;
+    }
+    __syncthreads();
+    const int a = a0 + warp;
+    if (a >= nQ) return;
+    const size_t row = (size_t)bh * nQ + a;
+    int32_t* cand = ws.cand + row * kPairCands;
+    if (a >= nB || kv_cnt[row] >= nB) {
+        if (lane < kPairCands) cand[lane] = -1;
+        if (lane == 0) ws.proposal[row] = -1;
+        return;
+    }
+    const uint32_t* ba = sbits + (size_t)(a - lo) * W;
+    // lane l scores a - 64 + l, a - 32 + l, a + 1 + l, a + 33 + l.  Preference as one
+    // ordered key: larger overlap, then smaller distance, then lower index.
+    constexpr int kSlots = 2 * kPairWindow / 32;
+    long long key[kSlots];
+#pragma unroll
+    for (int slot = 0; slot < kSlots; ++slot) {
+        const int half = kPairWindow / 32;
+        const int c = slot < half ? a - kPairWindow + 32 * slot + lane : a + 1 + 32 * (slot - half) + lane;
+        key[slot] = -1;
+        if (c < 0 || c >= nB) continue;
+        const uint32_t* bc = sbits + (size_t)(c - lo) * W;
+        int ov = 0;
+        for (int w = 0; w < W; ++w) ov += __popc(ba[w] & bc[w]);
+        const int dist = c > a ? c - a : a - c;
+        key[slot] = ((long long)ov << 40) | ((long long)(0xFFFFF - dist) << 20) | (long long)(0xFFFFF - c);
+    }
+    // the kPairCands best candidates, best first
+    for (int r = 0; r < kPairCands; ++r) {
+        long long mine = key[0];
+#pragma unroll
+        for (int slot = 1; slot < kSlots; ++slot) mine = key[slot] > mine ? key[slot] : mine;
+        long long best = mine;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const long long o = __shfl_xor_sync(0xffffffffu, best, off);
+            best = o > best ? o : best;
+        }
+        if (best >= 0 && mine == best) {
+#pragma unroll
+            for (int slot = 0; slot < kSlots; ++slot) key[slot] = key[slot] == best ? -1 : key[slot];
+        }
+        if (lane == 0) cand[r] = best < 0 ? -1 : (int)(0xFFFFF - (best & 0xFFFFF));
+    }
+    if (lane == 0) ws.proposal[row] = cand[0];
+}
+
+// Later rounds, one thread per (bh, a): propose the first still-unmatched cached candidate.
+__global__ void pair_repropose_kernel(PairWorkspace ws, int nQ, long long rows) {
+    const long long row = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (row >= rows) return;
+    const long long bh = row / nQ;
+    int prop = -1;
+    if (ws.partner[row] < 0) {
+        const int32_t* cand = ws.cand + row * kPairCands;
+        for (int r = 0; r < kPairCands; ++r) {
+            const int c = cand[r];
+            if (c >= 0 && ws.partner[bh * nQ + c] < 0) {
+                prop = c;
+                break;
+            }
+        }
+    }
+    ws.proposal[row] = prop;
+}
+
+// One thread per (bh, a): match mutual proposals.
+__global__ void pair_resolve_kernel(PairWorkspace ws, int nQ, long long rows) {
+    const long long row = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (row >= rows) return;
+    const long long bh = row / nQ;
+    const int c = ws.proposal[row];
+    if (c < 0 || ws.partner[row] >= 0) return;
+    if (ws.proposal[bh * nQ + c] == (int)(row % nQ)) ws.partner[row] = c;
+}
+
+// One warp per bh: the tile list pair_order[bh][2 * nP] (nP = ceil(nQ / 2)).
+__global__ void pair_emit_kernel(PairWorkspace ws, const int32_t* __restrict__ valid_len, int H, int nQ,
+                                 int32_t* __restrict__ pair_order, int BH) {
+    const int bh = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+    const int lane = threadIdx.x & 31;
+    if (bh >= BH) return;
+    const int L = valid_len ? valid_len[bh / H] : nQ * 64;
+    const int nB = (L + 63) / 64;
+    const int nP = (nQ + 1) / 2;
+    const int32_t* partner = ws.partner + (size_t)bh * nQ;
+    int32_t* out = pair_order + (size_t)bh * 2 * nP;
+    int pos = 0;
+    // matched pairs, by their lower block
+    for (int a0 = 0; a0 < nQ; a0 += 32) {
+        const int a = a0 + lane;
+        const int pa = a < nB ? partner[a] : -1;
+        const bool lead = a < nB && pa > a;
+        const uint32_t bal = __ballot_sync(0xffffffffu, lead);
+        if (lead) {
+            const int slot = pos + 2 * __popc(bal & ((1u << lane) - 1u));
+            out[slot] = a;
+            out[slot + 1] = pa;
+        }
+        pos += 2 * __popc(bal);
+    }
+    // unmatched valid blocks, then blocks past the valid length, two by two
+    for (int pass = 0; pass < 2; ++pass) {
+        for (int a0 = 0; a0 < nQ; a0 += 32) {
+            const int a = a0 + lane;
+            const bool take = pass == 0 ? (a < nB && partner[a] < 0) : (a >= nB && a < nQ);
+            const uint32_t bal = __ballot_sync(0xffffffffu, take);
+            if (take) out[pos + __popc(bal & ((1u << lane) - 1u))] = a;
+            pos += __popc(bal);
+        }
+    }
+    if (lane == 0 && pos < 2 * nP) out[pos] = -1;
+}
+
+}  // namespace sba

@@ -13,6 +13,7 @@
 #include "attention.cuh"
 #include "common.cuh"
 #include "select.cuh"
+#include "pair.cuh"
 
 namespace {
 
@@ -70,11 +71,11 @@ template <int D, int NS>
 sba_status launch_attention(const void* q, const void* k, const void* v, void* o, float* lse,
                             int B, int H, int Npad, const int32_t* valid_len,
                             const int32_t* kv_idx, const int32_t* kv_cnt, int kmax, int dense,
-                            float softmax_scale, cudaStream_t stream) {
+                            const int32_t* pair_order, float softmax_scale, cudaStream_t stream) {
     using SM = sba::AttnSmem<D, NS>;
     CUtensorMap tq, tk, tv;
     const int BH = B * H;
-    if (!make_map(&tq, q, BH, Npad, D, 128) || !make_map(&tk, k, BH, Npad, D, 64) ||
+    if (!make_map(&tq, q, BH, Npad, D, 64) || !make_map(&tk, k, BH, Npad, D, 64) ||
         !make_map(&tv, v, BH, Npad, D, 64))
         return SBA_ERR_CUDA;
     if (cudaFuncSetAttribute(sba::attn_kernel<D, NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -86,6 +87,7 @@ sba_status launch_attention(const void* q, const void* k, const void* v, void* o
     p.valid_len = valid_len;
     p.kv_idx = kv_idx;
     p.kv_cnt = kv_cnt;
+    p.pair_order = pair_order;
     p.H = H;
     p.Npad = Npad;
     p.kmax = kmax;
@@ -182,7 +184,8 @@ sba_status sba_block_means(const void* x, int B, int H, int Npad, int D, const i
 static sba_status attention_common(const void* q, const void* k, const void* v, void* o, float* lse,
                                    int B, int H, int Npad, int D, const int32_t* valid_len,
                                    int block, const int32_t* kv_idx, const int32_t* kv_cnt,
-                                   int kmax, int dense, float softmax_scale, void* stream) {
+                                   int kmax, int dense, const int32_t* pair_order,
+                                   float softmax_scale, void* stream) {
     sba_status st = check_shape(B, H, Npad, D, block);
     if (st != SBA_OK) return st;
     if (!q || !k || !v || !o) return SBA_ERR_INVALID_ARG;
@@ -192,14 +195,15 @@ static sba_status attention_common(const void* q, const void* k, const void* v, 
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(valid_len) ||
         (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) ||
         (kv_idx && (reinterpret_cast<uintptr_t>(kv_idx) & 3u)) ||
-        (kv_cnt && (reinterpret_cast<uintptr_t>(kv_cnt) & 3u)))
+        (kv_cnt && (reinterpret_cast<uintptr_t>(kv_cnt) & 3u)) ||
+        (pair_order && (reinterpret_cast<uintptr_t>(pair_order) & 3u)))
         return SBA_ERR_ALIGNMENT;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (D == 128)
         return launch_attention<128, 2>(q, k, v, o, lse, B, H, Npad, valid_len, kv_idx, kv_cnt, kmax,
-                                        dense, softmax_scale, s);
+                                        dense, pair_order, softmax_scale, s);
     return launch_attention<64, 4>(q, k, v, o, lse, B, H, Npad, valid_len, kv_idx, kv_cnt, kmax, dense,
-                                   softmax_scale, s);
+                                   pair_order, softmax_scale, s);
 }
 
 sba_status sba_attention(const void* q, const void* k, const void* v, void* o, float* lse, int B,
@@ -207,14 +211,23 @@ sba_status sba_attention(const void* q, const void* k, const void* v, void* o, f
                          const int32_t* kv_idx, const int32_t* kv_cnt, int kmax,
                          float softmax_scale, void* stream) {
     return attention_common(q, k, v, o, lse, B, H, Npad, D, valid_len, block, kv_idx, kv_cnt, kmax,
-                            0, softmax_scale, stream);
+                            0, nullptr, softmax_scale, stream);
+}
+
+sba_status sba_attention_paired(const void* q, const void* k, const void* v, void* o, float* lse,
+                                int B, int H, int Npad, int D, const int32_t* valid_len, int block,
+                                const int32_t* kv_idx, const int32_t* kv_cnt, int kmax,
+                                const int32_t* pair_order, float softmax_scale, void* stream) {
+    if (!pair_order) return SBA_ERR_INVALID_ARG;
+    return attention_common(q, k, v, o, lse, B, H, Npad, D, valid_len, block, kv_idx, kv_cnt, kmax,
+                            0, pair_order, softmax_scale, stream);
 }
 
 sba_status sba_dense_attention(const void* q, const void* k, const void* v, void* o, float* lse,
                                int B, int H, int Npad, int D, const int32_t* valid_len,
                                float softmax_scale, void* stream) {
     return attention_common(q, k, v, o, lse, B, H, Npad, D, valid_len, 64, nullptr, nullptr, 0, 1,
-                            softmax_scale, stream);
+                            nullptr, softmax_scale, stream);
 }
 
 sba_status sba_get_device_status(void* stream) {
@@ -245,6 +258,48 @@ const char* sba_strerror(sba_status status) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- query-block pairing
+extern "C" size_t sba_pair_workspace_size(int B, int H, int Npad, int block) {
+    if (check_shape(B, H, Npad, 64, block) != SBA_OK) return 0;
+    return sba::pair_workspace_bytes((size_t)B * H, (size_t)Npad / block);
+}
+
+extern "C" sba_status sba_pair_query_blocks(const int32_t* kv_idx, const int32_t* kv_cnt, int B, int H,
+                                            int Npad, int kmax, const int32_t* valid_len, int block,
+                                            int32_t* pair_order, void* workspace,
+                                            size_t workspace_bytes, void* stream) {
+    sba_status st = check_shape(B, H, Npad, 64, block);
+    if (st != SBA_OK) return st;
+    if (!kv_idx || !kv_cnt || !pair_order || !workspace || kmax <= 0) return SBA_ERR_INVALID_ARG;
+    const int nQ = Npad / block;
+    const size_t BH = (size_t)B * H;
+    if (workspace_bytes < sba::pair_workspace_bytes(BH, nQ)) return SBA_ERR_INVALID_ARG;
+    if (!aligned16(workspace) || !aligned16(valid_len) || (reinterpret_cast<uintptr_t>(kv_idx) & 3u) ||
+        (reinterpret_cast<uintptr_t>(kv_cnt) & 3u) || (reinterpret_cast<uintptr_t>(pair_order) & 3u))
+        return SBA_ERR_ALIGNMENT;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    sba::PairWorkspace ws = sba::carve_pair_workspace(workspace, BH, nQ);
+    const long long rows = (long long)BH * nQ;
+    const unsigned wgrid = (unsigned)((rows + 7) / 8);   // 8 warps per 256-thread CTA
+    sba::pair_bitmap_kernel<<<wgrid, 256, 8 * ((nQ + 31) / 32) * 4, s>>>(ws, kv_idx, kv_cnt, nQ, kmax, rows);
+    const int W = (nQ + 31) / 32;
+    const int tiles_per_bh = (nQ + sba::kPairWarps - 1) / sba::kPairWarps;
+    const size_t psmem = (size_t)sba::kPairSpan * W * 4;   // <= 136 x 128 x 4 = 68 KB
+    if (cudaFuncSetAttribute(sba::pair_propose_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)psmem) != cudaSuccess)
+        return SBA_ERR_CUDA;
+    const unsigned tgrid = (unsigned)((rows + 255) / 256);
+    sba::pair_propose_kernel<<<(unsigned)(BH * tiles_per_bh), 32 * sba::kPairWarps, psmem, s>>>(
+        ws, kv_cnt, valid_len, H, nQ, tiles_per_bh);
+    sba::pair_resolve_kernel<<<tgrid, 256, 0, s>>>(ws, nQ, rows);
+    for (int r = 1; r < sba::kPairRounds; ++r) {
+        sba::pair_repropose_kernel<<<tgrid, 256, 0, s>>>(ws, nQ, rows);
+        sba::pair_resolve_kernel<<<tgrid, 256, 0, s>>>(ws, nQ, rows);
+    }
+    sba::pair_emit_kernel<<<(unsigned)((BH + 7) / 8), 256, 0, s>>>(ws, valid_len, H, nQ, pair_order, (int)BH);
+    return cudaGetLastError() == cudaSuccess ? SBA_OK : SBA_ERR_CUDA;
+}
 
 // ---------------------------------------------------------------- routing without allocation
 // Scratch for sba_pool_select_noalloc: a fixed array in device memory that every

@@ -50,6 +50,13 @@ def lib() -> ctypes.CDLL:
         L.sba_block_means.argtypes = [vp, i32, i32, i32, i32, vp, i32, vp, vp]
         L.sba_attention.restype = i32
         L.sba_attention.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, i32, vp, vp, i32, f32, vp]
+        L.sba_pair_workspace_size.restype = sz
+        L.sba_pair_workspace_size.argtypes = [i32, i32, i32, i32]
+        L.sba_pair_query_blocks.restype = i32
+        L.sba_pair_query_blocks.argtypes = [vp, vp, i32, i32, i32, i32, vp, i32, vp, vp, sz, vp]
+        L.sba_attention_paired.restype = i32
+        L.sba_attention_paired.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, i32, vp, vp, i32, vp,
+                                           f32, vp]
         L.sba_dense_attention.restype = i32
         L.sba_dense_attention.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, f32, vp]
         L.sba_get_device_status.restype = i32
@@ -158,6 +165,38 @@ def attention(q, k, v, kv_idx, kv_cnt, valid_len=None, softmax_scale: float = 0.
     return out, lse
 
 
+def pair_query_blocks(kv_idx, kv_cnt, valid_len=None, block: int = BLOCK, pair_order=None,
+                      workspace=None, stream=None):
+    """Tiles of two query blocks with overlapping kept lists: int32 [B, H, 2*ceil(nQ/2)]."""
+    B, H, nQ, kmax = kv_idx.shape
+    Npad = nQ * block
+    if pair_order is None:
+        pair_order = torch.empty((B, H, 2 * ((nQ + 1) // 2)), dtype=torch.int32, device=kv_idx.device)
+    if workspace is None:
+        workspace = torch.empty(int(lib().sba_pair_workspace_size(B, H, Npad, block)), dtype=torch.uint8,
+                                device=kv_idx.device)
+    _check(lib().sba_pair_query_blocks(_ptr(kv_idx), _ptr(kv_cnt), B, H, Npad, kmax,
+                                       _ptr(_valid_len(valid_len, kv_idx.device)), block, _ptr(pair_order),
+                                       _ptr(workspace), workspace.numel(), _stream(stream)),
+           "sba_pair_query_blocks")
+    return pair_order
+
+
+def attention_paired(q, k, v, kv_idx, kv_cnt, pair_order, valid_len=None, softmax_scale: float = 0.0,
+                     out=None, lse=None, want_lse: bool = True, block: int = BLOCK, stream=None):
+    """sba_attention over the tiles of `pair_order`.  Returns (o bf16, lse fp32 or None)."""
+    B, H, Npad, D = _qkv(q, k, v)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H, Npad), dtype=torch.float32, device=q.device)
+    _check(lib().sba_attention_paired(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Npad, D,
+                                      _ptr(_valid_len(valid_len, q.device)), block, _ptr(kv_idx),
+                                      _ptr(kv_cnt), kv_idx.shape[-1], _ptr(pair_order), float(softmax_scale),
+                                      _stream(stream)), "sba_attention_paired")
+    return out, lse
+
+
 def dense_attention(q, k, v, valid_len=None, softmax_scale: float = 0.0, out=None, lse=None,
                     want_lse: bool = True, stream=None):
     """Dense attention over each sample's valid tokens.  Returns (o bf16, lse fp32 or None)."""
@@ -174,9 +213,11 @@ def dense_attention(q, k, v, valid_len=None, softmax_scale: float = 0.0, out=Non
 
 def sparse_attention(q, k, v, valid_len=None, sparsity: float = 0.75, softmax_scale: float = 0.0,
                      stream=None):
-    """The whole path: routing then block-sparse attention.  Returns (o, lse, kv_idx, kv_cnt)."""
+    """The whole path: routing, tile pairing, block-sparse attention.
+    Returns (o, lse, kv_idx, kv_cnt)."""
     kv_idx, kv_cnt = pool_select(q, k, valid_len, sparsity, stream=stream)
-    o, lse = attention(q, k, v, kv_idx, kv_cnt, valid_len, softmax_scale, stream=stream)
+    pair_order = pair_query_blocks(kv_idx, kv_cnt, valid_len, stream=stream)
+    o, lse = attention_paired(q, k, v, kv_idx, kv_cnt, pair_order, valid_len, softmax_scale, stream=stream)
     return o, lse, kv_idx, kv_cnt
 
 
