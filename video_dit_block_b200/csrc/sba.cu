@@ -13,6 +13,7 @@
 #include "attention.cuh"
 #include "common.cuh"
 #include "select.cuh"
+#include "score_mma.cuh"
 #include "pair.cuh"
 
 namespace {
@@ -132,32 +133,53 @@ sba_status sba_pool_select(const void* q, const void* k, int B, int H, int Npad,
     const long long groups = (long long)BH * nB;
     const int gpc = 256 / (D / 8);  // block groups per CTA
     const unsigned pool_grid = (unsigned)((groups + gpc - 1) / gpc);
-    // largest tile of query blocks whose score rows fit in shared memory
-    int TQ = 32;
-    while (TQ > 8 && sba::score_select_smem(D, TQ, nB) > 227 * 1024) TQ /= 2;
-    const size_t smem = sba::score_select_smem(D, TQ, nB);
-    if (smem > 227 * 1024) return SBA_ERR_UNSUPPORTED;
-    dim3 sgrid((nB + TQ - 1) / TQ, (unsigned)BH);
+    const int wpb = 8;              // top-k: one warp per routing row
+    const size_t tsmem = sba::topk_smem(wpb, ws.ld);
+    if (tsmem > 227 * 1024) return SBA_ERR_UNSUPPORTED;
+    const unsigned tgrid = (unsigned)((groups + wpb - 1) / wpb);
+    const auto* qb = static_cast<const __nv_bfloat16*>(q);
+    const auto* kb = static_cast<const __nv_bfloat16*>(k);
+    // scores are needed unless nothing is dropped for any sample
+    const bool need_scores = sparsity > 0.0;
+    CUtensorMap tqh, tql, tkh, tkl;
+    if (need_scores && (!make_map(&tqh, ws.qhi, (int)BH, nB, D, 128) || !make_map(&tql, ws.qlo, (int)BH, nB, D, 128) ||
+                        !make_map(&tkh, ws.khi, (int)BH, nB, D, 256) || !make_map(&tkl, ws.klo, (int)BH, nB, D, 256)))
+        return SBA_ERR_CUDA;
+    const dim3 sgrid((nB + 127) / 128, (nB + 255) / 256, (unsigned)BH);
     if (D == 128) {
-        sba::pool_kernel<128><<<pool_grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(q), valid_len, H, Npad,
-                                                        ws.qmean64, ws.qmean32, ws.qnorm, groups);
-        sba::pool_kernel<128><<<pool_grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(k), valid_len, H, Npad,
-                                                        ws.kmean64, ws.kmean32, ws.knorm, groups);
-        if (cudaFuncSetAttribute(sba::score_select_kernel<128>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        sba::pool_kernel<128><<<pool_grid, 256, 0, s>>>(qb, valid_len, H, Npad, ws.qmean64, ws.qhi, ws.qlo, ws.qnorm, groups);
+        sba::pool_kernel<128><<<pool_grid, 256, 0, s>>>(kb, valid_len, H, Npad, ws.kmean64, ws.khi, ws.klo, ws.knorm, groups);
+        sba::kmax_kernel<<<(unsigned)((BH + 7) / 8), 256, 0, s>>>(ws, valid_len, H, Npad, (int)BH);
+        if (need_scores) {
+            using SM = sba::ScoreSmem<128>;
+            if (cudaFuncSetAttribute(sba::score_mma_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     SM::kAlloc) != cudaSuccess)
+                return SBA_ERR_CUDA;
+            sba::score_mma_kernel<128><<<sgrid, 128, SM::kAlloc, s>>>(tqh, tql, tkh, tkl, ws.scores, nB, ws.ld,
+                                                                      g_wait_limit);
+        }
+        if (cudaFuncSetAttribute(sba::topk_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsmem) !=
+            cudaSuccess)
             return SBA_ERR_CUDA;
-        sba::score_select_kernel<128><<<sgrid, 256, smem, s>>>(ws, valid_len, H, Npad, sparsity, kmax,
-                                                               TQ, kv_idx, kv_cnt);
+        sba::topk_kernel<128><<<tgrid, 32 * wpb, tsmem, s>>>(ws, valid_len, H, Npad, sparsity, kmax, kv_idx, kv_cnt,
+                                                             groups);
     } else {
-        sba::pool_kernel<64><<<pool_grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(q), valid_len, H, Npad,
-                                                       ws.qmean64, ws.qmean32, ws.qnorm, groups);
-        sba::pool_kernel<64><<<pool_grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(k), valid_len, H, Npad,
-                                                       ws.kmean64, ws.kmean32, ws.knorm, groups);
-        if (cudaFuncSetAttribute(sba::score_select_kernel<64>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        sba::pool_kernel<64><<<pool_grid, 256, 0, s>>>(qb, valid_len, H, Npad, ws.qmean64, ws.qhi, ws.qlo, ws.qnorm, groups);
+        sba::pool_kernel<64><<<pool_grid, 256, 0, s>>>(kb, valid_len, H, Npad, ws.kmean64, ws.khi, ws.klo, ws.knorm, groups);
+        sba::kmax_kernel<<<(unsigned)((BH + 7) / 8), 256, 0, s>>>(ws, valid_len, H, Npad, (int)BH);
+        if (need_scores) {
+            using SM = sba::ScoreSmem<64>;
+            if (cudaFuncSetAttribute(sba::score_mma_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     SM::kAlloc) != cudaSuccess)
+                return SBA_ERR_CUDA;
+            sba::score_mma_kernel<64><<<sgrid, 128, SM::kAlloc, s>>>(tqh, tql, tkh, tkl, ws.scores, nB, ws.ld,
+                                                                     g_wait_limit);
+        }
+        if (cudaFuncSetAttribute(sba::topk_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsmem) !=
+            cudaSuccess)
             return SBA_ERR_CUDA;
-        sba::score_select_kernel<64><<<sgrid, 256, smem, s>>>(ws, valid_len, H, Npad, sparsity, kmax,
-                                                              TQ, kv_idx, kv_cnt);
+        sba::topk_kernel<64><<<tgrid, 32 * wpb, tsmem, s>>>(ws, valid_len, H, Npad, sparsity, kmax, kv_idx, kv_cnt,
+                                                            groups);
     }
     return cudaGetLastError() == cudaSuccess ? SBA_OK : SBA_ERR_CUDA;
 }
@@ -174,10 +196,10 @@ sba_status sba_block_means(const void* x, int B, int H, int Npad, int D, const i
     const unsigned grid = (unsigned)((groups + gpc - 1) / gpc);
     if (D == 128)
         sba::pool_kernel<128><<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), valid_len, H,
-                                                   Npad, out, nullptr, nullptr, groups);
+                                                   Npad, out, nullptr, nullptr, nullptr, groups);
     else
         sba::pool_kernel<64><<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), valid_len, H,
-                                                  Npad, out, nullptr, nullptr, groups);
+                                                  Npad, out, nullptr, nullptr, nullptr, groups);
     return cudaGetLastError() == cudaSuccess ? SBA_OK : SBA_ERR_CUDA;
 }
 

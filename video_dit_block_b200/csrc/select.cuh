@@ -27,42 +27,57 @@ namespace sba {
 constexpr int kBlock = 64;
 
 // Workspace layout of sba_pool_select (all offsets 256-byte aligned):
-//   qmean64, kmean64 : double [BH][nB][D]
-//   qmean32, kmean32 : float  [BH][nBc][D][64], nBc = ceil(nB / 64): block means
-//                      rounded to fp32, transposed in chunks of 64 blocks so the
-//                      scoring kernel stages them with straight copies
-//   qnorm,   knorm   : double [BH][nB]    (Euclidean norm of each block mean)
+//   qmean64, kmean64 : double [BH][nB][D]   block means
+//   qhi, qlo, khi, klo : bf16 [BH][nB][D]   hi/lo split of the means for the screen
+//   qnorm, knorm     : double [BH][nB]      Euclidean norm of each block mean
+//   kmaxn            : double [BH]          largest key-block norm of the sample
+//   scores           : float [BH][nB][ld]   screened scores, ld = 64 * ceil(nB / 64)
 struct SelectWorkspace {
     double* qmean64;
     double* kmean64;
-    float* qmean32;
-    float* kmean32;
+    __nv_bfloat16* qhi;
+    __nv_bfloat16* qlo;
+    __nv_bfloat16* khi;
+    __nv_bfloat16* klo;
     double* qnorm;
     double* knorm;
+    double* kmaxn;
+    float* scores;
+    int ld;
 };
 
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+__host__ __device__ inline size_t select_score_ld(size_t nB) { return (nB + 63) / 64 * 64; }
+
 __host__ __device__ inline size_t select_workspace_bytes(size_t BH, size_t nB, size_t D) {
-    size_t m64 = align256(BH * nB * D * sizeof(double));
-    size_t m32 = align256(BH * ((nB + 63) / 64) * 64 * D * sizeof(float));
-    size_t nrm = align256(BH * nB * sizeof(double));
-    return 2 * (m64 + m32 + nrm);
+    const size_t m64 = align256(BH * nB * D * sizeof(double));
+    const size_t m16 = align256(BH * nB * D * 2);
+    const size_t nrm = align256(BH * nB * sizeof(double));
+    const size_t kmx = align256(BH * sizeof(double));
+    const size_t sco = align256(BH * nB * select_score_ld(nB) * sizeof(float));
+    return 2 * m64 + 4 * m16 + 2 * nrm + kmx + sco;
 }
 
 __host__ __device__ inline SelectWorkspace carve_select_workspace(void* base, size_t BH, size_t nB,
                                                                   size_t D) {
     char* p = static_cast<char*>(base);
-    size_t m64 = align256(BH * nB * D * sizeof(double));
-    size_t m32 = align256(BH * ((nB + 63) / 64) * 64 * D * sizeof(float));
-    size_t nrm = align256(BH * nB * sizeof(double));
+    const size_t m64 = align256(BH * nB * D * sizeof(double));
+    const size_t m16 = align256(BH * nB * D * 2);
+    const size_t nrm = align256(BH * nB * sizeof(double));
+    const size_t kmx = align256(BH * sizeof(double));
     SelectWorkspace w;
     w.qmean64 = reinterpret_cast<double*>(p); p += m64;
     w.kmean64 = reinterpret_cast<double*>(p); p += m64;
-    w.qmean32 = reinterpret_cast<float*>(p); p += m32;
-    w.kmean32 = reinterpret_cast<float*>(p); p += m32;
+    w.qhi = reinterpret_cast<__nv_bfloat16*>(p); p += m16;
+    w.qlo = reinterpret_cast<__nv_bfloat16*>(p); p += m16;
+    w.khi = reinterpret_cast<__nv_bfloat16*>(p); p += m16;
+    w.klo = reinterpret_cast<__nv_bfloat16*>(p); p += m16;
     w.qnorm = reinterpret_cast<double*>(p); p += nrm;
-    w.knorm = reinterpret_cast<double*>(p);
+    w.knorm = reinterpret_cast<double*>(p); p += nrm;
+    w.kmaxn = reinterpret_cast<double*>(p); p += kmx;
+    w.scores = reinterpret_cast<float*>(p);
+    w.ld = (int)select_score_ld(nB);
     return w;
 }
 
@@ -87,13 +102,14 @@ __device__ __forceinline__ int sample_len(const int32_t* valid_len, int b, int N
 // ------------------------------------------------------------------ pooling
 // One group of D/8 lanes per (bh, block): lane g owns channels [8g, 8g+8) and
 // walks the block's valid rows in token order, 16-byte loads, fp64 sums.
-// Writes the fp64 mean and, when the pointers are non-null, its fp32 rounding
-// (chunk-transposed layout) and the norm of the block mean.
+// Writes the fp64 mean and, when the pointers are non-null, its bf16 hi/lo split
+// and the norm of the block mean.
 template <int D>
 __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restrict__ x,
                                                    const int32_t* __restrict__ valid_len, int H,
                                                    int Npad, double* __restrict__ mean64,
-                                                   float* __restrict__ mean32,
+                                                   __nv_bfloat16* __restrict__ hi16,
+                                                   __nv_bfloat16* __restrict__ lo16,
                                                    double* __restrict__ norm, long long n_groups) {
     constexpr int LPB = D / 8;  // lanes per block group
     constexpr int UNROLL = 16;
@@ -148,11 +164,21 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
     for (int e = 0; e < 8; e += 2) {
         *reinterpret_cast<double2*>(dst64 + e) = make_double2(m[e], m[e + 1]);
     }
-    if (mean32) {
-        const int nBc = (nB + 63) / 64;
-        float* dst32 = mean32 + (((size_t)bh * nBc + I / 64) * D + 8 * g) * 64 + (I % 64);
+    if (hi16) {
+        // hi = bf16(mean), lo = bf16(mean - hi): the split the tensor-core screen uses
+        uint32_t ph[4], pl[4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) dst32[(size_t)e * 64] = (float)m[e];
+        for (int e = 0; e < 8; e += 2) {
+            const __nv_bfloat16 h0 = __float2bfloat16_rn((float)m[e]);
+            const __nv_bfloat16 h1 = __float2bfloat16_rn((float)m[e + 1]);
+            const __nv_bfloat16 l0 = __float2bfloat16_rn((float)(m[e] - (double)__bfloat162float(h0)));
+            const __nv_bfloat16 l1 = __float2bfloat16_rn((float)(m[e + 1] - (double)__bfloat162float(h1)));
+            __nv_bfloat162 hh = __halves2bfloat162(h0, h1), ll = __halves2bfloat162(l0, l1);
+            ph[e / 2] = *reinterpret_cast<uint32_t*>(&hh);
+            pl[e / 2] = *reinterpret_cast<uint32_t*>(&ll);
+        }
+        *reinterpret_cast<uint4*>(hi16 + (size_t)grp * D + 8 * g) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
+        *reinterpret_cast<uint4*>(lo16 + (size_t)grp * D + 8 * g) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
     }
     if (norm && g == 0) norm[grp] = sqrt(sq);
 }
@@ -293,220 +319,174 @@ __device__ uint64_t warp_radix_select64(int n, int k, uint32_t* hist, KeyOf key_
     return prefix;
 }
 
-// Shared-memory bytes of score_select_kernel for a tile of TQ query blocks.
-__host__ __device__ inline size_t score_select_smem(int D, int TQ, int nBmax) {
-    const int nBpad = ((nBmax + 63) / 64) * 64;
-    return (size_t)D * TQ * 4 + (size_t)D * 64 * 4 + (size_t)TQ * nBpad * 4 + 8 * 256 * 4 +
-           8 * 32 * 4 + (size_t)TQ * 8 + 16;
+// Largest key-block-mean norm of each (b, h) over its sample's blocks; one warp each.
+__global__ void kmax_kernel(SelectWorkspace ws, const int32_t* __restrict__ valid_len, int H, int Npad,
+                            int BH) {
+    const int bh = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+    const int lane = threadIdx.x & 31;
+    if (bh >= BH) return;
+    const int nBmax = Npad / kBlock;
+    const int nB = (sample_len(valid_len, bh / H, Npad) + kBlock - 1) / kBlock;
+    double m = 0.0;
+    for (int j = lane; j < nB; j += 32) m = fmax(m, ws.knorm[(size_t)bh * nBmax + j]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, off));
+    if (lane == 0) ws.kmaxn[bh] = m;
 }
 
-// Scores and top-k routing for TQ (8, 16 or 32) consecutive query blocks of one
-// (b, h) = blockIdx.y; 256 threads.  Phase 1 computes fp32 scores of all key
-// blocks into shared memory (warp w owns rows 4w..4w+3, lane owns columns
-// 2*lane, 2*lane+1 of each 64-block chunk).  Phase 2: one warp per row selects.
+// Shared-memory bytes of topk_kernel for `warps` warps per CTA.
+__host__ __device__ inline size_t topk_smem(int warps, int ld) {
+    return (size_t)warps * ((size_t)ld * 4 + 256 * 4 + 32 * 4);
+}
+
+// Top-k routing of one (b, h, I) row per warp, from the screened scores.
+//
+// Screen error.  The scores come from score_mma_kernel: S = qhi.khi + qhi.klo +
+// qlo.khi in fp32, with hi = bf16(x), lo = bf16(x - hi) (each through fp32).  Per
+// term d the dropped parts (qlo.klo and the remainders of the split) are below
+// 4 * 2^-16 |qbar_d kbar_d|; the products are exact in fp32 and the accumulation
+// of the 3D products in fp32 adds at most 3D * 2^-22 of sum |qbar_d kbar_d| (two
+// units in the last place per addition, whatever the order).  With Cauchy-Schwarz,
+// |S - qbar.kbar| <= (4 * 2^-16 + 3D * 2^-22) |qbar_I| max_J |kbar_J|, doubled here
+// for margin, plus an absolute term for values in the subnormal range.
 template <int D>
-__global__ void __launch_bounds__(256) score_select_kernel(
-    SelectWorkspace ws, const int32_t* __restrict__ valid_len, int H, int Npad, double sparsity,
-    int kmax, int TQ, int32_t* __restrict__ kv_idx, int32_t* __restrict__ kv_cnt) {
+__global__ void __launch_bounds__(256) topk_kernel(SelectWorkspace ws, const int32_t* __restrict__ valid_len,
+                                                   int H, int Npad, double sparsity, int kmax,
+                                                   int32_t* __restrict__ kv_idx, int32_t* __restrict__ kv_cnt,
+                                                   long long rows) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int wpb = blockDim.x >> 5;
+    const long long rid = (long long)blockIdx.x * wpb + warp;
+    if (rid >= rows) return;
     const int nBmax = Npad / kBlock;
-    const int nBc = (nBmax + 63) / 64;
-    const int nBpad = nBc * 64;
-    const int bh = blockIdx.y;
-    const int b = bh / H;
-    const int L = sample_len(valid_len, b, Npad);
+    const int ld = ws.ld;
+    const long long bh = rid / nBmax;
+    const int I = (int)(rid % nBmax);
+    const int L = sample_len(valid_len, (int)(bh / H), Npad);
     const int nB = (L + kBlock - 1) / kBlock;
     const int k = keep_count(nB, sparsity);
-    const int I0 = blockIdx.x * TQ;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    int32_t* cnt_out = kv_cnt + (size_t)bh * nBmax;
-    int32_t* idx_out = kv_idx + (size_t)bh * nBmax * kmax;
-
-    int nrows = nBmax - I0;
-    nrows = nrows > TQ ? TQ : nrows;
-    int nact = nB - I0;  // rows with I < nB
-    nact = nact < 0 ? 0 : (nact > nrows ? nrows : nact);
-    for (int r = nact + tid; r < nrows; r += 256) cnt_out[I0 + r] = 0;
-    if (nact == 0) return;
-    if (k >= nB) {  // nothing dropped: every block, ascending
-        for (int r = warp; r < nact; r += 8) {
-            int32_t* out = idx_out + (size_t)(I0 + r) * kmax;
-            for (int j = lane; j < nB; j += 32) out[j] = j;
-            if (lane == 0) cnt_out[I0 + r] = nB;
-        }
+    int32_t* out = kv_idx + (size_t)rid * kmax;
+    if (I >= nB) {
+        if (lane == 0) kv_cnt[rid] = 0;
         return;
     }
-
-    float* sq = reinterpret_cast<float*>(smem_raw);          // [D][TQ]
-    float* sk = sq + D * TQ;                                  // [D][64]
-    float* ssc = sk + D * 64;                                 // [TQ][nBpad]
-    uint32_t* hist = reinterpret_cast<uint32_t*>(ssc + (size_t)TQ * nBpad);  // [8][256]
-    int32_t* slots = reinterpret_cast<int32_t*>(hist + 8 * 256);             // [8][32]
-    double* qn = reinterpret_cast<double*>(slots + 8 * 32);                  // [TQ]
-    double* kmaxn = qn + TQ;                                                 // [1]
-
-    // stage the fp32 query means of this tile: [D][TQ] from the [D][64] chunk layout
-    const float* qsrc = ws.qmean32 + ((size_t)bh * nBc + I0 / 64) * D * 64 + (I0 % 64);
-    for (int i = tid; i < D * TQ; i += 256) {
-        const int d = i / TQ, r = i % TQ;
-        sq[i] = qsrc[(size_t)d * 64 + r];
+    if (k >= nB) {  // nothing dropped: every block, ascending
+        for (int j = lane; j < nB; j += 32) out[j] = j;
+        if (lane == 0) kv_cnt[rid] = nB;
+        return;
     }
-    for (int r = tid; r < TQ; r += 256) qn[r] = r < nact ? ws.qnorm[(size_t)bh * nBmax + I0 + r] : 0.0;
-    if (warp == 0) {  // largest key-block mean norm over the sample's blocks
-        double m = 0.0;
-        for (int j = lane; j < nB; j += 32) m = fmax(m, ws.knorm[(size_t)bh * nBmax + j]);
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, off));
-        if (lane == 0) *kmaxn = m;
-    }
-
-    // phase 1: fp32 scores, chunk by chunk of 64 key blocks
-    const int nchunks = (nB + 63) / 64;
-    const float* ksrc = ws.kmean32 + (size_t)bh * nBc * D * 64;
-    for (int c = 0; c < nchunks; ++c) {
-        __syncthreads();
-        const float4* src4 = reinterpret_cast<const float4*>(ksrc + (size_t)c * D * 64);
-        float4* dst4 = reinterpret_cast<float4*>(sk);
-        for (int i = tid; i < D * 16; i += 256) dst4[i] = __ldg(src4 + i);
-        __syncthreads();
-        if (4 * warp < TQ) {
-            float acc[4][2];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = 0.f;
-#pragma unroll 8
-            for (int d = 0; d < D; ++d) {
-                const float4 q4 = *reinterpret_cast<const float4*>(sq + d * TQ + 4 * warp);
-                const float2 k2 = *reinterpret_cast<const float2*>(sk + d * 64 + 2 * lane);
-                acc[0][0] = fmaf(q4.x, k2.x, acc[0][0]);
-                acc[0][1] = fmaf(q4.x, k2.y, acc[0][1]);
-                acc[1][0] = fmaf(q4.y, k2.x, acc[1][0]);
-                acc[1][1] = fmaf(q4.y, k2.y, acc[1][1]);
-                acc[2][0] = fmaf(q4.z, k2.x, acc[2][0]);
-                acc[2][1] = fmaf(q4.z, k2.y, acc[2][1]);
-                acc[3][0] = fmaf(q4.w, k2.x, acc[3][0]);
-                acc[3][1] = fmaf(q4.w, k2.y, acc[3][1]);
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                *reinterpret_cast<float2*>(ssc + (size_t)(4 * warp + i) * nBpad + c * 64 + 2 * lane) =
-                    make_float2(acc[i][0], acc[i][1]);
-        }
-    }
-    __syncthreads();
-
-    // phase 2: per-row selection, one warp per row
+    float* row = reinterpret_cast<float*>(smem_raw + (size_t)warp * ((size_t)ld * 4 + 256 * 4 + 32 * 4));
+    uint32_t* whist = reinterpret_cast<uint32_t*>(row + ld);
+    int32_t* wslots = reinterpret_cast<int32_t*>(whist + 256);
+    const float* src = ws.scores + (size_t)rid * ld;
+    for (int j = lane; j < nB; j += 32) row[j] = __ldg(src + j);
+    __syncwarp();
     const double inv = __ddiv_rn(1.0, __dsqrt_rn((double)D));
-    uint32_t* whist = hist + warp * 256;
-    int32_t* wslots = slots + warp * 32;
-    for (int r = warp; r < nact; r += 8) {
-        const int I = I0 + r;
-        const float* row = ssc + (size_t)r * nBpad;
-        const double* qrow64 = ws.qmean64 + ((size_t)bh * nBmax + I) * D;
-        const double* kbase64 = ws.kmean64 + (size_t)bh * nBmax * D;
-        int32_t* out = idx_out + (size_t)I * kmax;
+    const double qn = ws.qnorm[rid];
+    const double kmx = ws.kmaxn[bh];
+    const double* qrow64 = ws.qmean64 + (size_t)rid * D;
+    const double* kbase64 = ws.kmean64 + (size_t)bh * nBmax * D;
 
-        // k-th largest fp32 score
-        const uint32_t tau_key = warp_radix_select32(nB, k, whist, [&](int j, bool& ok) {
-            ok = true;
-            return f32_key(row[j]);
-        });
-        const double tau = (double)key_to_f32(tau_key);
-        // Error bound of an fp32 score against the fp64 one: D fused multiply-adds
-        // plus the two fp32 roundings of the means give (D + 3) u sum|q_d k_d|
-        // <= (D + 3) u |qbar| |kbar| (Cauchy-Schwarz), u = 2^-24; doubled for
-        // margin, plus an absolute term for gradual underflow.
-        const double delta = 2.0 * (D + 4) * 0x1p-24 * qn[r] * (*kmaxn) + D * 0x1p-126;
-        const double hi = tau + 2.0 * delta, lo = tau - 2.0 * delta;
+    // k-th largest fp32 score
+    const uint32_t tau_key = warp_radix_select32(nB, k, whist, [&](int j, bool& ok) {
+        ok = true;
+        return f32_key(row[j]);
+    });
+    const double tau = (double)key_to_f32(tau_key);
+    // screen error bound (see above); the band [tau - 2 delta, tau + 2 delta] is
+    // decided in fp64, everything above it is kept and everything below dropped
+    const double delta = 2.0 * (4.0 * 0x1p-16 + 3.0 * D * 0x1p-22) * qn * kmx +
+                         3.0 * D * 0x1p-120 * (1.0 + qn + kmx);
+    const double hi = tau + 2.0 * delta, lo = tau - 2.0 * delta;
 
-        int n_in = 0, n_band = 0;
+    int n_in = 0, n_band = 0;
+    for (int j0 = 0; j0 < nB; j0 += 32) {
+        const int j = j0 + lane;
+        const double f = j < nB ? (double)row[j] : -INFINITY;
+        const bool in_a = j < nB && f > hi;
+        const bool in_b = j < nB && !in_a && f >= lo;
+        n_in += __popc(__ballot_sync(0xffffffffu, in_a));
+        n_band += __popc(__ballot_sync(0xffffffffu, in_b));
+    }
+    const int need = k - n_in;  // band members to keep, 1 <= need <= n_band
+
+    // mode 0: keep the whole band; 1: small band ranked in registers; 2: wide band
+    int mode = need >= n_band ? 0 : (n_band <= 32 ? 1 : 2);
+    uint32_t chosen_mask = 0xffffffffu;
+    uint64_t tau_x = 0;
+    int eq_take = 0;
+    if (mode == 1) {
+        int base = 0;
         for (int j0 = 0; j0 < nB; j0 += 32) {
             const int j = j0 + lane;
             const double f = j < nB ? (double)row[j] : -INFINITY;
-            const bool in_a = j < nB && f > hi;
-            const bool in_b = j < nB && !in_a && f >= lo;
-            n_in += __popc(__ballot_sync(0xffffffffu, in_a));
-            n_band += __popc(__ballot_sync(0xffffffffu, in_b));
-        }
-        const int need = k - n_in;  // band members to keep, 1 <= need <= n_band
-
-        // mode 0: keep the whole band; 1: small band ranked in registers; 2: wide band
-        int mode = need >= n_band ? 0 : (n_band <= 32 ? 1 : 2);
-        uint32_t chosen_mask = 0xffffffffu;
-        uint64_t tau_x = 0;
-        int eq_take = 0;
-        if (mode == 1) {
-            int base = 0;
-            for (int j0 = 0; j0 < nB; j0 += 32) {
-                const int j = j0 + lane;
-                const double f = j < nB ? (double)row[j] : -INFINITY;
-                const bool in_b = j < nB && !(f > hi) && f >= lo;
-                const uint32_t bb = __ballot_sync(0xffffffffu, in_b);
-                if (in_b) wslots[base + __popc(bb & lanemask_lt())] = j;
-                base += __popc(bb);
-            }
-            __syncwarp();
-            const int myj = lane < n_band ? wslots[lane] : 0;
-            const double my_s = lane < n_band ? exact_score(qrow64, kbase64 + (size_t)myj * D, D, inv)
-                                              : -INFINITY;
-            int rank = 0;
-            for (int t = 0; t < n_band; ++t) {
-                const double s_t = __shfl_sync(0xffffffffu, my_s, t);
-                const int j_t = __shfl_sync(0xffffffffu, myj, t);
-                rank += (s_t > my_s || (s_t == my_s && j_t < myj)) ? 1 : 0;
-            }
-            chosen_mask = __ballot_sync(0xffffffffu, lane < n_band && rank < need);
-            __syncwarp();
-        } else if (mode == 2) {
-            auto band_key = [&](int j, bool& ok) -> uint64_t {
-                const double f = (double)row[j];
-                ok = !(f > hi) && f >= lo;
-                return ok ? f64_key(exact_score(qrow64, kbase64 + (size_t)j * D, D, inv)) : 0ull;
-            };
-            tau_x = warp_radix_select64(nB, need, whist, band_key);
-            int gt = 0;
-            for (int j0 = 0; j0 < nB; j0 += 32) {
-                const int j = j0 + lane;
-                bool ok = false;
-                uint64_t x = 0;
-                if (j < nB) x = band_key(j, ok);
-                gt += __popc(__ballot_sync(0xffffffffu, ok && x > tau_x));
-            }
-            eq_take = need - gt;
-        }
-
-        // emit the kept blocks in ascending order
-        int pos = 0, band_seen = 0, eq_seen = 0;
-        for (int j0 = 0; j0 < nB; j0 += 32) {
-            const int j = j0 + lane;
-            const double f = j < nB ? (double)row[j] : -INFINITY;
-            const bool in_a = j < nB && f > hi;
-            const bool in_b = j < nB && !in_a && f >= lo;
+            const bool in_b = j < nB && !(f > hi) && f >= lo;
             const uint32_t bb = __ballot_sync(0xffffffffu, in_b);
-            bool sel = in_a;
-            if (mode == 0) {
-                sel = sel || in_b;
-            } else if (mode == 1) {
-                const int slot = band_seen + __popc(bb & lanemask_lt());
-                sel = sel || (in_b && ((chosen_mask >> slot) & 1u));
-            } else {
-                uint64_t x = 0;
-                if (in_b) x = f64_key(exact_score(qrow64, kbase64 + (size_t)j * D, D, inv));
-                const bool eq = in_b && x == tau_x;
-                const uint32_t eb = __ballot_sync(0xffffffffu, eq);
-                const int eq_rank = eq_seen + __popc(eb & lanemask_lt());
-                sel = sel || (in_b && x > tau_x) || (eq && eq_rank < eq_take);
-                eq_seen += __popc(eb);
-            }
-            band_seen += __popc(bb);
-            const uint32_t sb = __ballot_sync(0xffffffffu, sel);
-            if (sel) out[pos + __popc(sb & lanemask_lt())] = j;
-            pos += __popc(sb);
-        }
-        if (lane == 0) {
-            cnt_out[I] = pos;
-            if (pos != k) raise_device_error(kErrBadRouting);
+            if (in_b) wslots[base + __popc(bb & lanemask_lt())] = j;
+            base += __popc(bb);
         }
         __syncwarp();
+        const int myj = lane < n_band ? wslots[lane] : 0;
+        const double my_s = lane < n_band ? exact_score(qrow64, kbase64 + (size_t)myj * D, D, inv)
+                                          : -INFINITY;
+        int rank = 0;
+        for (int t = 0; t < n_band; ++t) {
+            const double s_t = __shfl_sync(0xffffffffu, my_s, t);
+            const int j_t = __shfl_sync(0xffffffffu, myj, t);
+            rank += (s_t > my_s || (s_t == my_s && j_t < myj)) ? 1 : 0;
+        }
+        chosen_mask = __ballot_sync(0xffffffffu, lane < n_band && rank < need);
+        __syncwarp();
+    } else if (mode == 2) {
+        auto band_key = [&](int j, bool& ok) -> uint64_t {
+            const double f = (double)row[j];
+            ok = !(f > hi) && f >= lo;
+            return ok ? f64_key(exact_score(qrow64, kbase64 + (size_t)j * D, D, inv)) : 0ull;
+        };
+        tau_x = warp_radix_select64(nB, need, whist, band_key);
+        int gt = 0;
+        for (int j0 = 0; j0 < nB; j0 += 32) {
+            const int j = j0 + lane;
+            bool ok = false;
+            uint64_t x = 0;
+            if (j < nB) x = band_key(j, ok);
+            gt += __popc(__ballot_sync(0xffffffffu, ok && x > tau_x));
+        }
+        eq_take = need - gt;
+    }
+
+    // emit the kept blocks in ascending order
+    int pos = 0, band_seen = 0, eq_seen = 0;
+    for (int j0 = 0; j0 < nB; j0 += 32) {
+        const int j = j0 + lane;
+        const double f = j < nB ? (double)row[j] : -INFINITY;
+        const bool in_a = j < nB && f > hi;
+        const bool in_b = j < nB && !in_a && f >= lo;
+        const uint32_t bb = __ballot_sync(0xffffffffu, in_b);
+        bool sel = in_a;
+        if (mode == 0) {
+            sel = sel || in_b;
+        } else if (mode == 1) {
+            const int slot = band_seen + __popc(bb & lanemask_lt());
+            sel = sel || (in_b && ((chosen_mask >> slot) & 1u));
+        } else {
+            uint64_t x = 0;
+            if (in_b) x = f64_key(exact_score(qrow64, kbase64 + (size_t)j * D, D, inv));
+            const bool eq = in_b && x == tau_x;
+            const uint32_t eb = __ballot_sync(0xffffffffu, eq);
+            const int eq_rank = eq_seen + __popc(eb & lanemask_lt());
+            sel = sel || (in_b && x > tau_x) || (eq && eq_rank < eq_take);
+            eq_seen += __popc(eb);
+        }
+        band_seen += __popc(bb);
+        const uint32_t sb = __ballot_sync(0xffffffffu, sel);
+        if (sel) out[pos + __popc(sb & lanemask_lt())] = j;
+        pos += __popc(sb);
+    }
+    if (lane == 0) {
+        kv_cnt[rid] = pos;
+        if (pos != k) raise_device_error(kErrBadRouting);
     }
 }
 
