@@ -49,9 +49,10 @@ def parse():
 
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one attention launch,
-# from the ncu capture summarised in profiles/attn_kernel_480p_dense.md, and the hash
+# from the ncu captures summarised in profiles/attn_kernel_*.md, and the hash
 # of the kernel sources it was taken with.  Reported only while the sources match.
-ATTN_TRAFFIC = {"480p_dense": (636370688 + 190253568, "33c27d24287ca6f9")}
+ATTN_TRAFFIC = {"480p_dense": (632697856 + 189443072, "f94215845bc4f30c"),
+                "720p": (3019749376 + 805242368, "f94215845bc4f30c")}
 KERNEL_SOURCES = ("video_dit_block_b200/csrc/attention.cuh", "video_dit_block_b200/csrc/ptx.cuh",
                   "video_dit_block_b200/csrc/common.cuh")
 
