@@ -139,6 +139,21 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def max_over_ranks(values, dist=None, device=None):
+    """Element-wise maximum of a list of floats over all ranks (identity without a
+    process group).  Every rank calls it at the same point."""
+    import torch
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if dist is not None and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
+def whole_job_value(kept_flops_per_rank, ms_per_step, world):
+    """Whole-job TFLOP/s: every rank runs one replica of the workload."""
+    return world * kept_flops_per_rank / (ms_per_step * 1e-3) / 1e12
+
+
 def oracle_sample(w, target_s=10.0, seed=0):
     """Time the fp64 oracle, as it stands, on a bounded sample of the workload: the
     full routing of head (b=0, h=0) and the attention of a seeded subset of that head's
@@ -298,12 +313,9 @@ def run_ours(args):
     attn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
     if sba.device_status(stream) != 0:
         raise RuntimeError("device status error in the timed region")
-    vals = torch.tensor([total_ms, attn_ms, sel_ms], dtype=torch.float64, device=dev)
-    if dist is not None:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    total_ms, attn_ms, sel_ms = (float(x) for x in vals.cpu())
+    total_ms, attn_ms, sel_ms = max_over_ranks([total_ms, attn_ms, sel_ms], dist, dev)
     ms_step = total_ms / K
-    value = world * f_step / (ms_step * 1e-3) / 1e12
+    value = whole_job_value(f_step, ms_step, world)
 
     # ---- end to end through the public API with host buffers
     e2e = None
@@ -328,12 +340,9 @@ def run_ours(args):
             oh.copy_(o, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize(dev)
-        e_ms = torch.tensor([e0.elapsed_time(e1) / Ke], dtype=torch.float64, device=dev)
-        if dist is not None:
-            dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
-        e_ms = float(e_ms.item())
+        e_ms = max_over_ranks([e0.elapsed_time(e1) / Ke], dist, dev)[0]
         bi = 3 * q.numel() * 2 + vl.numel() * 4
-        e2e = {"value": world * f_step / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e2e = {"value": whole_job_value(f_step, e_ms, world), "unit": "TFLOP/s",
                "ms_per_step": e_ms, "h2d_bytes_per_step": bi, "d2h_bytes_per_step": o.numel() * 2}
 
     if rank != 0:
