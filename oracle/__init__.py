@@ -50,6 +50,9 @@ def _load():
         _lib.oracle_select.restype = i32
         _lib.oracle_select.argtypes = [vp, vp, i32, i32, i32, i32, vp, i32, f64, i32, vp, vp,
                                        vp, vp, vp]
+        _lib.oracle_select_lse.restype = i32
+        _lib.oracle_select_lse.argtypes = [vp, vp, i32, i32, i32, i32, vp, i32, i32, f64, i32, i32, vp,
+                                           vp, vp]
         _lib.oracle_attention.restype = i32
         _lib.oracle_attention.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, i32, vp, vp, i32,
                                           f64, vp, i32, vp, vp]
@@ -149,6 +152,35 @@ def select(q, k, valid_len=None, sparsity: float = 0.0, kmax: int | None = None,
     if return_intermediates:
         return idx, cnt, pq, pk, S
     return idx, cnt
+
+
+def keep_count_budget(n_blocks: int, sparsity: float, budget: int = 1) -> int:
+    """keep(n, s) rounded up to a multiple of `budget`, at most n."""
+    k = keep_count(n_blocks, sparsity)
+    if budget > 1:
+        k = min(int(n_blocks), -(-k // budget) * budget)
+    return k
+
+
+def select_lse(q, k, valid_len=None, sparsity: float = 0.0, nsub: int = 4, budget: int = 1,
+               kmax: int | None = None, block: int = 64, return_scores: bool = False):
+    """Sub-block log-sum-exp router: (kv_idx, kv_cnt[, scores [B,H,nB,nB]])."""
+    q, k = _bf16(q), _bf16(k)
+    B, H, Npad, D = q.shape
+    vl = _vl(valid_len, B, Npad)
+    if kmax is None:
+        kmax = max(keep_count_budget(n_blocks(L, block), sparsity, budget) for L in vl)
+    nB = Npad // block
+    idx = np.empty((B, H, nB, kmax), dtype=np.int32)
+    cnt = np.empty((B, H, nB), dtype=np.int32)
+    S = np.empty((B, H, nB, nB)) if return_scores else None
+    st = _load().oracle_select_lse(_p(q), _p(k), B, H, Npad, D, _p(vl), block, nsub, float(sparsity),
+                                   int(budget), kmax, _p(idx), _p(cnt), _p(S))
+    if st == -2:
+        raise ValueError("nsub must divide the block size and be at most 16")
+    if st != 0:
+        raise ValueError("kmax smaller than the kept count")
+    return (idx, cnt, S) if return_scores else (idx, cnt)
 
 
 def attention(q, k, v, kv_idx, kv_cnt, valid_len=None, scale: float = 0.0, block: int = 64,

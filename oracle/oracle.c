@@ -317,3 +317,105 @@ int oracle_probs(const uint16_t* q, const uint16_t* k, const uint16_t* v,
     free(tok); free(buf); free(orow);
     return st;
 }
+
+/* ---------------------------------------------------------------------------
+ * Sub-block log-sum-exp router (the SubBlock router with n_q = n_k = nsub).
+ * Same page and section as above: each 64-token block is split into nsub
+ * sub-blocks of block/nsub tokens; pooling and a log-sum-exp estimate the
+ * unnormalised softmax mass of each key block for each query block and head:
+ *   score(I, J) = log sum_{a,b} c_{I,a} c_{J,b} exp(qbar_{I,a} . kbar_{J,b} / sqrt(D))
+ * where qbar_{I,a} is the mean of the valid q rows of sub-block a of block I and
+ * c_{I,a} their count (empty sub-blocks contribute nothing).  The kept count is
+ * keep(nB, s), optionally rounded up to a multiple of `budget` (at most nB).
+ * The log-sum-exp is evaluated as m + log(sum exp(x - m)), m = max x.
+ * ------------------------------------------------------------------------- */
+int oracle_select_lse(const uint16_t* q, const uint16_t* k, int B, int H, int Npad, int D,
+                      const int32_t* valid_len, int block, int nsub, double sparsity, int budget,
+                      int kmax, int32_t* kv_idx, int32_t* kv_cnt, double* scores) {
+    if (nsub < 1 || nsub > 16 || block % nsub != 0) return -2;
+    const int sub = block / nsub;
+    const int nBmax = Npad / block;
+    const int nS = Npad / sub;
+    const double inv = 1.0 / sqrt((double)D);
+    size_t np_ = (size_t)B * H * nS * D, ns = (size_t)B * H * nBmax * nBmax;
+    double* pq = (double*)malloc(sizeof(double) * np_);
+    double* pk = (double*)malloc(sizeof(double) * np_);
+    double* S = scores ? scores : (double*)malloc(sizeof(double) * ns);
+    oracle_pool(q, B, H, Npad, D, valid_len, sub, pq);   /* sub-block means */
+    oracle_pool(k, B, H, Npad, D, valid_len, sub, pk);
+#pragma omp parallel for collapse(2) schedule(dynamic)
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H; ++h) {
+            const int L = valid_len[b], nB = n_blocks_of(L, block);
+            const double* qb = pq + ((size_t)b * H + h) * nS * D;
+            const double* kb = pk + ((size_t)b * H + h) * nS * D;
+            double* Sb = S + ((size_t)b * H + h) * nBmax * nBmax;
+            double x[256];
+            for (int I = 0; I < nBmax; ++I)
+                for (int J = 0; J < nBmax; ++J) {
+                    if (I >= nB || J >= nB) { Sb[(size_t)I * nBmax + J] = NAN; continue; }
+                    int nx = 0;
+                    for (int a = 0; a < nsub; ++a) {
+                        const int sa = I * nsub + a, n0a = sa * sub;
+                        const int ca = (L - n0a) < 0 ? 0 : ((L - n0a) > sub ? sub : (L - n0a));
+                        if (ca == 0) continue;
+                        for (int c = 0; c < nsub; ++c) {
+                            const int sc_ = J * nsub + c, n0c = sc_ * sub;
+                            const int cc = (L - n0c) < 0 ? 0 : ((L - n0c) > sub ? sub : (L - n0c));
+                            if (cc == 0) continue;
+                            double s = 0.0;
+                            for (int d = 0; d < D; ++d) s += qb[(size_t)sa * D + d] * kb[(size_t)sc_ * D + d];
+                            x[nx++] = s * inv + log((double)ca) + log((double)cc);
+                        }
+                    }
+                    double m = -INFINITY;
+                    for (int t = 0; t < nx; ++t) if (x[t] > m) m = x[t];
+                    double z = 0.0;
+                    for (int t = 0; t < nx; ++t) z += exp(x[t] - m);
+                    Sb[(size_t)I * nBmax + J] = m + log(z);
+                }
+        }
+    /* kept count with the optional budget rounding, then the same top-k as above */
+    int status = 0;
+    int32_t* vl_k = (int32_t*)malloc(sizeof(int32_t) * (size_t)B);
+    for (int b = 0; b < B; ++b) vl_k[b] = valid_len[b];
+#pragma omp parallel
+    {
+        scored_block* row = (scored_block*)malloc(sizeof(scored_block) * (size_t)(nBmax > 0 ? nBmax : 1));
+#pragma omp for collapse(2) schedule(dynamic)
+        for (int b = 0; b < B; ++b)
+            for (int h = 0; h < H; ++h) {
+                const int nB = n_blocks_of(vl_k[b], block);
+                int kk = oracle_keep_count(nB, sparsity);
+                if (budget > 1) {
+                    kk = ((kk + budget - 1) / budget) * budget;
+                    if (kk > nB) kk = nB;
+                }
+                if (kk > kmax) {
+#pragma omp atomic write
+                    status = -1;
+                    kk = kmax;
+                }
+                for (int I = 0; I < nBmax; ++I) {
+                    size_t r = ((size_t)b * H + h) * nBmax + I;
+                    int32_t* idx = kv_idx + r * kmax;
+                    for (int t = 0; t < kmax; ++t) idx[t] = -1;
+                    if (I >= nB) { kv_cnt[r] = 0; continue; }
+                    for (int J = 0; J < nB; ++J) {
+                        row[J].score = S[r * nBmax + J];
+                        row[J].index = J;
+                    }
+                    qsort(row, (size_t)nB, sizeof(scored_block), by_score_desc_index_asc);
+                    for (int t = 0; t < kk; ++t) idx[t] = row[t].index;
+                    qsort(idx, (size_t)kk, sizeof(int32_t), int_asc);
+                    kv_cnt[r] = kk;
+                }
+            }
+        free(row);
+    }
+    free(vl_k);
+    free(pq);
+    free(pk);
+    if (!scores) free(S);
+    return status;
+}
