@@ -6,6 +6,11 @@ sba_pair_query_blocks (which two query blocks share an attention tile) and
 sba_attention_paired over the kept blocks.  Prints ONE JSON line (rank 0).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+                  [--router mean|lse] [--budget B]
+
+`--router lse` routes with the sub-block log-sum-exp score (sba_pool_select_lse,
+16-token sub-blocks) and `--budget` rounds its kept count up to a multiple of B
+blocks; the default is the block-mean router with no rounding.
 
 Metric: effective TFLOP/s on the kept blocks, counted as
 4 * D * sum_{b,h,I} c_I * sum_{J kept} c_J (c = valid tokens of a block), divided by
@@ -45,6 +50,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--router", default="mean", choices=["mean", "lse"])
+    ap.add_argument("--budget", type=int, default=1)
     return ap.parse_args()
 
 
@@ -154,7 +161,7 @@ def whole_job_value(kept_flops_per_rank, ms_per_step, world):
     return world * kept_flops_per_rank / (ms_per_step * 1e-3) / 1e12
 
 
-def oracle_sample(w, target_s=10.0, seed=0):
+def oracle_sample(w, target_s=10.0, seed=0, router="mean", budget=1):
     """Time the fp64 oracle, as it stands, on a bounded sample of the workload: the
     full routing of head (b=0, h=0) and the attention of a seeded subset of that head's
     query blocks, sized to about `target_s` seconds.
@@ -166,7 +173,10 @@ def oracle_sample(w, target_s=10.0, seed=0):
     q1, k1, v1 = (np.ascontiguousarray(x[:1, :1]) for x in (w.q, w.k, w.v))
     vl1 = np.ascontiguousarray(w.valid_len[:1])
     t0 = time.perf_counter()
-    idx, cnt = oracle.select(q1, k1, vl1, w.sparsity)
+    if router == "lse":
+        idx, cnt = oracle.select_lse(q1, k1, vl1, w.sparsity, budget=budget)
+    else:
+        idx, cnt = oracle.select(q1, k1, vl1, w.sparsity)
     t_sel = time.perf_counter() - t0
     f_head = kept_flops(idx, cnt, vl1, w.D)
     L = int(vl1[0])
@@ -205,6 +215,12 @@ def workload_config(w, extra=None):
     return c
 
 
+def router_config(args):
+    if args.router == "mean":
+        return {"router": "block mean"}
+    return {"router": "sub-block log-sum-exp (4 x 16 tokens)", "budget": args.budget}
+
+
 def run_reference(args):
     """The oracle as the reference arm, rank 0 only: every step is a bounded sample."""
     from workloads import CONFIGS, make_workload
@@ -214,14 +230,14 @@ def run_reference(args):
     per = []
     target = max(2.0, 60.0 / max(1, args.steps + args.warmup))
     for i in range(args.warmup + args.steps):
-        s = oracle_sample(w, target_s=target, seed=i)
+        s = oracle_sample(w, target_s=target, seed=i, router=args.router, budget=args.budget)
         if i >= args.warmup:
             per.append(s)
     value = statistics.mean(s["value"] for s in per)
     t_step = statistics.mean(s["t_sel"] + s["t_attn"] for s in per)
     cb = cpu_baseline_from(per[-1])
     cb["value"] = value
-    cfg = workload_config(w, {"H": CONFIGS[args.config]["H"],
+    cfg = workload_config(w, {"H": CONFIGS[args.config]["H"], **router_config(args),
                               "sample": "each step: oracle routing of head (0,0) + attention of a "
                                         "seeded subset of its query blocks"})
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
@@ -256,10 +272,12 @@ def run_ours(args):
     q, k, v = t(w.q), t(w.k), t(w.v)
     vl = torch.from_numpy(w.valid_len).to(dev)
     B, H, Npad, D = q.shape
-    kmax = sba.kmax_for(Npad, w.sparsity)
+    lse_router = args.router == "lse"
+    kmax = sba.keep_count_budget(Npad // 64, w.sparsity, args.budget) if lse_router else sba.kmax_for(Npad, w.sparsity)
     kv_idx = torch.empty((B, H, Npad // 64, kmax), dtype=torch.int32, device=dev)
     kv_cnt = torch.empty((B, H, Npad // 64), dtype=torch.int32, device=dev)
-    ws = torch.empty(sba.workspace_size(B, H, Npad, D), dtype=torch.uint8, device=dev)
+    wsz = sba.lse_workspace_size(B, H, Npad, D) if lse_router else sba.workspace_size(B, H, Npad, D)
+    ws = torch.empty(wsz, dtype=torch.uint8, device=dev)
     o = torch.empty_like(q)
     lse = torch.empty((B, H, Npad), dtype=torch.float32, device=dev)
     nQ = Npad // 64
@@ -268,8 +286,12 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
 
     def route(qq=q, kk=k, vll=vl):
-        sba.pool_select(qq, kk, vll, w.sparsity, kmax, kv_idx=kv_idx, kv_cnt=kv_cnt, workspace=ws,
-                        stream=stream)
+        if lse_router:
+            sba.pool_select_lse(qq, kk, vll, w.sparsity, budget=args.budget, kmax=kmax, kv_idx=kv_idx,
+                                kv_cnt=kv_cnt, workspace=ws, stream=stream)
+        else:
+            sba.pool_select(qq, kk, vll, w.sparsity, kmax, kv_idx=kv_idx, kv_cnt=kv_cnt, workspace=ws,
+                            stream=stream)
         sba.pair_query_blocks(kv_idx, kv_cnt, vll, pair_order=pair_order, workspace=pws, stream=stream)
 
     def attend(qq=q, kk=k, vv=v, vll=vl):
@@ -361,22 +383,23 @@ def run_ours(args):
         "data": "synthetic (seeded smooth field + noise, bf16; no weights involved)",
         "config": workload_config(w, {
             "l2": f"inputs {3 * q.numel() * 2 / 1e6:.0f} MB > 126 MB L2; no flush between steps",
-            "kmax": kmax}),
+            "kmax": kmax, **router_config(args)}),
         "pct_of_spec_bf16_peak": 100.0 * value / world / SPEC_BF16_TFLOPS,
         "attn_ms": attn_ms, "select_ms": sel_ms, "kept_tflop_per_step": f_step / 1e12,
         "roofline": {"bound": "tensor", "kernel": "attn_kernel<128,2>" if D == 128 else "attn_kernel<64,4>",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_source": f"{src} bf16_tflops_sustained (kernel timed inside a seconds-long loop)",
                      "traffic": traffic},
-        # per step: 2 pooling + 1 scoring/top-k, 10 pairing (bitmaps, 4 x propose/resolve,
-        # emit), 1 attention
-        "gpu_launches": 14 * K,
+        # per step: routing = 2 pooling + key-norm maximum + screen (only when blocks are
+        # dropped) + top-k; pairing = bitmaps + 4 x (propose, resolve) + emit; 1 attention
+        "gpu_launches": (4 + (1 if w.sparsity > 0 else 0) + 10 + 1) * K,
         "clocks": clk,
     }
     if e2e is not None:
         line["e2e"] = e2e
     if not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline_from(oracle_sample(w, target_s=15.0))
+        line["cpu_baseline"] = cpu_baseline_from(oracle_sample(w, target_s=15.0, router=args.router,
+                                                               budget=args.budget))
     print(json.dumps(line), flush=True)
     if dist is not None:
         dist.destroy_process_group()

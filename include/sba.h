@@ -91,6 +91,38 @@ sba_status sba_pool_select(const void* q, const void* k, int B, int H, int Npad,
                            int32_t* kv_idx, int32_t* kv_cnt,
                            void* workspace, size_t workspace_bytes, void* stream);
 
+/* Bytes of device workspace sba_pool_select_lse needs (0 on bad arguments or an
+ * unsupported nsub).  It holds the pooled sub-block means (nsub per block). */
+size_t sba_pool_select_lse_workspace_size(int B, int H, int Npad, int D, int block, int nsub);
+
+/* Routing step with the sub-block log-sum-exp score, the SubBlock router's own
+ * form (same page and section: every 64-token block split into n_q = n_k = 4
+ * sub-blocks of 16 tokens; pooling and a log-sum-exp estimate each key block's
+ * unnormalised softmax mass for each query block and head; the kept count is
+ * subject to rounding to an 8-block budget):
+ *   qbar[I,a] = mean of q over the valid tokens of sub-block a of block I,
+ *               n[I,a] = their count (kbar, n[J,c] likewise)
+ *   score[I][J] = log sum over non-empty (a, c) of
+ *                 n[I,a] n[J,c] exp(qbar[I,a] . kbar[J,c] / sqrt(D))
+ *   kept(I) = the keep(nB_b, s) blocks of highest score, keep rounded up to a
+ *             multiple of `budget` and capped at nB_b; equal scores go to the
+ *             lower index.
+ * For tokens constant within each sub-block the score is exactly the log of
+ * sum_{i in I, j in J} exp(q_i . k_j / sqrt(D)).
+ *   nsub     sub-blocks per block; 4 is the one supported value (else UNSUPPORTED)
+ *   budget   >= 1; 1 = no rounding
+ *   kmax     must be >= the budget-rounded keep(Npad/block, s)
+ *   other arguments as sba_pool_select; workspace of at least
+ *   sba_pool_select_lse_workspace_size bytes.
+ * The kept set equals the top-k of the fp64 evaluation of the score in the
+ * stated order (dot products summed over d in order, then the max-shifted
+ * log-sum-exp in (a, c) order); scores within a few fp64 rounding steps of each
+ * other may be ordered either way. */
+sba_status sba_pool_select_lse(const void* q, const void* k, int B, int H, int Npad, int D,
+                               const int32_t* valid_len, int block, int nsub, double sparsity,
+                               int budget, int kmax, int32_t* kv_idx, int32_t* kv_cnt,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
 /* Block means of x as fp64 values [B, H, Npad/block, D] (inspection helper;
  * blocks past nB_b are written as 0).  `out` is device memory. */
 sba_status sba_block_means(const void* x, int B, int H, int Npad, int D,

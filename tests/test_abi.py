@@ -124,3 +124,27 @@ def test_binding_refuses_cpu_tensors():
         sba.dense_attention(x, x, x)
     with pytest.raises(ValueError):
         sba.pool_select(x, x, None, 0.5)
+
+
+def pool_select_lse(lib, q=A, k=A, B=1, H=2, Npad=1024, D=64, vl=NULL, block=64, nsub=4, s=0.5, budget=8,
+                    kmax=8, idx=A, cnt=A, ws=A, wsb=1 << 30):
+    return lib.sba_pool_select_lse(q, k, B, H, Npad, D, vl, block, nsub, s, budget, kmax, idx, cnt, ws, wsb, S)
+
+
+@pytest.mark.parametrize("kwargs,code", [
+    (dict(q=NULL), 1), (dict(ws=NULL), 1), (dict(nsub=2), 2), (dict(nsub=1), 2), (dict(nsub=16), 2),
+    (dict(budget=0), 1), (dict(budget=-3), 1), (dict(s=1.0), 1), (dict(D=96), 2), (dict(Npad=1000), 1),
+    # 16 blocks at s = 0.5 keep 8; a budget of 3 rounds that up to 9
+    (dict(budget=3, kmax=8), 1), (dict(s=0.6, budget=1, kmax=6), 1),
+    (dict(wsb=1024), 1), (dict(q=MIS), 3), (dict(vl=MIS), 3),
+])
+def test_pool_select_lse_rejects(lib, kwargs, code):
+    assert pool_select_lse(lib, **kwargs) == code
+
+
+def test_lse_workspace_size(lib):
+    one = lib.sba_pool_select_workspace_size(1, 24, 32768, 128, 64)
+    four = lib.sba_pool_select_lse_workspace_size(1, 24, 32768, 128, 64, 4)
+    assert four > one
+    assert lib.sba_pool_select_lse_workspace_size(1, 24, 32768, 128, 64, 2) == 0
+    assert lib.sba_pool_select_lse_workspace_size(1, 24, 32760, 128, 64, 4) == 0

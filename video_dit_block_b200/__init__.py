@@ -4,8 +4,9 @@ The compute path is a C-ABI CUDA library (include/sba.h, csrc/); this package is
 Python binding.  See `sba` for the calls.
 """
 from .sba import (SbaError, attention, attention_paired, block_means, dense_attention, device_status, keep_count,
-                  kmax_for, lib, pair_query_blocks, pool_select, set_wait_limit, sparse_attention, workspace_size)
+                  keep_count_budget, kmax_for, lib, lse_workspace_size, pair_query_blocks, pool_select,
+                  pool_select_lse, set_wait_limit, sparse_attention, workspace_size)
 
 __all__ = ["SbaError", "attention", "attention_paired", "block_means", "dense_attention", "device_status",
-           "keep_count", "kmax_for", "lib", "pair_query_blocks", "pool_select", "set_wait_limit", "sparse_attention",
-           "workspace_size"]
+           "keep_count", "keep_count_budget", "kmax_for", "lib", "lse_workspace_size", "pair_query_blocks",
+           "pool_select", "pool_select_lse", "set_wait_limit", "sparse_attention", "workspace_size"]

@@ -101,6 +101,56 @@ sba_status launch_attention(const void* q, const void* k, const void* v, void* o
     return cudaGetLastError() == cudaSuccess ? SBA_OK : SBA_ERR_CUDA;
 }
 
+// Routing launches shared by both routers: pool Q and K (blocks, or NSUB
+// sub-blocks per block), largest key norm, screened scores on the tensor cores
+// (skipped when nothing is dropped), then the per-row top-k.  Arguments checked
+// by the caller.
+template <int D, int NSUB>
+sba_status run_select(const void* q, const void* k, int B, int H, int Npad, const int32_t* valid_len,
+                      double sparsity, int budget, int kmax, int32_t* kv_idx, int32_t* kv_cnt,
+                      void* workspace, cudaStream_t s) {
+    constexpr int BLK = 64 / NSUB;
+    const size_t BH = (size_t)B * H;
+    const int nB = Npad / 64;
+    const int nP = nB * NSUB;
+    sba::SelectWorkspace ws = sba::carve_select_workspace(workspace, BH, nB, D, NSUB);
+    const long long pgroups = (long long)BH * nP;
+    const int gpc = 256 / (D / 8);  // pooled rows per CTA
+    const unsigned pool_grid = (unsigned)((pgroups + gpc - 1) / gpc);
+    const long long rows = (long long)BH * nB;
+    const int wpb = 8;              // top-k: one warp per routing row
+    const size_t tsmem = sba::topk_smem(wpb, ws.ld);
+    if (tsmem > 227 * 1024) return SBA_ERR_UNSUPPORTED;
+    const unsigned tgrid = (unsigned)((rows + wpb - 1) / wpb);
+    const auto* qb = static_cast<const __nv_bfloat16*>(q);
+    const auto* kb = static_cast<const __nv_bfloat16*>(k);
+    const bool need_scores = sparsity > 0.0;
+    CUtensorMap tqh, tql, tkh, tkl;
+    if (need_scores && (!make_map(&tqh, ws.qhi, (int)BH, nP, D, 128) || !make_map(&tql, ws.qlo, (int)BH, nP, D, 128) ||
+                        !make_map(&tkh, ws.khi, (int)BH, nP, D, 256) || !make_map(&tkl, ws.klo, (int)BH, nP, D, 256)))
+        return SBA_ERR_CUDA;
+    sba::pool_kernel<D, BLK><<<pool_grid, 256, 0, s>>>(qb, valid_len, H, Npad, ws.qmean64, ws.qhi, ws.qlo, ws.qnorm,
+                                                       pgroups);
+    sba::pool_kernel<D, BLK><<<pool_grid, 256, 0, s>>>(kb, valid_len, H, Npad, ws.kmean64, ws.khi, ws.klo, ws.knorm,
+                                                       pgroups);
+    sba::kmax_kernel<<<(unsigned)((BH + 7) / 8), 256, 0, s>>>(ws, valid_len, H, Npad, (int)BH, BLK);
+    if (need_scores) {
+        using SM = sba::ScoreSmem<D>;
+        if (cudaFuncSetAttribute(sba::score_mma_kernel<D, NSUB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 SM::kAlloc) != cudaSuccess)
+            return SBA_ERR_CUDA;
+        const dim3 sgrid((nP + 127) / 128, (nP + 255) / 256, (unsigned)BH);
+        sba::score_mma_kernel<D, NSUB><<<sgrid, 128, SM::kAlloc, s>>>(tqh, tql, tkh, tkl, ws.scores, nB, ws.ld,
+                                                                      valid_len, H, Npad, g_wait_limit);
+    }
+    if (cudaFuncSetAttribute(sba::topk_kernel<D, NSUB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsmem) !=
+        cudaSuccess)
+        return SBA_ERR_CUDA;
+    sba::topk_kernel<D, NSUB><<<tgrid, 32 * wpb, tsmem, s>>>(ws, valid_len, H, Npad, sparsity, budget, kmax, kv_idx,
+                                                             kv_cnt, rows);
+    return cudaGetLastError() == cudaSuccess ? SBA_OK : SBA_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
@@ -128,60 +178,36 @@ sba_status sba_pool_select(const void* q, const void* k, int B, int H, int Npad,
     if (!aligned16(q) || !aligned16(k) || !aligned16(workspace) || !aligned16(valid_len))
         return SBA_ERR_ALIGNMENT;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const size_t BH = (size_t)B * H;
-    sba::SelectWorkspace ws = sba::carve_select_workspace(workspace, BH, nB, D);
-    const long long groups = (long long)BH * nB;
-    const int gpc = 256 / (D / 8);  // block groups per CTA
-    const unsigned pool_grid = (unsigned)((groups + gpc - 1) / gpc);
-    const int wpb = 8;              // top-k: one warp per routing row
-    const size_t tsmem = sba::topk_smem(wpb, ws.ld);
-    if (tsmem > 227 * 1024) return SBA_ERR_UNSUPPORTED;
-    const unsigned tgrid = (unsigned)((groups + wpb - 1) / wpb);
-    const auto* qb = static_cast<const __nv_bfloat16*>(q);
-    const auto* kb = static_cast<const __nv_bfloat16*>(k);
-    // scores are needed unless nothing is dropped for any sample
-    const bool need_scores = sparsity > 0.0;
-    CUtensorMap tqh, tql, tkh, tkl;
-    if (need_scores && (!make_map(&tqh, ws.qhi, (int)BH, nB, D, 128) || !make_map(&tql, ws.qlo, (int)BH, nB, D, 128) ||
-                        !make_map(&tkh, ws.khi, (int)BH, nB, D, 256) || !make_map(&tkl, ws.klo, (int)BH, nB, D, 256)))
-        return SBA_ERR_CUDA;
-    const dim3 sgrid((nB + 127) / 128, (nB + 255) / 256, (unsigned)BH);
-    if (D == 128) {
-        sba::pool_kernel<128><<<pool_grid, 256, 0, s>>>(qb, valid_len, H, Npad, ws.qmean64, ws.qhi, ws.qlo, ws.qnorm, groups);
-        sba::pool_kernel<128><<<pool_grid, 256, 0, s>>>(kb, valid_len, H, Npad, ws.kmean64, ws.khi, ws.klo, ws.knorm, groups);
-        sba::kmax_kernel<<<(unsigned)((BH + 7) / 8), 256, 0, s>>>(ws, valid_len, H, Npad, (int)BH);
-        if (need_scores) {
-            using SM = sba::ScoreSmem<128>;
-            if (cudaFuncSetAttribute(sba::score_mma_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     SM::kAlloc) != cudaSuccess)
-                return SBA_ERR_CUDA;
-            sba::score_mma_kernel<128><<<sgrid, 128, SM::kAlloc, s>>>(tqh, tql, tkh, tkl, ws.scores, nB, ws.ld,
-                                                                      g_wait_limit);
-        }
-        if (cudaFuncSetAttribute(sba::topk_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsmem) !=
-            cudaSuccess)
-            return SBA_ERR_CUDA;
-        sba::topk_kernel<128><<<tgrid, 32 * wpb, tsmem, s>>>(ws, valid_len, H, Npad, sparsity, kmax, kv_idx, kv_cnt,
-                                                             groups);
-    } else {
-        sba::pool_kernel<64><<<pool_grid, 256, 0, s>>>(qb, valid_len, H, Npad, ws.qmean64, ws.qhi, ws.qlo, ws.qnorm, groups);
-        sba::pool_kernel<64><<<pool_grid, 256, 0, s>>>(kb, valid_len, H, Npad, ws.kmean64, ws.khi, ws.klo, ws.knorm, groups);
-        sba::kmax_kernel<<<(unsigned)((BH + 7) / 8), 256, 0, s>>>(ws, valid_len, H, Npad, (int)BH);
-        if (need_scores) {
-            using SM = sba::ScoreSmem<64>;
-            if (cudaFuncSetAttribute(sba::score_mma_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     SM::kAlloc) != cudaSuccess)
-                return SBA_ERR_CUDA;
-            sba::score_mma_kernel<64><<<sgrid, 128, SM::kAlloc, s>>>(tqh, tql, tkh, tkl, ws.scores, nB, ws.ld,
-                                                                     g_wait_limit);
-        }
-        if (cudaFuncSetAttribute(sba::topk_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsmem) !=
-            cudaSuccess)
-            return SBA_ERR_CUDA;
-        sba::topk_kernel<64><<<tgrid, 32 * wpb, tsmem, s>>>(ws, valid_len, H, Npad, sparsity, kmax, kv_idx, kv_cnt,
-                                                            groups);
-    }
-    return cudaGetLastError() == cudaSuccess ? SBA_OK : SBA_ERR_CUDA;
+    if (D == 128)
+        return run_select<128, 1>(q, k, B, H, Npad, valid_len, sparsity, 1, kmax, kv_idx, kv_cnt, workspace, s);
+    return run_select<64, 1>(q, k, B, H, Npad, valid_len, sparsity, 1, kmax, kv_idx, kv_cnt, workspace, s);
+}
+
+size_t sba_pool_select_lse_workspace_size(int B, int H, int Npad, int D, int block, int nsub) {
+    if (check_shape(B, H, Npad, D, block) != SBA_OK || nsub != sba::kNsub) return 0;
+    return sba::select_workspace_bytes((size_t)B * H, (size_t)Npad / block, (size_t)D, (size_t)nsub);
+}
+
+sba_status sba_pool_select_lse(const void* q, const void* k, int B, int H, int Npad, int D,
+                               const int32_t* valid_len, int block, int nsub, double sparsity, int budget,
+                               int kmax, int32_t* kv_idx, int32_t* kv_cnt, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+    sba_status st = check_shape(B, H, Npad, D, block);
+    if (st != SBA_OK) return st;
+    if (nsub != sba::kNsub) return SBA_ERR_UNSUPPORTED;
+    if (!q || !k || !kv_idx || !kv_cnt || !workspace) return SBA_ERR_INVALID_ARG;
+    if (!(sparsity >= 0.0 && sparsity < 1.0) || budget < 1) return SBA_ERR_INVALID_ARG;
+    const int nB = Npad / block;
+    if (kmax < sba::keep_count_budget(nB, sparsity, budget)) return SBA_ERR_INVALID_ARG;
+    if (workspace_bytes < sba::select_workspace_bytes((size_t)B * H, nB, D, nsub)) return SBA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(workspace) || !aligned16(valid_len))
+        return SBA_ERR_ALIGNMENT;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (D == 128)
+        return run_select<128, sba::kNsub>(q, k, B, H, Npad, valid_len, sparsity, budget, kmax, kv_idx, kv_cnt,
+                                           workspace, s);
+    return run_select<64, sba::kNsub>(q, k, B, H, Npad, valid_len, sparsity, budget, kmax, kv_idx, kv_cnt,
+                                      workspace, s);
 }
 
 sba_status sba_block_means(const void* x, int B, int H, int Npad, int D, const int32_t* valid_len,

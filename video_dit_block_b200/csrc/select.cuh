@@ -26,12 +26,14 @@ namespace sba {
 
 constexpr int kBlock = 64;
 
-// Workspace layout of sba_pool_select (all offsets 256-byte aligned):
-//   qmean64, kmean64 : double [BH][nB][D]   block means
-//   qhi, qlo, khi, klo : bf16 [BH][nB][D]   hi/lo split of the means for the screen
-//   qnorm, knorm     : double [BH][nB]      Euclidean norm of each block mean
-//   kmaxn            : double [BH]          largest key-block norm of the sample
-//   scores           : float [BH][nB][ld]   screened scores, ld = 64 * ceil(nB / 64)
+// Workspace layout of the routers (all offsets 256-byte aligned).  Means are
+// pooled over 64-token blocks (nsub = 1) or over the nsub sub-blocks of each
+// block (the log-sum-exp router, nsub = 4); nP = nB * nsub pooled rows:
+//   qmean64, kmean64 : double [BH][nP][D]   pooled means
+//   qhi, qlo, khi, klo : bf16 [BH][nP][D]   hi/lo split of the means for the screen
+//   qnorm, knorm     : double [BH][nP]      Euclidean norm of each mean
+//   kmaxn            : double [BH]          largest key-mean norm of the sample
+//   scores           : float [BH][nB][ld]   screened block scores, ld = 64 * ceil(nB / 64)
 struct SelectWorkspace {
     double* qmean64;
     double* kmean64;
@@ -50,21 +52,23 @@ __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_
 
 __host__ __device__ inline size_t select_score_ld(size_t nB) { return (nB + 63) / 64 * 64; }
 
-__host__ __device__ inline size_t select_workspace_bytes(size_t BH, size_t nB, size_t D) {
-    const size_t m64 = align256(BH * nB * D * sizeof(double));
-    const size_t m16 = align256(BH * nB * D * 2);
-    const size_t nrm = align256(BH * nB * sizeof(double));
+__host__ __device__ inline size_t select_workspace_bytes(size_t BH, size_t nB, size_t D, size_t nsub = 1) {
+    const size_t nP = nB * nsub;
+    const size_t m64 = align256(BH * nP * D * sizeof(double));
+    const size_t m16 = align256(BH * nP * D * 2);
+    const size_t nrm = align256(BH * nP * sizeof(double));
     const size_t kmx = align256(BH * sizeof(double));
     const size_t sco = align256(BH * nB * select_score_ld(nB) * sizeof(float));
     return 2 * m64 + 4 * m16 + 2 * nrm + kmx + sco;
 }
 
 __host__ __device__ inline SelectWorkspace carve_select_workspace(void* base, size_t BH, size_t nB,
-                                                                  size_t D) {
+                                                                  size_t D, size_t nsub = 1) {
     char* p = static_cast<char*>(base);
-    const size_t m64 = align256(BH * nB * D * sizeof(double));
-    const size_t m16 = align256(BH * nB * D * 2);
-    const size_t nrm = align256(BH * nB * sizeof(double));
+    const size_t nP = nB * nsub;
+    const size_t m64 = align256(BH * nP * D * sizeof(double));
+    const size_t m16 = align256(BH * nP * D * 2);
+    const size_t nrm = align256(BH * nP * sizeof(double));
     const size_t kmx = align256(BH * sizeof(double));
     SelectWorkspace w;
     w.qmean64 = reinterpret_cast<double*>(p); p += m64;
@@ -81,6 +85,10 @@ __host__ __device__ inline SelectWorkspace carve_select_workspace(void* base, si
     return w;
 }
 
+// The log-sum-exp router splits each 64-token block into kNsub sub-blocks.
+constexpr int kNsub = 4;
+constexpr int kSubBlock = kBlock / kNsub;
+
 // keep(n, s) with the same fp64 operations, in the same order, as the host rule.
 __host__ __device__ inline int keep_count(int n, double s) {
     if (n <= 0) return 0;
@@ -95,6 +103,16 @@ __host__ __device__ inline int keep_count(int n, double s) {
     return (int)x;
 }
 
+// keep(n, s) rounded up to a multiple of `budget` blocks, at most n.
+__host__ __device__ inline int keep_count_budget(int n, double s, int budget) {
+    int k = keep_count(n, s);
+    if (budget > 1) {
+        k = (k + budget - 1) / budget * budget;
+        if (k > n) k = n;
+    }
+    return k;
+}
+
 __device__ __forceinline__ int sample_len(const int32_t* valid_len, int b, int Npad) {
     return valid_len ? valid_len[b] : Npad;
 }
@@ -103,8 +121,9 @@ __device__ __forceinline__ int sample_len(const int32_t* valid_len, int b, int N
 // One group of D/8 lanes per (bh, block): lane g owns channels [8g, 8g+8) and
 // walks the block's valid rows in token order, 16-byte loads, fp64 sums.
 // Writes the fp64 mean and, when the pointers are non-null, its bf16 hi/lo split
-// and the norm of the block mean.
-template <int D>
+// and the norm of the block mean.  BLK is the pooling granularity: 64-token
+// blocks, or the 16-token sub-blocks of the log-sum-exp router.
+template <int D, int BLK = kBlock>
 __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restrict__ x,
                                                    const int32_t* __restrict__ valid_len, int H,
                                                    int Npad, double* __restrict__ mean64,
@@ -113,7 +132,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
                                                    double* __restrict__ norm, long long n_groups) {
     constexpr int LPB = D / 8;  // lanes per block group
     constexpr int UNROLL = 16;
-    const int nB = Npad / kBlock;
+    const int nB = Npad / BLK;
     long long grp = (long long)blockIdx.x * (256 / LPB) + threadIdx.x / LPB;
     const int g = threadIdx.x % LPB;
     const bool active = grp < n_groups;
@@ -122,9 +141,9 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
     const int I = (int)(grp % nB);
     const int b = (int)(bh / H);
     const int L = sample_len(valid_len, b, Npad);
-    const int n0 = I * kBlock;
+    const int n0 = I * BLK;
     int cnt = L - n0;
-    cnt = cnt < 0 ? 0 : (cnt > kBlock ? kBlock : cnt);
+    cnt = cnt < 0 ? 0 : (cnt > BLK ? BLK : cnt);
 
     const uint4* src = reinterpret_cast<const uint4*>(x + ((size_t)bh * Npad + n0) * D) + g;
     double s[8];
@@ -207,8 +226,96 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
 __device__ __forceinline__ double exact_score(const double* __restrict__ q,
                                               const double* __restrict__ k, int D, double inv) {
     double s = 0.0;
+#pragma unroll 4
     for (int d = 0; d < D; ++d) s = __dadd_rn(s, __dmul_rn(q[d], k[d]));
     return __dadd_rn(__dmul_rn(s, inv), 0.0);
+}
+
+// fp64 log-sum-exp block score of query block I against key block J, in the same
+// operation order as the definition it restates: for every pair (a, c) of
+// non-empty sub-blocks, a-major,
+//   x = ((qbar_a . kbar_c) * inv + log(n_a)) + log(n_c)
+// with the dot product summed over d in order, each step rounded to nearest; then
+// m = max x, z = sum over the pairs (same order) of exp(x - m), score = m + log z.
+// q4, k4: the NSUB consecutive fp64 sub-block means of the two blocks.
+template <int NSUB>
+__device__ double exact_lse(const double* __restrict__ q4, const double* __restrict__ k4, int D, int L,
+                            int I, int J, double inv) {
+    constexpr int SUB = kBlock / NSUB;
+    double x[NSUB * NSUB];
+    double m = -INFINITY;
+#pragma unroll
+    for (int a = 0; a < NSUB; ++a) {
+        int na = L - (I * NSUB + a) * SUB;
+        na = na < 0 ? 0 : (na > SUB ? SUB : na);
+#pragma unroll
+        for (int c = 0; c < NSUB; ++c) {
+            int nc = L - (J * NSUB + c) * SUB;
+            nc = nc < 0 ? 0 : (nc > SUB ? SUB : nc);
+            x[a * NSUB + c] = -INFINITY;  // empty pair: no term
+            if (na > 0 && nc > 0) {
+                const double* qa = q4 + (size_t)a * D;
+                const double* kc = k4 + (size_t)c * D;
+                double s = 0.0;
+#pragma unroll 4
+                for (int d = 0; d < D; ++d) s = __dadd_rn(s, __dmul_rn(qa[d], kc[d]));
+                const double xv = __dadd_rn(__dadd_rn(__dmul_rn(s, inv), log((double)na)), log((double)nc));
+                x[a * NSUB + c] = xv;
+                m = xv > m ? xv : m;
+            }
+        }
+    }
+    double z = 0.0;
+#pragma unroll
+    for (int t = 0; t < NSUB * NSUB; ++t)
+        if (x[t] != -INFINITY) z = __dadd_rn(z, exp(__dadd_rn(x[t], -m)));
+    return __dadd_rn(__dadd_rn(m, log(z)), 0.0);
+}
+
+// Exact log-sum-exp scores of the n_band (<= kBandCache) key blocks listed in
+// `slots` for query block I, by one warp: the NSUB^2 sub-block pairs of a block go
+// to NSUB^2 lanes (32 / NSUB^2 blocks per pass), each lane forms its pair's logit
+// (same operations as exact_lse), the group takes the max, each lane its
+// exponential, and the group's first lane sums them in pair order and takes the
+// log.  Bitwise the same values as exact_lse.  Writes out[t] for t < n_band.
+template <int NSUB>
+__device__ void band_exact_lse(const double* __restrict__ q4, const double* __restrict__ kbase, int D, int L,
+                               int I, double inv, const int32_t* slots, int n_band, double* out) {
+    constexpr int SUB = kBlock / NSUB;
+    constexpr int PAIRS = NSUB * NSUB;
+    constexpr int PER_PASS = 32 / PAIRS;
+    static_assert(PAIRS <= 32 && 32 % PAIRS == 0, "pairs of a block must tile a warp");
+    const int lane = threadIdx.x & 31;
+    const int p = lane % PAIRS, a = p / NSUB, c = p % NSUB;
+    const int g0 = lane - p;  // first lane of this lane's group
+    int na = L - (I * NSUB + a) * SUB;
+    na = na < 0 ? 0 : (na > SUB ? SUB : na);
+    const double lna = na > 0 ? log((double)na) : 0.0;
+    for (int t0 = 0; t0 < n_band; t0 += PER_PASS) {
+        const int t = t0 + lane / PAIRS;
+        double x = -INFINITY;
+        if (t < n_band) {
+            const int J = slots[t];
+            int nc = L - (J * NSUB + c) * SUB;
+            nc = nc < 0 ? 0 : (nc > SUB ? SUB : nc);
+            if (na > 0 && nc > 0) {
+                const double* qa = q4 + (size_t)a * D;
+                const double* kc = kbase + ((size_t)J * NSUB + c) * D;
+                double s = 0.0;
+#pragma unroll 4
+                for (int d = 0; d < D; ++d) s = __dadd_rn(s, __dmul_rn(qa[d], kc[d]));
+                x = __dadd_rn(__dadd_rn(__dmul_rn(s, inv), lna), log((double)nc));
+            }
+        }
+        double m = x;
+#pragma unroll
+        for (int off = 1; off < PAIRS; off <<= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, off));
+        const double e = x != -INFINITY ? exp(__dadd_rn(x, -m)) : 0.0;  // an empty pair adds 0 exactly
+        double z = 0.0;
+#pragma unroll
+        for (int u = 0; u < PAIRS; ++u) z = __dadd_rn(z, __shfl_sync(0xffffffffu, e, g0 + u));
+        if (p == 0 && t < n_band) out[t] = __dadd_rn(__dadd_rn(m, log(z)), 0.0);
+    }
 }
 
 // Warp-cooperative radix select: the k-th largest (1-based) of the 32-bit keys
@@ -319,14 +426,15 @@ __device__ uint64_t warp_radix_select64(int n, int k, uint32_t* hist, KeyOf key_
     return prefix;
 }
 
-// Largest key-block-mean norm of each (b, h) over its sample's blocks; one warp each.
+// Largest key-mean norm of each (b, h) over its sample's pooled rows (blocks of
+// `blk` tokens); one warp each.
 __global__ void kmax_kernel(SelectWorkspace ws, const int32_t* __restrict__ valid_len, int H, int Npad,
-                            int BH) {
+                            int BH, int blk) {
     const int bh = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
     const int lane = threadIdx.x & 31;
     if (bh >= BH) return;
-    const int nBmax = Npad / kBlock;
-    const int nB = (sample_len(valid_len, bh / H, Npad) + kBlock - 1) / kBlock;
+    const int nBmax = Npad / blk;
+    const int nB = (sample_len(valid_len, bh / H, Npad) + blk - 1) / blk;
     double m = 0.0;
     for (int j = lane; j < nB; j += 32) m = fmax(m, ws.knorm[(size_t)bh * nBmax + j]);
 #pragma unroll
@@ -334,10 +442,18 @@ __global__ void kmax_kernel(SelectWorkspace ws, const int32_t* __restrict__ vali
     if (lane == 0) ws.kmaxn[bh] = m;
 }
 
-// Shared-memory bytes of topk_kernel for `warps` warps per CTA.
-__host__ __device__ inline size_t topk_smem(int warps, int ld) {
-    return (size_t)warps * ((size_t)ld * 4 + 256 * 4 + 32 * 4);
+// Band members whose exact scores are cached (and ranked) in shared memory; a wider
+// band falls back to a radix select that re-evaluates them.
+constexpr int kBandCache = 64;
+
+// Shared-memory bytes of one top-k warp: the screened row, a 256-bin histogram,
+// the band's block indices and their exact scores.
+__host__ __device__ inline size_t topk_warp_smem(int ld) {
+    return (size_t)ld * 4 + 256 * 4 + kBandCache * 4 + kBandCache * 8;
 }
+
+// Shared-memory bytes of topk_kernel for `warps` warps per CTA.
+__host__ __device__ inline size_t topk_smem(int warps, int ld) { return (size_t)warps * topk_warp_smem(ld); }
 
 // Top-k routing of one (b, h, I) row per warp, from the screened scores.
 //
@@ -348,10 +464,32 @@ __host__ __device__ inline size_t topk_smem(int warps, int ld) {
 // of the 3D products in fp32 adds at most 3D * 2^-22 of sum |qbar_d kbar_d| (two
 // units in the last place per addition, whatever the order).  With Cauchy-Schwarz,
 // |S - qbar.kbar| <= (4 * 2^-16 + 3D * 2^-22) |qbar_I| max_J |kbar_J|, doubled here
-// for margin, plus an absolute term for values in the subnormal range.
-template <int D>
+// for margin, plus an absolute term for values in the subnormal range.  (The
+// screen now sums hi.hi apart from the two cross terms, which only lowers the
+// accumulation error; this bound is kept as it stands.)
+//
+// Log-sum-exp router (NSUB = 4).  The screen (score_mma_kernel's epilogue) forms
+// every sub-block logit x' = fp32(fp32(hh + cross) * fp32(1/sqrt(D))), hh = the D
+// products hi.hi summed in one fp32 accumulator, cross = the 2D products hi.lo and
+// lo.hi (each below 2^-8 |qbar_d kbar_d|) in another.  Per logit, relative to
+// R_ac = |qbar_a| |kbar_c| / sqrt(D):
+//   dropped split terms      4 * 2^-16
+//   hh accumulation          1.01 D * 2^-22   (two ulps per addition)
+//   cross accumulation       1.01 D * 2^-28
+//   final add, 1/sqrt(D), product    3 * 2^-24
+// so |x' - x| <= (4 * 2^-16 + (D + 2) * 2^-22 + D * 2^-27) R, R = max_a |qbar_a| *
+// max_c |kbar_c| / sqrt(D), plus the subnormal term.  The log-sum-exp is
+// 1-Lipschitz in the largest logit error, so the block score inherits the bound.
+// Its fp32 evaluation adds at most 2^-20 R + 2^-17: the max is exact; each gap to
+// the max, times fp32(log2 e), carries three roundings (relative 2^-24 each) of a
+// value below 3R, which moves each exponential by at most a relative 2^-21 R;
+// ex2.approx is taken as accurate to 2^-20 relative; the count-weighted sum of at
+// most 16 terms (at least 1, the term of the max) to 2^-19; the log of a value
+// below 4097 to two ulps (2^-19); the last add to 2^-24 (R + 9).  The total is
+// multiplied by 1.25 for margin.
+template <int D, int NSUB = 1>
 __global__ void __launch_bounds__(256) topk_kernel(SelectWorkspace ws, const int32_t* __restrict__ valid_len,
-                                                   int H, int Npad, double sparsity, int kmax,
+                                                   int H, int Npad, double sparsity, int budget, int kmax,
                                                    int32_t* __restrict__ kv_idx, int32_t* __restrict__ kv_cnt,
                                                    long long rows) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -365,7 +503,7 @@ __global__ void __launch_bounds__(256) topk_kernel(SelectWorkspace ws, const int
     const int I = (int)(rid % nBmax);
     const int L = sample_len(valid_len, (int)(bh / H), Npad);
     const int nB = (L + kBlock - 1) / kBlock;
-    const int k = keep_count(nB, sparsity);
+    const int k = keep_count_budget(nB, sparsity, budget);
     int32_t* out = kv_idx + (size_t)rid * kmax;
     if (I >= nB) {
         if (lane == 0) kv_cnt[rid] = 0;
@@ -376,17 +514,27 @@ __global__ void __launch_bounds__(256) topk_kernel(SelectWorkspace ws, const int
         if (lane == 0) kv_cnt[rid] = nB;
         return;
     }
-    float* row = reinterpret_cast<float*>(smem_raw + (size_t)warp * ((size_t)ld * 4 + 256 * 4 + 32 * 4));
+    float* row = reinterpret_cast<float*>(smem_raw + (size_t)warp * topk_warp_smem(ld));
     uint32_t* whist = reinterpret_cast<uint32_t*>(row + ld);
     int32_t* wslots = reinterpret_cast<int32_t*>(whist + 256);
+    double* bx = reinterpret_cast<double*>(wslots + kBandCache);  // 8-byte aligned: ld % 64 == 0
     const float* src = ws.scores + (size_t)rid * ld;
     for (int j = lane; j < nB; j += 32) row[j] = __ldg(src + j);
     __syncwarp();
     const double inv = __ddiv_rn(1.0, __dsqrt_rn((double)D));
-    const double qn = ws.qnorm[rid];
+    const size_t prow = (size_t)bh * nBmax * NSUB + (size_t)I * NSUB;  // first pooled row of block I
+    double qn = ws.qnorm[prow];
+#pragma unroll
+    for (int a = 1; a < NSUB; ++a) qn = fmax(qn, ws.qnorm[prow + a]);
     const double kmx = ws.kmaxn[bh];
-    const double* qrow64 = ws.qmean64 + (size_t)rid * D;
-    const double* kbase64 = ws.kmean64 + (size_t)bh * nBmax * D;
+    const double* qrow64 = ws.qmean64 + prow * D;
+    const double* kbase64 = ws.kmean64 + (size_t)bh * nBmax * NSUB * D;
+    auto exact = [&](int j) -> double {
+        if constexpr (NSUB == 1)
+            return exact_score(qrow64, kbase64 + (size_t)j * D, D, inv);
+        else
+            return exact_lse<NSUB>(qrow64, kbase64 + (size_t)j * NSUB * D, D, L, I, j, inv);
+    };
 
     // k-th largest fp32 score
     const uint32_t tau_key = warp_radix_select32(nB, k, whist, [&](int j, bool& ok) {
@@ -396,8 +544,12 @@ __global__ void __launch_bounds__(256) topk_kernel(SelectWorkspace ws, const int
     const double tau = (double)key_to_f32(tau_key);
     // screen error bound (see above); the band [tau - 2 delta, tau + 2 delta] is
     // decided in fp64, everything above it is kept and everything below dropped
-    const double delta = 2.0 * (4.0 * 0x1p-16 + 3.0 * D * 0x1p-22) * qn * kmx +
-                         3.0 * D * 0x1p-120 * (1.0 + qn + kmx);
+    double delta;
+    if constexpr (NSUB == 1)
+        delta = 2.0 * (4.0 * 0x1p-16 + 3.0 * D * 0x1p-22) * qn * kmx + 3.0 * D * 0x1p-120 * (1.0 + qn + kmx);
+    else
+        delta = 1.25 * ((4.0 * 0x1p-16 + (D + 2.0) * 0x1p-22 + D * 0x1p-27 + 0x1p-20) * qn * kmx * inv +
+                        3.0 * D * 0x1p-120 * (1.0 + qn + kmx) + 0x1p-17);
     const double hi = tau + 2.0 * delta, lo = tau - 2.0 * delta;
 
     int n_in = 0, n_band = 0;
@@ -411,9 +563,10 @@ __global__ void __launch_bounds__(256) topk_kernel(SelectWorkspace ws, const int
     }
     const int need = k - n_in;  // band members to keep, 1 <= need <= n_band
 
-    // mode 0: keep the whole band; 1: small band ranked in registers; 2: wide band
-    int mode = need >= n_band ? 0 : (n_band <= 32 ? 1 : 2);
-    uint32_t chosen_mask = 0xffffffffu;
+    // mode 0: keep the whole band; 1: band of at most kBandCache, exact scores cached
+    // and ranked in shared memory; 2: wide band, radix select
+    int mode = need >= n_band ? 0 : (n_band <= kBandCache ? 1 : 2);
+    uint64_t chosen_mask = ~0ull;
     uint64_t tau_x = 0;
     int eq_take = 0;
     if (mode == 1) {
@@ -427,22 +580,40 @@ __global__ void __launch_bounds__(256) topk_kernel(SelectWorkspace ws, const int
             base += __popc(bb);
         }
         __syncwarp();
-        const int myj = lane < n_band ? wslots[lane] : 0;
-        const double my_s = lane < n_band ? exact_score(qrow64, kbase64 + (size_t)myj * D, D, inv)
-                                          : -INFINITY;
-        int rank = 0;
-        for (int t = 0; t < n_band; ++t) {
-            const double s_t = __shfl_sync(0xffffffffu, my_s, t);
-            const int j_t = __shfl_sync(0xffffffffu, myj, t);
-            rank += (s_t > my_s || (s_t == my_s && j_t < myj)) ? 1 : 0;
+        if constexpr (NSUB == 1) {
+            for (int t = lane; t < n_band; t += 32) bx[t] = exact(wslots[t]);
+        } else {
+            band_exact_lse<NSUB>(qrow64, kbase64, D, L, I, inv, wslots, n_band, bx);
         }
-        chosen_mask = __ballot_sync(0xffffffffu, lane < n_band && rank < need);
+        __syncwarp();
+        // rank of each member: members with a higher exact score, or an equal one
+        // and a lower block index, come first
+        bool pick[kBandCache / 32];
+#pragma unroll
+        for (int h = 0; h < kBandCache / 32; ++h) {
+            const int t = lane + 32 * h;
+            pick[h] = false;
+            if (t < n_band) {
+                const double st = bx[t];
+                const int jt = wslots[t];
+                int rank = 0;
+                for (int u = 0; u < n_band; ++u) {
+                    const double su = bx[u];
+                    rank += (su > st || (su == st && wslots[u] < jt)) ? 1 : 0;
+                }
+                pick[h] = rank < need;
+            }
+        }
+        chosen_mask = 0ull;
+#pragma unroll
+        for (int h = 0; h < kBandCache / 32; ++h)
+            chosen_mask |= (uint64_t)__ballot_sync(0xffffffffu, pick[h]) << (32 * h);
         __syncwarp();
     } else if (mode == 2) {
         auto band_key = [&](int j, bool& ok) -> uint64_t {
             const double f = (double)row[j];
             ok = !(f > hi) && f >= lo;
-            return ok ? f64_key(exact_score(qrow64, kbase64 + (size_t)j * D, D, inv)) : 0ull;
+            return ok ? f64_key(exact(j)) : 0ull;
         };
         tau_x = warp_radix_select64(nB, need, whist, band_key);
         int gt = 0;
@@ -469,10 +640,10 @@ __global__ void __launch_bounds__(256) topk_kernel(SelectWorkspace ws, const int
             sel = sel || in_b;
         } else if (mode == 1) {
             const int slot = band_seen + __popc(bb & lanemask_lt());
-            sel = sel || (in_b && ((chosen_mask >> slot) & 1u));
+            sel = sel || (in_b && ((chosen_mask >> slot) & 1ull));
         } else {
             uint64_t x = 0;
-            if (in_b) x = f64_key(exact_score(qrow64, kbase64 + (size_t)j * D, D, inv));
+            if (in_b) x = f64_key(exact(j));
             const bool eq = in_b && x == tau_x;
             const uint32_t eb = __ballot_sync(0xffffffffu, eq);
             const int eq_rank = eq_seen + __popc(eb & lanemask_lt());

@@ -46,6 +46,11 @@ def lib() -> ctypes.CDLL:
         L.sba_pool_select_workspace_size.argtypes = [i32, i32, i32, i32, i32]
         L.sba_pool_select.restype = i32
         L.sba_pool_select.argtypes = [vp, vp, i32, i32, i32, i32, vp, i32, f64, i32, vp, vp, vp, sz, vp]
+        L.sba_pool_select_lse_workspace_size.restype = sz
+        L.sba_pool_select_lse_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32]
+        L.sba_pool_select_lse.restype = i32
+        L.sba_pool_select_lse.argtypes = [vp, vp, i32, i32, i32, i32, vp, i32, i32, f64, i32, i32, vp, vp, vp,
+                                          sz, vp]
         L.sba_block_means.restype = i32
         L.sba_block_means.argtypes = [vp, i32, i32, i32, i32, vp, i32, vp, vp]
         L.sba_attention.restype = i32
@@ -138,6 +143,41 @@ def pool_select(q, k, valid_len=None, sparsity: float = 0.0, kmax: int | None = 
     return kv_idx, kv_cnt
 
 
+def keep_count_budget(n_blocks: int, sparsity: float, budget: int = 1) -> int:
+    """keep(n, s) rounded up to a multiple of `budget`, at most n."""
+    k = keep_count(n_blocks, sparsity)
+    if budget > 1:
+        k = min(int(n_blocks), -(-k // budget) * budget)
+    return k
+
+
+def lse_workspace_size(B: int, H: int, Npad: int, D: int, nsub: int = 4, block: int = BLOCK) -> int:
+    return int(lib().sba_pool_select_lse_workspace_size(B, H, Npad, D, block, nsub))
+
+
+def pool_select_lse(q, k, valid_len=None, sparsity: float = 0.0, nsub: int = 4, budget: int = 1,
+                    kmax: int | None = None, block: int = BLOCK, kv_idx=None, kv_cnt=None, workspace=None,
+                    stream=None):
+    """Sub-block log-sum-exp routing: (kv_idx int32 [B,H,Npad/64,kmax], kv_cnt int32 [B,H,Npad/64])."""
+    B, H, Npad, D = _qkv(q, k)
+    vl = _valid_len(valid_len, q.device)
+    nB = Npad // block
+    if kmax is None:
+        kmax = keep_count_budget(nB, sparsity, budget)
+    if kv_idx is None:
+        kv_idx = torch.empty((B, H, nB, kmax), dtype=torch.int32, device=q.device)
+    if kv_cnt is None:
+        kv_cnt = torch.empty((B, H, nB), dtype=torch.int32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(lse_workspace_size(B, H, Npad, D, nsub, block), dtype=torch.uint8,
+                                device=q.device)
+    _check(lib().sba_pool_select_lse(_ptr(q), _ptr(k), B, H, Npad, D, _ptr(vl), block, int(nsub),
+                                     float(sparsity), int(budget), int(kmax), _ptr(kv_idx), _ptr(kv_cnt),
+                                     _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                     _stream(stream)), "sba_pool_select_lse")
+    return kv_idx, kv_cnt
+
+
 def block_means(x, valid_len=None, block: int = BLOCK, stream=None):
     """fp64 block means [B, H, Npad/64, D]."""
     B, H, Npad, D = _qkv(x)
@@ -212,10 +252,17 @@ def dense_attention(q, k, v, valid_len=None, softmax_scale: float = 0.0, out=Non
 
 
 def sparse_attention(q, k, v, valid_len=None, sparsity: float = 0.75, softmax_scale: float = 0.0,
-                     stream=None):
+                     router: str = "mean", budget: int = 1, stream=None):
     """The whole path: routing, tile pairing, block-sparse attention.
+    router "mean": block-mean scores (sba_pool_select); "lse": sub-block
+    log-sum-exp scores with an optional kept-count budget (sba_pool_select_lse).
     Returns (o, lse, kv_idx, kv_cnt)."""
-    kv_idx, kv_cnt = pool_select(q, k, valid_len, sparsity, stream=stream)
+    if router == "mean":
+        kv_idx, kv_cnt = pool_select(q, k, valid_len, sparsity, stream=stream)
+    elif router == "lse":
+        kv_idx, kv_cnt = pool_select_lse(q, k, valid_len, sparsity, budget=budget, stream=stream)
+    else:
+        raise ValueError(f"unknown router {router!r}")
     pair_order = pair_query_blocks(kv_idx, kv_cnt, valid_len, stream=stream)
     o, lse = attention_paired(q, k, v, kv_idx, kv_cnt, pair_order, valid_len, softmax_scale, stream=stream)
     return o, lse, kv_idx, kv_cnt
