@@ -14,6 +14,7 @@
 #include "common.cuh"
 #include "select.cuh"
 #include "score_mma.cuh"
+#include "score_lse.cuh"
 #include "pair.cuh"
 
 namespace {
@@ -126,22 +127,38 @@ sba_status run_select(const void* q, const void* k, int B, int H, int Npad, cons
     const auto* kb = static_cast<const __nv_bfloat16*>(k);
     const bool need_scores = sparsity > 0.0;
     CUtensorMap tqh, tql, tkh, tkl;
+    const int brows = NSUB == 1 ? 256 : 128;  // key-side box rows of the screen
     if (need_scores && (!make_map(&tqh, ws.qhi, (int)BH, nP, D, 128) || !make_map(&tql, ws.qlo, (int)BH, nP, D, 128) ||
-                        !make_map(&tkh, ws.khi, (int)BH, nP, D, 256) || !make_map(&tkl, ws.klo, (int)BH, nP, D, 256)))
+                        !make_map(&tkh, ws.khi, (int)BH, nP, D, brows) ||
+                        !make_map(&tkl, ws.klo, (int)BH, nP, D, brows)))
         return SBA_ERR_CUDA;
     sba::pool_kernel<D, BLK><<<pool_grid, 256, 0, s>>>(qb, valid_len, H, Npad, ws.qmean64, ws.qhi, ws.qlo, ws.qnorm,
                                                        pgroups);
     sba::pool_kernel<D, BLK><<<pool_grid, 256, 0, s>>>(kb, valid_len, H, Npad, ws.kmean64, ws.khi, ws.klo, ws.knorm,
                                                        pgroups);
     sba::kmax_kernel<<<(unsigned)((BH + 7) / 8), 256, 0, s>>>(ws, valid_len, H, Npad, (int)BH, BLK);
-    if (need_scores) {
+    if (need_scores && NSUB == 1) {
         using SM = sba::ScoreSmem<D>;
-        if (cudaFuncSetAttribute(sba::score_mma_kernel<D, NSUB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(sba::score_mma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  SM::kAlloc) != cudaSuccess)
             return SBA_ERR_CUDA;
         const dim3 sgrid((nP + 127) / 128, (nP + 255) / 256, (unsigned)BH);
-        sba::score_mma_kernel<D, NSUB><<<sgrid, 128, SM::kAlloc, s>>>(tqh, tql, tkh, tkl, ws.scores, nB, ws.ld,
-                                                                      valid_len, H, Npad, g_wait_limit);
+        sba::score_mma_kernel<D><<<sgrid, 128, SM::kAlloc, s>>>(tqh, tql, tkh, tkl, ws.scores, nB, ws.ld,
+                                                                g_wait_limit);
+    } else if (need_scores) {
+        // persistent: one CTA per SM over the (b, h, query tile) items
+        using SM = sba::LseSmem<D>;
+        if (cudaFuncSetAttribute(sba::score_lse_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 SM::kAlloc) != cudaSuccess)
+            return SBA_ERR_CUDA;
+        int dev = 0, sms = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+            return SBA_ERR_CUDA;
+        const long long items = (long long)BH * ((nP + 127) / 128);
+        const unsigned grid = (unsigned)(items < sms ? items : sms);
+        sba::score_lse_kernel<D><<<grid, 320, SM::kAlloc, s>>>(tqh, tql, tkh, tkl, ws.scores, nB, ws.ld, valid_len,
+                                                               H, Npad, (int)BH, g_wait_limit);
     }
     if (cudaFuncSetAttribute(sba::topk_kernel<D, NSUB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsmem) !=
         cudaSuccess)

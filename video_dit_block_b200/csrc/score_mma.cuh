@@ -15,14 +15,7 @@
 // 192 KB for D = 128) and the MMAs; all four warps read the 128 x 256 fp32 tile out
 // of TMEM (thread r = row r = TMEM lane r) and store it.
 // Every wait is bounded (SBA_ERR_TIMEOUT, then the CTA drains and exits).
-//
-// NSUB = 4 (the log-sum-exp router): the operand rows are 16-token sub-block means,
-// so one tile holds the 4 x 4 sub-block logits of 32 query blocks x 64 key blocks.
-// The epilogue turns them into block scores
-//     log sum_{a,c} n_a n_c exp(x_ac),  x_ac = qbar_a . kbar_c / sqrt(D),
-// over the non-empty sub-blocks (n = valid tokens of the sub-block): each thread
-// folds the 4 key sub-blocks of its own row, and the 4 lanes holding the rows of
-// one query block combine through shuffles (max, then the weighted sum of exp).
+
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -46,15 +39,13 @@ struct ScoreSmem {
     static constexpr int kAlloc = kTotal + 1024 > 116 * 1024 ? kTotal + 1024 : 116 * 1024;
 };
 
-// maps: bf16 [BH][nP][D] (nP = nB * NSUB pooled rows) viewed as 3-D (D, nP, BH); A maps
-// box 64 x 128 rows, B maps box 64 x 256 rows.  scores: fp32 [BH][nB][ld]; columns
-// past the sample's blocks hold unused values.
-template <int D, int NSUB = 1>
+// maps: bf16 [BH][nB][D] viewed as 3-D (D, nB, BH); A maps box 64 x 128 rows, B maps
+// box 64 x 256 rows.  scores: fp32 [BH][nB][ld], columns >= nB not written.
+template <int D>
 __global__ void __launch_bounds__(128, 1)
     score_mma_kernel(const __grid_constant__ CUtensorMap tmQh, const __grid_constant__ CUtensorMap tmQl,
                      const __grid_constant__ CUtensorMap tmKh, const __grid_constant__ CUtensorMap tmKl,
-                     float* __restrict__ scores, int nB, int ld, const int32_t* __restrict__ valid_len,
-                     int H, int Npad, unsigned long long wait_limit) {
+                     float* __restrict__ scores, int nB, int ld, unsigned long long wait_limit) {
     using SM = ScoreSmem<D>;
     constexpr int NCH = D / 64;
     constexpr uint32_t kIdesc = idesc_bf16_f32(128, 256, 0, 0);
@@ -114,57 +105,7 @@ __global__ void __launch_bounds__(128, 1)
     const int row = m0 + warp * 32 + lane;
     const uint32_t tl = tmem + (static_cast<uint32_t>(warp * 32) << 16);
     const bool go = __all_sync(0xffffffffu, ok && !*abort_flag);
-    if constexpr (NSUB > 1) {
-      if (go) {
-        constexpr int SUB = 64 / NSUB;
-        constexpr float kInv = D == 128 ? 0.0883883476483184405f : 0.125f;  // fp32(1 / sqrt(D))
-        constexpr float kLog2e = 1.4426950408889634f;
-        const int L = valid_len ? valid_len[bh / H] : Npad;
-        const int I = row / NSUB;                    // lanes 4i..4i+3 hold the rows of one block
-        int na = L - row * SUB;
-        na = na < 0 ? 0 : (na > SUB ? SUB : na);
-        const float wa = (float)na;
-        float* dst = scores + ((size_t)bh * nB + I) * ld + n0 / NSUB;
-#pragma unroll 1
-        for (int c0 = 0; c0 < 256; c0 += 32) {
-            uint32_t v[32], v2[32];
-            tmem_ld32(tl + c0, v);
-            tmem_ld32(tl + 256 + c0, v2);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) + __uint_as_float(v2[i]));
-            float blk[32 / NSUB];
-#pragma unroll
-            for (int jb = 0; jb < 32 / NSUB; ++jb) {
-                float x[NSUB], w[NSUB];
-                float m = -INFINITY;
-#pragma unroll
-                for (int c = 0; c < NSUB; ++c) {
-                    int nc = L - (n0 + c0 + jb * NSUB + c) * SUB;
-                    nc = nc < 0 ? 0 : (nc > SUB ? SUB : nc);
-                    w[c] = wa * (float)nc;  // exact: at most 256
-                    x[c] = __uint_as_float(v[jb * NSUB + c]) * kInv;
-                    if (w[c] > 0.f) m = fmaxf(m, x[c]);
-                }
-#pragma unroll
-                for (int off = 1; off < NSUB; off <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-                float z = 0.f;
-#pragma unroll
-                for (int c = 0; c < NSUB; ++c)
-                    if (w[c] > 0.f) z = fmaf(w[c], ex2_approx((x[c] - m) * kLog2e), z);
-#pragma unroll
-                for (int off = 1; off < NSUB; off <<= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
-                blk[jb] = m == -INFINITY ? -INFINITY : m + logf(z);
-            }
-            if ((lane % NSUB) == 0 && I < nB) {
-                float4* d4 = reinterpret_cast<float4*>(dst + c0 / NSUB);
-#pragma unroll
-                for (int i = 0; i < 32 / NSUB / 4; ++i)
-                    d4[i] = make_float4(blk[4 * i], blk[4 * i + 1], blk[4 * i + 2], blk[4 * i + 3]);
-            }
-        }
-      }
-    } else if (go) {
+    if (go) {
         float* dst = scores + ((size_t)bh * nB + row) * ld + n0;
 #pragma unroll 1
         for (int c0 = 0; c0 < 256; c0 += 32) {

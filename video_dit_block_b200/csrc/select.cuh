@@ -122,7 +122,10 @@ __device__ __forceinline__ int sample_len(const int32_t* valid_len, int b, int N
 // walks the block's valid rows in token order, 16-byte loads, fp64 sums.
 // Writes the fp64 mean and, when the pointers are non-null, its bf16 hi/lo split
 // and the norm of the block mean.  BLK is the pooling granularity: 64-token
-// blocks, or the 16-token sub-blocks of the log-sum-exp router.
+// blocks, or the 16-token sub-blocks of the log-sum-exp router.  The fp64 means of
+// the kBlock / BLK sub-blocks of a block are interleaved channel by channel,
+// [..][block][D][kBlock / BLK], so that the lanes re-scoring the sub-block pairs of
+// a block read adjacent words; hi/lo and the norms stay one row per pooled row.
 template <int D, int BLK = kBlock>
 __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restrict__ x,
                                                    const int32_t* __restrict__ valid_len, int H,
@@ -178,10 +181,17 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
 #pragma unroll
     for (int off = LPB / 2; off > 0; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
     if (!active) return;
-    double* dst64 = mean64 + (size_t)grp * D + 8 * g;
+    if constexpr (BLK == kBlock) {
+        double* dst64 = mean64 + (size_t)grp * D + 8 * g;
 #pragma unroll
-    for (int e = 0; e < 8; e += 2) {
-        *reinterpret_cast<double2*>(dst64 + e) = make_double2(m[e], m[e + 1]);
+        for (int e = 0; e < 8; e += 2) *reinterpret_cast<double2*>(dst64 + e) = make_double2(m[e], m[e + 1]);
+    } else {
+        constexpr int NS = kBlock / BLK;
+        const long long blk = grp / NS;
+        const int a = (int)(grp % NS);
+        double* dst64 = mean64 + ((size_t)blk * D + 8 * g) * NS + a;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) dst64[(size_t)e * NS] = m[e];
     }
     if (hi16) {
         // hi = bf16(mean), lo = bf16(mean - hi): the split the tensor-core screen uses
@@ -237,36 +247,34 @@ __device__ __forceinline__ double exact_score(const double* __restrict__ q,
 //   x = ((qbar_a . kbar_c) * inv + log(n_a)) + log(n_c)
 // with the dot product summed over d in order, each step rounded to nearest; then
 // m = max x, z = sum over the pairs (same order) of exp(x - m), score = m + log z.
-// q4, k4: the NSUB consecutive fp64 sub-block means of the two blocks.
+// q4, k4: the fp64 sub-block means of the two blocks, [D][NSUB] (sub-block innermost).
 template <int NSUB>
 __device__ double exact_lse(const double* __restrict__ q4, const double* __restrict__ k4, int D, int L,
                             int I, int J, double inv) {
+    // Only the wide-band fallback calls this (one lane per block), so the loops stay
+    // rolled: the 16 logits live in local memory rather than in registers.
     constexpr int SUB = kBlock / NSUB;
     double x[NSUB * NSUB];
     double m = -INFINITY;
-#pragma unroll
-    for (int a = 0; a < NSUB; ++a) {
+#pragma unroll 1
+    for (int p = 0; p < NSUB * NSUB; ++p) {
+        const int a = p / NSUB, c = p % NSUB;
         int na = L - (I * NSUB + a) * SUB;
         na = na < 0 ? 0 : (na > SUB ? SUB : na);
-#pragma unroll
-        for (int c = 0; c < NSUB; ++c) {
-            int nc = L - (J * NSUB + c) * SUB;
-            nc = nc < 0 ? 0 : (nc > SUB ? SUB : nc);
-            x[a * NSUB + c] = -INFINITY;  // empty pair: no term
-            if (na > 0 && nc > 0) {
-                const double* qa = q4 + (size_t)a * D;
-                const double* kc = k4 + (size_t)c * D;
-                double s = 0.0;
+        int nc = L - (J * NSUB + c) * SUB;
+        nc = nc < 0 ? 0 : (nc > SUB ? SUB : nc);
+        x[p] = -INFINITY;  // empty pair: no term
+        if (na > 0 && nc > 0) {
+            double s = 0.0;
 #pragma unroll 4
-                for (int d = 0; d < D; ++d) s = __dadd_rn(s, __dmul_rn(qa[d], kc[d]));
-                const double xv = __dadd_rn(__dadd_rn(__dmul_rn(s, inv), log((double)na)), log((double)nc));
-                x[a * NSUB + c] = xv;
-                m = xv > m ? xv : m;
-            }
+            for (int d = 0; d < D; ++d) s = __dadd_rn(s, __dmul_rn(q4[d * NSUB + a], k4[d * NSUB + c]));
+            const double xv = __dadd_rn(__dadd_rn(__dmul_rn(s, inv), log((double)na)), log((double)nc));
+            x[p] = xv;
+            m = xv > m ? xv : m;
         }
     }
     double z = 0.0;
-#pragma unroll
+#pragma unroll 1
     for (int t = 0; t < NSUB * NSUB; ++t)
         if (x[t] != -INFINITY) z = __dadd_rn(z, exp(__dadd_rn(x[t], -m)));
     return __dadd_rn(__dadd_rn(m, log(z)), 0.0);
@@ -299,11 +307,10 @@ __device__ void band_exact_lse(const double* __restrict__ q4, const double* __re
             int nc = L - (J * NSUB + c) * SUB;
             nc = nc < 0 ? 0 : (nc > SUB ? SUB : nc);
             if (na > 0 && nc > 0) {
-                const double* qa = q4 + (size_t)a * D;
-                const double* kc = kbase + ((size_t)J * NSUB + c) * D;
+                const double* k4 = kbase + (size_t)J * NSUB * D;
                 double s = 0.0;
 #pragma unroll 4
-                for (int d = 0; d < D; ++d) s = __dadd_rn(s, __dmul_rn(qa[d], kc[d]));
+                for (int d = 0; d < D; ++d) s = __dadd_rn(s, __dmul_rn(q4[d * NSUB + a], k4[d * NSUB + c]));
                 x = __dadd_rn(__dadd_rn(__dmul_rn(s, inv), lna), log((double)nc));
             }
         }
@@ -468,25 +475,25 @@ __host__ __device__ inline size_t topk_smem(int warps, int ld) { return (size_t)
 // screen now sums hi.hi apart from the two cross terms, which only lowers the
 // accumulation error; this bound is kept as it stands.)
 //
-// Log-sum-exp router (NSUB = 4).  The screen (score_mma_kernel's epilogue) forms
-// every sub-block logit x' = fp32(fp32(hh + cross) * fp32(1/sqrt(D))), hh = the D
-// products hi.hi summed in one fp32 accumulator, cross = the 2D products hi.lo and
-// lo.hi (each below 2^-8 |qbar_d kbar_d|) in another.  Per logit, relative to
-// R_ac = |qbar_a| |kbar_c| / sqrt(D):
-//   dropped split terms      4 * 2^-16
-//   hh accumulation          1.01 D * 2^-22   (two ulps per addition)
-//   cross accumulation       1.01 D * 2^-28
-//   final add, 1/sqrt(D), product    3 * 2^-24
+// Log-sum-exp router (NSUB = 4).  The screen (score_lse_kernel) forms every
+// sub-block logit in log2 units, y' = fp32(acc * fp32(log2(e) / sqrt(D))), where acc
+// accumulates in fp32 first the 2D cross products hi.lo and lo.hi (each below
+// 2^-8 |qbar_d kbar_d|), then the D products hi.hi.  Per logit, relative to
+// R_ac = |qbar_a| |kbar_c| / sqrt(D), the error of x' = y' ln 2 is at most
+//   dropped split terms              4 * 2^-16
+//   hi.hi accumulation               1.02 D * 2^-22  (two ulps per addition of a
+//                                    partial sum below 1.02 sum_d |qbar_d kbar_d|)
+//   cross accumulation               1.01 D * 2^-28
+//   scale constant and product       2 * 2^-24
 // so |x' - x| <= (4 * 2^-16 + (D + 2) * 2^-22 + D * 2^-27) R, R = max_a |qbar_a| *
 // max_c |kbar_c| / sqrt(D), plus the subnormal term.  The log-sum-exp is
 // 1-Lipschitz in the largest logit error, so the block score inherits the bound.
 // Its fp32 evaluation adds at most 2^-20 R + 2^-17: the max is exact; each gap to
-// the max, times fp32(log2 e), carries three roundings (relative 2^-24 each) of a
-// value below 3R, which moves each exponential by at most a relative 2^-21 R;
-// ex2.approx is taken as accurate to 2^-20 relative; the count-weighted sum of at
-// most 16 terms (at least 1, the term of the max) to 2^-19; the log of a value
-// below 4097 to two ulps (2^-19); the last add to 2^-24 (R + 9).  The total is
-// multiplied by 1.25 for margin.
+// the max (one rounding of a value below 3R) moves its exponential by at most a
+// relative 2^-21 R; ex2.approx is taken as accurate to 2^-20 relative; the
+// count-weighted sum of at most 16 terms (at least 1, the term of the max) to
+// 2^-19; log2 of a value below 4097 to two ulps; the last add and the product by
+// ln 2 to 2^-23 (R + 12).  The total is multiplied by 1.25 for margin.
 template <int D, int NSUB = 1>
 __global__ void __launch_bounds__(256) topk_kernel(SelectWorkspace ws, const int32_t* __restrict__ valid_len,
                                                    int H, int Npad, double sparsity, int budget, int kmax,
