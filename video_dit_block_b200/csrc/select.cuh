@@ -280,48 +280,83 @@ __device__ double exact_lse(const double* __restrict__ q4, const double* __restr
     return __dadd_rn(__dadd_rn(m, log(z)), 0.0);
 }
 
-// Exact log-sum-exp scores of the n_band (<= kBandCache) key blocks listed in
-// `slots` for query block I, by one warp: the NSUB^2 sub-block pairs of a block go
-// to NSUB^2 lanes (32 / NSUB^2 blocks per pass), each lane forms its pair's logit
-// (same operations as exact_lse), the group takes the max, each lane its
-// exponential, and the group's first lane sums them in pair order and takes the
-// log.  Bitwise the same values as exact_lse.  Writes out[t] for t < n_band.
-template <int NSUB>
-__device__ void band_exact_lse(const double* __restrict__ q4, const double* __restrict__ kbase, int D, int L,
-                               int I, double inv, const int32_t* slots, int n_band, double* out) {
-    constexpr int SUB = kBlock / NSUB;
-    constexpr int PAIRS = NSUB * NSUB;
-    constexpr int PER_PASS = 32 / PAIRS;
-    static_assert(PAIRS <= 32 && 32 % PAIRS == 0, "pairs of a block must tile a warp");
+// fp64 log-sum-exp scores of the n_band (<= kBandCache) key blocks listed in
+// `slots` for query block I (4 sub-blocks per block), one block at a time by the
+// whole warp.  For each half of the 16 sub-block pairs (query sub-blocks 2h, 2h + 1),
+// lane l forms partial dot products over channels l, l + 32, .. (fp64 fused
+// multiply-adds) and a transposing butterfly leaves the 4 lanes with equal bits
+// 4..2 one pair's dot product; then the max, the exponentials and their sum go over
+// the 16 pairs.  Same definition as exact_lse, evaluated in another order: values
+// agree with it to a few fp64 roundings.  q4, k4: sub-block means [D][4].  Writes
+// out[t], t < n_band.
+template <int D>
+__device__ void band_lse_warp(const double* __restrict__ q4, const double* __restrict__ kbase, int L, int I,
+                              double inv, const int32_t* slots, int n_band, double* out) {
+    constexpr int NSUB = 4, SUB = kBlock / NSUB, CPL = D / 32;  // channels per lane
     const int lane = threadIdx.x & 31;
-    const int p = lane % PAIRS, a = p / NSUB, c = p % NSUB;
-    const int g0 = lane - p;  // first lane of this lane's group
-    int na = L - (I * NSUB + a) * SUB;
-    na = na < 0 ? 0 : (na > SUB ? SUB : na);
-    const double lna = na > 0 ? log((double)na) : 0.0;
-    for (int t0 = 0; t0 < n_band; t0 += PER_PASS) {
-        const int t = t0 + lane / PAIRS;
-        double x = -INFINITY;
-        if (t < n_band) {
-            const int J = slots[t];
-            int nc = L - (J * NSUB + c) * SUB;
-            nc = nc < 0 ? 0 : (nc > SUB ? SUB : nc);
-            if (na > 0 && nc > 0) {
-                const double* k4 = kbase + (size_t)J * NSUB * D;
-                double s = 0.0;
-#pragma unroll 4
-                for (int d = 0; d < D; ++d) s = __dadd_rn(s, __dmul_rn(q4[d * NSUB + a], k4[d * NSUB + c]));
-                x = __dadd_rn(__dadd_rn(__dmul_rn(s, inv), lna), log((double)nc));
+    // pair within a half held after the butterfly: bits 4, 3, 2 of the lane index
+    const int ph = 4 * ((lane >> 4) & 1) + 2 * ((lane >> 3) & 1) + ((lane >> 2) & 1);
+    const int c = ph & 3;
+    double lna[2];
+    bool va[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int a = 2 * h + (ph >> 2);
+        int na = L - (I * NSUB + a) * SUB;
+        na = na < 0 ? 0 : (na > SUB ? SUB : na);
+        va[h] = na > 0;
+        lna[h] = na > 0 ? log((double)na) : 0.0;
+    }
+    for (int t = 0; t < n_band; ++t) {
+        const int J = slots[t];
+        const double* k4 = kbase + (size_t)J * NSUB * D;
+        int nc = L - (J * NSUB + c) * SUB;
+        nc = nc < 0 ? 0 : (nc > SUB ? SUB : nc);
+        const double lnc = nc > 0 ? log((double)nc) : 0.0;
+        double x[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            double p[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) p[e] = 0.0;
+#pragma unroll
+            for (int i = 0; i < CPL; ++i) {
+                const size_t d = (size_t)(lane + 32 * i) * NSUB;
+                const double2 qq = *reinterpret_cast<const double2*>(q4 + d + 2 * h);
+                const double2 u = *reinterpret_cast<const double2*>(k4 + d);
+                const double2 w = *reinterpret_cast<const double2*>(k4 + d + 2);
+                const double kv[4] = {u.x, u.y, w.x, w.y};
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    p[cc] = fma(qq.x, kv[cc], p[cc]);
+                    p[4 + cc] = fma(qq.y, kv[cc], p[4 + cc]);
+                }
             }
+            double h4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const bool up = (lane >> 4) & 1;
+                h4[e] = (up ? p[4 + e] : p[e]) + __shfl_xor_sync(0xffffffffu, up ? p[e] : p[4 + e], 16);
+            }
+            double h2[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const bool up = (lane >> 3) & 1;
+                h2[e] = (up ? h4[2 + e] : h4[e]) + __shfl_xor_sync(0xffffffffu, up ? h4[e] : h4[2 + e], 8);
+            }
+            const bool up2 = (lane >> 2) & 1;
+            double dot = (up2 ? h2[1] : h2[0]) + __shfl_xor_sync(0xffffffffu, up2 ? h2[0] : h2[1], 4);
+            dot += __shfl_xor_sync(0xffffffffu, dot, 2);
+            dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+            x[h] = (va[h] && nc > 0) ? dot * inv + lna[h] + lnc : -INFINITY;
         }
-        double m = x;
+        double m = fmax(x[0], x[1]);
 #pragma unroll
-        for (int off = 1; off < PAIRS; off <<= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, off));
-        const double e = x != -INFINITY ? exp(__dadd_rn(x, -m)) : 0.0;  // an empty pair adds 0 exactly
-        double z = 0.0;
+        for (int off = 4; off < 32; off <<= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, off));
+        double z = (x[0] != -INFINITY ? exp(x[0] - m) : 0.0) + (x[1] != -INFINITY ? exp(x[1] - m) : 0.0);
 #pragma unroll
-        for (int u = 0; u < PAIRS; ++u) z = __dadd_rn(z, __shfl_sync(0xffffffffu, e, g0 + u));
-        if (p == 0 && t < n_band) out[t] = __dadd_rn(__dadd_rn(m, log(z)), 0.0);
+        for (int off = 4; off < 32; off <<= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
+        if (lane == 0) out[t] = m + log(z);
     }
 }
 
@@ -495,7 +530,7 @@ __host__ __device__ inline size_t topk_smem(int warps, int ld) { return (size_t)
 // 2^-19; log2 of a value below 4097 to two ulps; the last add and the product by
 // ln 2 to 2^-23 (R + 12).  The total is multiplied by 1.25 for margin.
 template <int D, int NSUB = 1>
-__global__ void __launch_bounds__(256) topk_kernel(SelectWorkspace ws, const int32_t* __restrict__ valid_len,
+__global__ void __launch_bounds__(256, NSUB == 1 ? 4 : 3) topk_kernel(SelectWorkspace ws, const int32_t* __restrict__ valid_len,
                                                    int H, int Npad, double sparsity, int budget, int kmax,
                                                    int32_t* __restrict__ kv_idx, int32_t* __restrict__ kv_cnt,
                                                    long long rows) {
@@ -525,9 +560,115 @@ __global__ void __launch_bounds__(256) topk_kernel(SelectWorkspace ws, const int
     uint32_t* whist = reinterpret_cast<uint32_t*>(row + ld);
     int32_t* wslots = reinterpret_cast<int32_t*>(whist + 256);
     double* bx = reinterpret_cast<double*>(wslots + kBandCache);  // 8-byte aligned: ld % 64 == 0
+    float* bval = reinterpret_cast<float*>(bx);                    // bucket members' values (before bx is used)
+
+    // ---- the screened row, with its smallest and largest value
     const float* src = ws.scores + (size_t)rid * ld;
-    for (int j = lane; j < nB; j += 32) row[j] = __ldg(src + j);
+    float vmin = INFINITY, vmax = -INFINITY;
+    for (int j = lane; j < nB; j += 32) {
+        const float f = __ldg(src + j);
+        row[j] = f;
+        vmin = fminf(vmin, f);
+        vmax = fmaxf(vmax, f);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        vmin = fminf(vmin, __shfl_xor_sync(0xffffffffu, vmin, off));
+        vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, off));
+    }
     __syncwarp();
+
+    // ---- tau = the k-th largest screened value.  A 256-bucket histogram between the
+    // row's min and max finds the bucket holding it; when that bucket has at most
+    // kBandCache members they are ranked directly, otherwise a radix select over
+    // all the values decides.  Both give the same value.
+    float tau = 0.f;
+    bool have_tau = false;
+    const float range = vmax - vmin;
+    const float bscale = 256.0f / range;
+    if (range > 0.f && range <= 3.0e38f && bscale <= 3.0e38f) {
+        auto bucket = [&](float f) { return min(255, (int)((f - vmin) * bscale)); };
+        for (int i = lane; i < 256; i += 32) whist[i] = 0u;
+        __syncwarp();
+        for (int j = lane; j < nB; j += 32) atomicAdd(&whist[bucket(row[j])], 1u);
+        __syncwarp();
+        // lane l holds buckets 255 - 8l - e (e = 0..7), highest first
+        uint32_t c[8], tot = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            c[e] = whist[255 - (8 * lane + e)];
+            tot += c[e];
+        }
+        uint32_t incl = tot;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const uint32_t v = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += v;
+        }
+        const uint32_t excl = incl - tot;
+        const uint32_t ball = __ballot_sync(0xffffffffu, excl < (uint32_t)k && (uint32_t)k <= incl);
+        const int src_lane = ball ? __ffs(ball) - 1 : 31;
+        int bstar = 0;
+        uint32_t above = 0, bcount = 0;
+        if (lane == src_lane) {
+            uint32_t acc = excl;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                if (acc + c[e] >= (uint32_t)k) {
+                    bstar = 255 - (8 * lane + e);
+                    above = acc;
+                    bcount = c[e];
+                    break;
+                }
+                acc += c[e];
+            }
+        }
+        bstar = __shfl_sync(0xffffffffu, bstar, src_lane);
+        above = __shfl_sync(0xffffffffu, above, src_lane);
+        bcount = __shfl_sync(0xffffffffu, bcount, src_lane);
+        if (bcount >= 1 && bcount <= (uint32_t)kBandCache) {
+            // the bucket's values, then the (k - above)-th largest of them
+            int base = 0;
+            for (int j0 = 0; j0 < nB; j0 += 32) {
+                const int j = j0 + lane;
+                const bool in = j < nB && bucket(row[j]) == bstar;
+                const uint32_t bb = __ballot_sync(0xffffffffu, in);
+                if (in) bval[base + __popc(bb & lanemask_lt())] = row[j];
+                base += __popc(bb);
+            }
+            __syncwarp();
+            const int kk = k - (int)above;  // 1 <= kk <= bcount
+            bool hit = false;
+            float hv = 0.f;
+            for (int t = lane; t < (int)bcount; t += 32) {
+                const float vt = bval[t];
+                int gt = 0, ge = 0;
+                for (int u = 0; u < (int)bcount; ++u) {
+                    const float vu = bval[u];
+                    gt += vu > vt ? 1 : 0;
+                    ge += vu >= vt ? 1 : 0;
+                }
+                if (gt < kk && kk <= ge) {
+                    hit = true;
+                    hv = vt;
+                }
+            }
+            const uint32_t hb = __ballot_sync(0xffffffffu, hit);
+            if (hb) {
+                tau = __shfl_sync(0xffffffffu, hv, __ffs(hb) - 1);
+                have_tau = true;
+            }
+            __syncwarp();
+        }
+    }
+    if (!have_tau) {
+        const uint32_t tau_key = warp_radix_select32(nB, k, whist, [&](int j, bool& ok) {
+            ok = true;
+            return f32_key(row[j]);
+        });
+        tau = key_to_f32(tau_key);
+    }
+
     const double inv = __ddiv_rn(1.0, __dsqrt_rn((double)D));
     const size_t prow = (size_t)bh * nBmax * NSUB + (size_t)I * NSUB;  // first pooled row of block I
     double qn = ws.qnorm[prow];
@@ -543,54 +684,46 @@ __global__ void __launch_bounds__(256) topk_kernel(SelectWorkspace ws, const int
             return exact_lse<NSUB>(qrow64, kbase64 + (size_t)j * NSUB * D, D, L, I, j, inv);
     };
 
-    // k-th largest fp32 score
-    const uint32_t tau_key = warp_radix_select32(nB, k, whist, [&](int j, bool& ok) {
-        ok = true;
-        return f32_key(row[j]);
-    });
-    const double tau = (double)key_to_f32(tau_key);
-    // screen error bound (see above); the band [tau - 2 delta, tau + 2 delta] is
-    // decided in fp64, everything above it is kept and everything below dropped
+    // screen error bound (see above); everything above the band [tau - 2 delta,
+    // tau + 2 delta] is kept, everything below dropped, the band decided in fp64.
+    // The edges are rounded outwards to fp32 so that the tests run in fp32; that can
+    // only move values into the band.
     double delta;
     if constexpr (NSUB == 1)
         delta = 2.0 * (4.0 * 0x1p-16 + 3.0 * D * 0x1p-22) * qn * kmx + 3.0 * D * 0x1p-120 * (1.0 + qn + kmx);
     else
         delta = 1.25 * ((4.0 * 0x1p-16 + (D + 2.0) * 0x1p-22 + D * 0x1p-27 + 0x1p-20) * qn * kmx * inv +
                         3.0 * D * 0x1p-120 * (1.0 + qn + kmx) + 0x1p-17);
-    const double hi = tau + 2.0 * delta, lo = tau - 2.0 * delta;
+    const float hi = __double2float_ru((double)tau + 2.0 * delta);
+    const float lo = __double2float_rd((double)tau - 2.0 * delta);
 
+    // ---- classify: count the sure keeps, list the band (its first kBandCache members)
     int n_in = 0, n_band = 0;
     for (int j0 = 0; j0 < nB; j0 += 32) {
         const int j = j0 + lane;
-        const double f = j < nB ? (double)row[j] : -INFINITY;
+        const float f = j < nB ? row[j] : -INFINITY;
         const bool in_a = j < nB && f > hi;
         const bool in_b = j < nB && !in_a && f >= lo;
         n_in += __popc(__ballot_sync(0xffffffffu, in_a));
-        n_band += __popc(__ballot_sync(0xffffffffu, in_b));
+        const uint32_t bb = __ballot_sync(0xffffffffu, in_b);
+        const int slot = n_band + __popc(bb & lanemask_lt());
+        if (in_b && slot < kBandCache) wslots[slot] = j;
+        n_band += __popc(bb);
     }
     const int need = k - n_in;  // band members to keep, 1 <= need <= n_band
+    __syncwarp();
 
     // mode 0: keep the whole band; 1: band of at most kBandCache, exact scores cached
     // and ranked in shared memory; 2: wide band, radix select
-    int mode = need >= n_band ? 0 : (n_band <= kBandCache ? 1 : 2);
+    const int mode = need >= n_band ? 0 : (n_band <= kBandCache ? 1 : 2);
     uint64_t chosen_mask = ~0ull;
     uint64_t tau_x = 0;
     int eq_take = 0;
     if (mode == 1) {
-        int base = 0;
-        for (int j0 = 0; j0 < nB; j0 += 32) {
-            const int j = j0 + lane;
-            const double f = j < nB ? (double)row[j] : -INFINITY;
-            const bool in_b = j < nB && !(f > hi) && f >= lo;
-            const uint32_t bb = __ballot_sync(0xffffffffu, in_b);
-            if (in_b) wslots[base + __popc(bb & lanemask_lt())] = j;
-            base += __popc(bb);
-        }
-        __syncwarp();
         if constexpr (NSUB == 1) {
             for (int t = lane; t < n_band; t += 32) bx[t] = exact(wslots[t]);
         } else {
-            band_exact_lse<NSUB>(qrow64, kbase64, D, L, I, inv, wslots, n_band, bx);
+            band_lse_warp<D>(qrow64, kbase64, L, I, inv, wslots, n_band, bx);
         }
         __syncwarp();
         // rank of each member: members with a higher exact score, or an equal one
@@ -618,7 +751,7 @@ __global__ void __launch_bounds__(256) topk_kernel(SelectWorkspace ws, const int
         __syncwarp();
     } else if (mode == 2) {
         auto band_key = [&](int j, bool& ok) -> uint64_t {
-            const double f = (double)row[j];
+            const float f = row[j];
             ok = !(f > hi) && f >= lo;
             return ok ? f64_key(exact(j)) : 0ull;
         };
@@ -634,11 +767,11 @@ __global__ void __launch_bounds__(256) topk_kernel(SelectWorkspace ws, const int
         eq_take = need - gt;
     }
 
-    // emit the kept blocks in ascending order
+    // ---- emit the kept blocks in ascending order
     int pos = 0, band_seen = 0, eq_seen = 0;
     for (int j0 = 0; j0 < nB; j0 += 32) {
         const int j = j0 + lane;
-        const double f = j < nB ? (double)row[j] : -INFINITY;
+        const float f = j < nB ? row[j] : -INFINITY;
         const bool in_a = j < nB && f > hi;
         const bool in_b = j < nB && !in_a && f >= lo;
         const uint32_t bb = __ballot_sync(0xffffffffu, in_b);
