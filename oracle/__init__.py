@@ -53,6 +53,8 @@ def _load():
         _lib.oracle_select_lse.restype = i32
         _lib.oracle_select_lse.argtypes = [vp, vp, i32, i32, i32, i32, vp, i32, i32, f64, i32, i32, vp,
                                            vp, vp]
+        _lib.oracle_qk_norm_rope.restype = i32
+        _lib.oracle_qk_norm_rope.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, f64, f64, vp, vp]
         _lib.oracle_attention.restype = i32
         _lib.oracle_attention.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, i32, vp, vp, i32,
                                           f64, vp, i32, vp, vp]
@@ -181,6 +183,35 @@ def select_lse(q, k, valid_len=None, sparsity: float = 0.0, nsub: int = 4, budge
     if st != 0:
         raise ValueError("kmax smaller than the kept count")
     return (idx, cnt, S) if return_scores else (idx, cnt)
+
+
+def raster_positions(grid_thw, Npad: int, B: int = 1) -> np.ndarray:
+    """int32 [B, Npad, 3] (t, y, x) of tokens n = (t*Hg + y)*Wg + x; padding rows get
+    the positions that the raster order continues with."""
+    T, Hg, Wg = grid_thw
+    n = np.arange(Npad)
+    p = np.stack([n // (Hg * Wg), (n // Wg) % Hg, n % Wg], axis=1).astype(np.int32)
+    return np.ascontiguousarray(np.broadcast_to(p, (B, Npad, 3)))
+
+
+def qk_norm_rope(x, weight, pos, rope_dim: int = 96, base: float = 10000.0, eps: float = 1e-6,
+                 return_unrounded: bool = False):
+    """QK RMSNorm (over D, weight [D]) then 3D RoPE on channels [0, rope_dim), rounding
+    to bf16 after the norm and after the rotation.  Returns bf16 bits [B,H,Npad,D]
+    (and the fp64 values before the last rounding)."""
+    x = _bf16(x)
+    B, H, Npad, D = x.shape
+    w = np.ascontiguousarray(weight, dtype=np.uint16)
+    assert w.shape == (D,)
+    pos = np.ascontiguousarray(pos, dtype=np.int32)
+    assert pos.shape == (B, Npad, 3)
+    out = np.empty_like(x)
+    out64 = np.empty(x.shape) if return_unrounded else None
+    st = _load().oracle_qk_norm_rope(_p(x), _p(w), _p(pos), B, H, Npad, D, int(rope_dim), float(base),
+                                     float(eps), _p(out), _p(out64))
+    if st == -2:
+        raise ValueError("rope_dim must be a multiple of 6 in [0, D]")
+    return (out, out64) if return_unrounded else out
 
 
 def attention(q, k, v, kv_idx, kv_cnt, valid_len=None, scale: float = 0.0, block: int = 64,

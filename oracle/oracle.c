@@ -419,3 +419,83 @@ int oracle_select_lse(const uint16_t* q, const uint16_t* k, int B, int H, int Np
     if (!scores) free(S);
     return status;
 }
+
+/* ---------------------------------------------------------------------------
+ * The producer step before the router: QK RMSNorm with 3D RoPE, then block
+ * pooling.  The page "MiniMax-H3 on 8xH200 benchmark", section on the kernel
+ * layer, fuses the QK RMSNorm and the 3D RoPE of the attention inputs into one
+ * kernel, with head dimension 128 and RoPE dimension 96, on the rounding path
+ * that rounds the normalised value before the rotation.  Per (b, h, token n):
+ *   y_d = bf16( x_d / sqrt(mean_e(x_e^2) + eps) * w_d )        (RMSNorm over D)
+ *   channels [0, rope_dim) form three axes of da = rope_dim/3 channels, for the
+ *   token's (t, y, x) position; channel pair (2i, 2i+1) of axis a turns by
+ *   theta = pos_a * base^(-2i/da):
+ *       o_2i   = bf16( y_2i cos(theta) - y_2i+1 sin(theta) )
+ *       o_2i+1 = bf16( y_2i sin(theta) + y_2i+1 cos(theta) )
+ *   channels [rope_dim, D) pass through: o_d = y_d.
+ * bf16() rounds an fp64 value to the nearest bf16 value, ties to even.
+ * ------------------------------------------------------------------------- */
+
+/* Nearest bf16 value (8 significant bits, exponent range of fp32, ties to even)
+ * of a finite double, as bits.  Rounds once, directly from the double. */
+static uint16_t bf16_rne(double v) {
+    if (v == 0.0) return signbit(v) ? 0x8000u : 0u;
+    double a = fabs(v), r;
+    if (a < ldexp(1.0, -126)) {
+        r = rint(a / ldexp(1.0, -133)) * ldexp(1.0, -133);   /* subnormal grid */
+    } else {
+        int e;
+        double m = frexp(a, &e);          /* a = m 2^e, m in [0.5, 1) */
+        r = ldexp(rint(ldexp(m, 8)), e - 8);  /* 8 significant bits, ties to even */
+    }
+    float f = (float)(signbit(v) ? -r : r);  /* exact: r is a bf16 value */
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return (uint16_t)(u >> 16);
+}
+
+/* x: bf16 [B,H,Npad,D]; w: bf16 [D]; pos: int32 [B][Npad][3] (t, y, x).
+ * out: bf16 [B,H,Npad,D], every row computed; out64 (optional, may be NULL):
+ * fp64 [B,H,Npad,D], the rotated values before their final rounding (for pins).
+ * Returns -2 if rope_dim is not a multiple of 6 in [0, D]. */
+int oracle_qk_norm_rope(const uint16_t* x, const uint16_t* w, const int32_t* pos, int B, int H,
+                        int Npad, int D, int rope_dim, double base, double eps, uint16_t* out,
+                        double* out64) {
+    if (rope_dim < 0 || rope_dim > D || rope_dim % 6 != 0) return -2;
+    const int da = rope_dim / 3;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H; ++h) {
+            double* y = (double*)malloc(sizeof(double) * (size_t)D);
+            for (int n = 0; n < Npad; ++n) {
+                const size_t row = (((size_t)b * H + h) * Npad + n) * (size_t)D;
+                double ss = 0.0;
+                for (int d = 0; d < D; ++d) {
+                    const double v = bf16_to_f64(x[row + d]);
+                    ss += v * v;
+                }
+                const double inv = 1.0 / sqrt(ss / D + eps);
+                for (int d = 0; d < D; ++d)
+                    y[d] = bf16_to_f64(bf16_rne(bf16_to_f64(x[row + d]) * inv * bf16_to_f64(w[d])));
+                const int32_t* p = pos + ((size_t)b * Npad + n) * 3;
+                for (int d = 0; d < D; d += 2) {
+                    double o0 = y[d], o1 = y[d + 1];
+                    if (d < rope_dim) {
+                        const int a = d / da, i = (d % da) / 2;
+                        const double theta = (double)p[a] * pow(base, -2.0 * i / da);
+                        const double c = cos(theta), s = sin(theta);
+                        o0 = y[d] * c - y[d + 1] * s;
+                        o1 = y[d] * s + y[d + 1] * c;
+                    }
+                    if (out64) {
+                        out64[row + d] = o0;
+                        out64[row + d + 1] = o1;
+                    }
+                    out[row + d] = bf16_rne(o0);
+                    out[row + d + 1] = bf16_rne(o1);
+                }
+            }
+            free(y);
+        }
+    return 0;
+}
