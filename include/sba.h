@@ -123,6 +123,48 @@ sba_status sba_pool_select_lse(const void* q, const void* k, int B, int H, int N
                                int budget, int kmax, int32_t* kv_idx, int32_t* kv_cnt,
                                void* workspace, size_t workspace_bytes, void* stream);
 
+/* The producer step before the router, fused with its pooling: QK RMSNorm then 3D
+ * RoPE, as the page "MiniMax-H3 on 8xH200 benchmark" (news.paixiangai.cn), the
+ * kernel layer, fuses them (head dimension 128, RoPE dimension 96, the normalised
+ * value rounded to bf16 before the rotation).  Per (b, h, token n):
+ *   y_d = bf16( x_d / sqrt(mean_e(x_e^2) + eps) * weight_d )
+ *   channels [0, rope_dim) are three axes of da = rope_dim/3 channels for the
+ *   token's position (t, y, x) = pos[b][n]; pair (2i, 2i+1) of axis a turns by
+ *   theta = pos_a * rope_base^(-2i/da):
+ *     out_2i = bf16(y_2i cos theta - y_2i+1 sin theta),
+ *     out_2i+1 = bf16(y_2i sin theta + y_2i+1 cos theta);
+ *   channels [rope_dim, D) pass through (out_d = y_d).
+ * Arithmetic in fp32 (the sines and cosines of fp32 angles), rounded to bf16 at
+ * the two points above, so results can differ from an exact evaluation by one bf16
+ * unit in the last place.  Call once for Q and once for K.
+ *   x         bf16 [B, H, Npad, D] (read); may equal `out` (in place)
+ *   weight    bf16 [D], shared by all heads; 16-byte aligned
+ *   pos       int32 [B, Npad, 3] device, (t, y, x) per token, each in [0, 65536)
+ *             (outside that range the rotation angles are wrong, never a fault);
+ *             every row read
+ *   rope_dim  a multiple of 6 in [0, D] (0 = no rotation)
+ *   rope_base > 0; eps >= 0 (1e-6 is usual)
+ *   out       bf16 [B, H, Npad, D] (written, every row)
+ *   means     fp64 [B, H, Npad/block, D] (written) or NULL: the block means of `out`
+ *             over each sample's valid tokens, bit for bit what sba_block_means
+ *             returns for `out`, ready for sba_pool_select_means.
+ * Errors as the other calls; a bad rope_dim, base or eps is SBA_ERR_INVALID_ARG.
+ * The page defines nothing beyond the fused norm + RoPE; pooling in the same pass
+ * is this library's. */
+sba_status sba_qk_norm_rope_pool(const void* x, const void* weight, const int32_t* pos, int B, int H,
+                                 int Npad, int D, const int32_t* valid_len, int block, int rope_dim,
+                                 double rope_base, float eps, void* out, double* means, void* stream);
+
+/* sba_pool_select with the block means given (as written by sba_qk_norm_rope_pool
+ * or sba_block_means) instead of pooled from Q and K: the same routing, without
+ * the pass over Q and K.  qmean, kmean: fp64 [B, H, Npad/block, D] device, read
+ * while the call runs, blocks past nB_b holding 0.  Other arguments as
+ * sba_pool_select (same workspace size). */
+sba_status sba_pool_select_means(const double* qmean, const double* kmean, int B, int H, int Npad,
+                                 int D, const int32_t* valid_len, int block, double sparsity,
+                                 int kmax, int32_t* kv_idx, int32_t* kv_cnt, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+
 /* Block means of x as fp64 values [B, H, Npad/block, D] (inspection helper;
  * blocks past nB_b are written as 0).  `out` is device memory. */
 sba_status sba_block_means(const void* x, int B, int H, int Npad, int D,

@@ -185,15 +185,6 @@ def select_lse(q, k, valid_len=None, sparsity: float = 0.0, nsub: int = 4, budge
     return (idx, cnt, S) if return_scores else (idx, cnt)
 
 
-def raster_positions(grid_thw, Npad: int, B: int = 1) -> np.ndarray:
-    """int32 [B, Npad, 3] (t, y, x) of tokens n = (t*Hg + y)*Wg + x; padding rows get
-    the positions that the raster order continues with."""
-    T, Hg, Wg = grid_thw
-    n = np.arange(Npad)
-    p = np.stack([n // (Hg * Wg), (n // Wg) % Hg, n % Wg], axis=1).astype(np.int32)
-    return np.ascontiguousarray(np.broadcast_to(p, (B, Npad, 3)))
-
-
 def qk_norm_rope(x, weight, pos, rope_dim: int = 96, base: float = 10000.0, eps: float = 1e-6,
                  return_unrounded: bool = False):
     """QK RMSNorm (over D, weight [D]) then 3D RoPE on channels [0, rope_dim), rounding

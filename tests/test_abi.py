@@ -148,3 +148,27 @@ def test_lse_workspace_size(lib):
     assert four > one
     assert lib.sba_pool_select_lse_workspace_size(1, 24, 32768, 128, 64, 2) == 0
     assert lib.sba_pool_select_lse_workspace_size(1, 24, 32760, 128, 64, 4) == 0
+
+
+def producer(lib, x=A, w=A, pos=A, B=1, H=2, Npad=1024, D=128, vl=NULL, block=64, rd=96, base=10000.0,
+             eps=1e-6, out=A, means=A):
+    return lib.sba_qk_norm_rope_pool(x, w, pos, B, H, Npad, D, vl, block, rd, base, eps, out, means, S)
+
+
+@pytest.mark.parametrize("kwargs,code", [
+    (dict(x=NULL), 1), (dict(w=NULL), 1), (dict(pos=NULL), 1), (dict(out=NULL), 1),
+    (dict(rd=100), 1), (dict(rd=-6), 1), (dict(rd=132), 1), (dict(base=0.0), 1), (dict(base=float("inf")), 1),
+    (dict(eps=float("nan")), 1), (dict(eps=-1.0), 1), (dict(D=96), 2), (dict(Npad=1000), 1),
+    (dict(x=MIS), 3), (dict(w=MIS), 3), (dict(means=MIS), 3), (dict(pos=ctypes.c_void_p(0x10002)), 3),
+])
+def test_producer_rejects(lib, kwargs, code):
+    assert producer(lib, **kwargs) == code
+
+
+def test_pool_select_means_rejects(lib):
+    f = lambda qm=A, km=A, D=128, s=0.5, kmax=8, ws=A, wsb=1 << 30: lib.sba_pool_select_means(
+        qm, km, 1, 2, 1024, D, NULL, 64, s, kmax, A, A, ws, wsb, S)
+    assert f(qm=NULL) == 1 and f(km=NULL) == 1 and f(ws=NULL) == 1
+    assert f(kmax=7) == 1 and f(s=1.0) == 1 and f(wsb=16) == 1
+    assert f(D=80) == 2
+    assert f(qm=MIS) == 3

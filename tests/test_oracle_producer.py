@@ -133,15 +133,17 @@ def test_power_of_two_scalings_are_exact(oracle_mod):
     np.testing.assert_array_equal(f64(o2), 2.0 * f64(o1))  # a doubled weight doubles every output
 
 
-def test_raster_positions(oracle_mod):
-    p = oracle_mod.raster_positions((2, 3, 4), 32, B=2)
-    assert p.shape == (2, 32, 3)
-    n = 17
-    t, y, x = p[1, n]
-    assert (t * 3 + y) * 4 + x == n
+def test_workload_positions():
+    w = make_custom(2, 1, 64, (2, 3, 4), 0.5, drop_rate=0.3, seed=9)
+    for b in range(2):
+        L = int(w.valid_len[b])
+        t, y, x = w.positions[b, :L].T
+        n = (t * 3 + y) * 4 + x
+        assert np.all(np.diff(n) > 0) and n.max() < 24  # kept tokens, raster order
+        assert np.all(w.positions[b, L:] == 0)
 
 
 def test_bad_rope_dim_rejected(oracle_mod):
     w = make_custom(1, 1, 128, (1, 4, 16), 0.5, seed=1)
     with pytest.raises(ValueError):
-        oracle_mod.qk_norm_rope(w.q, bf(np.ones(128)), oracle_mod.raster_positions((1, 4, 16), 64), rope_dim=100)
+        oracle_mod.qk_norm_rope(w.q, bf(np.ones(128)), w.positions, rope_dim=100)

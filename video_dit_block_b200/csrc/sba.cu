@@ -16,6 +16,7 @@
 #include "score_mma.cuh"
 #include "score_lse.cuh"
 #include "pair.cuh"
+#include "producer.cuh"
 
 namespace {
 
@@ -106,10 +107,13 @@ sba_status launch_attention(const void* q, const void* k, const void* v, void* o
 // sub-blocks per block), largest key norm, screened scores on the tensor cores
 // (skipped when nothing is dropped), then the per-row top-k.  Arguments checked
 // by the caller.
+// With qmean/kmean given (fp64 block means [BH][nB][D], NSUB = 1), pooling is replaced
+// by splitting those means for the screen, and the top-k re-scores from them.
 template <int D, int NSUB>
 sba_status run_select(const void* q, const void* k, int B, int H, int Npad, const int32_t* valid_len,
                       double sparsity, int budget, int kmax, int32_t* kv_idx, int32_t* kv_cnt,
-                      void* workspace, cudaStream_t s) {
+                      void* workspace, cudaStream_t s, const double* qmean = nullptr,
+                      const double* kmean = nullptr) {
     constexpr int BLK = 64 / NSUB;
     const size_t BH = (size_t)B * H;
     const int nB = Npad / 64;
@@ -132,10 +136,17 @@ sba_status run_select(const void* q, const void* k, int B, int H, int Npad, cons
                         !make_map(&tkh, ws.khi, (int)BH, nP, D, brows) ||
                         !make_map(&tkl, ws.klo, (int)BH, nP, D, brows)))
         return SBA_ERR_CUDA;
-    sba::pool_kernel<D, BLK><<<pool_grid, 256, 0, s>>>(qb, valid_len, H, Npad, ws.qmean64, ws.qhi, ws.qlo, ws.qnorm,
-                                                       pgroups);
-    sba::pool_kernel<D, BLK><<<pool_grid, 256, 0, s>>>(kb, valid_len, H, Npad, ws.kmean64, ws.khi, ws.klo, ws.knorm,
-                                                       pgroups);
+    if (qmean && kmean) {
+        ws.qmean64 = const_cast<double*>(qmean);
+        ws.kmean64 = const_cast<double*>(kmean);
+        sba::split_means_kernel<D><<<pool_grid, 256, 0, s>>>(qmean, ws.qhi, ws.qlo, ws.qnorm, pgroups);
+        sba::split_means_kernel<D><<<pool_grid, 256, 0, s>>>(kmean, ws.khi, ws.klo, ws.knorm, pgroups);
+    } else {
+        sba::pool_kernel<D, BLK><<<pool_grid, 256, 0, s>>>(qb, valid_len, H, Npad, ws.qmean64, ws.qhi, ws.qlo,
+                                                           ws.qnorm, pgroups);
+        sba::pool_kernel<D, BLK><<<pool_grid, 256, 0, s>>>(kb, valid_len, H, Npad, ws.kmean64, ws.khi, ws.klo,
+                                                           ws.knorm, pgroups);
+    }
     sba::kmax_kernel<<<(unsigned)((BH + 7) / 8), 256, 0, s>>>(ws, valid_len, H, Npad, (int)BH, BLK);
     if (need_scores && NSUB == 1) {
         using SM = sba::ScoreSmem<D>;
@@ -198,6 +209,59 @@ sba_status sba_pool_select(const void* q, const void* k, int B, int H, int Npad,
     if (D == 128)
         return run_select<128, 1>(q, k, B, H, Npad, valid_len, sparsity, 1, kmax, kv_idx, kv_cnt, workspace, s);
     return run_select<64, 1>(q, k, B, H, Npad, valid_len, sparsity, 1, kmax, kv_idx, kv_cnt, workspace, s);
+}
+
+sba_status sba_pool_select_means(const double* qmean, const double* kmean, int B, int H, int Npad, int D,
+                                 const int32_t* valid_len, int block, double sparsity, int kmax,
+                                 int32_t* kv_idx, int32_t* kv_cnt, void* workspace, size_t workspace_bytes,
+                                 void* stream) {
+    sba_status st = check_shape(B, H, Npad, D, block);
+    if (st != SBA_OK) return st;
+    if (!qmean || !kmean || !kv_idx || !kv_cnt || !workspace) return SBA_ERR_INVALID_ARG;
+    if (!(sparsity >= 0.0 && sparsity < 1.0)) return SBA_ERR_INVALID_ARG;
+    const int nB = Npad / block;
+    if (kmax < sba::keep_count(nB, sparsity)) return SBA_ERR_INVALID_ARG;
+    if (workspace_bytes < sba::select_workspace_bytes((size_t)B * H, nB, D)) return SBA_ERR_INVALID_ARG;
+    if (!aligned16(qmean) || !aligned16(kmean) || !aligned16(workspace) || !aligned16(valid_len))
+        return SBA_ERR_ALIGNMENT;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (D == 128)
+        return run_select<128, 1>(nullptr, nullptr, B, H, Npad, valid_len, sparsity, 1, kmax, kv_idx, kv_cnt,
+                                  workspace, s, qmean, kmean);
+    return run_select<64, 1>(nullptr, nullptr, B, H, Npad, valid_len, sparsity, 1, kmax, kv_idx, kv_cnt, workspace,
+                             s, qmean, kmean);
+}
+
+sba_status sba_qk_norm_rope_pool(const void* x, const void* weight, const int32_t* pos, int B, int H, int Npad,
+                                 int D, const int32_t* valid_len, int block, int rope_dim, double rope_base,
+                                 float eps, void* out, double* means, void* stream) {
+    sba_status st = check_shape(B, H, Npad, D, block);
+    if (st != SBA_OK) return st;
+    if (!x || !weight || !pos || !out) return SBA_ERR_INVALID_ARG;
+    if (rope_dim < 0 || rope_dim > D || rope_dim % 6 != 0 || rope_dim / 6 > sba::kMaxRopePairs)
+        return SBA_ERR_INVALID_ARG;
+    if (!(rope_base > 0.0) || !std::isfinite(rope_base) || !(eps >= 0.f) || !std::isfinite(eps))
+        return SBA_ERR_INVALID_ARG;
+    if ((long long)B * H * (Npad / block) > 0x7fffffffll) return SBA_ERR_UNSUPPORTED;
+    if (!aligned16(x) || !aligned16(out) || !aligned16(weight) || !aligned16(means) || !aligned16(valid_len) ||
+        (reinterpret_cast<uintptr_t>(pos) & 3u))
+        return SBA_ERR_ALIGNMENT;
+    sba::RopeFreqs f;
+    const int da = rope_dim / 3;
+    for (int i = 0; i < sba::kMaxRopePairs; ++i)
+        f.inv_freq[i] = (da > 0 && 2 * i < da) ? (float)std::pow(rope_base, -2.0 * i / da) : 0.f;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const unsigned grid = (unsigned)((long long)B * H * (Npad / block));
+    const auto* xb = static_cast<const __nv_bfloat16*>(x);
+    const auto* wb = static_cast<const __nv_bfloat16*>(weight);
+    auto* ob = static_cast<__nv_bfloat16*>(out);
+    if (D == 128)
+        sba::qk_norm_rope_pool_kernel<128><<<grid, 256, 0, s>>>(xb, wb, pos, valid_len, H, Npad, rope_dim, f, eps, ob,
+                                                                means);
+    else
+        sba::qk_norm_rope_pool_kernel<64><<<grid, 256, 0, s>>>(xb, wb, pos, valid_len, H, Npad, rope_dim, f, eps, ob,
+                                                               means);
+    return cudaGetLastError() == cudaSuccess ? SBA_OK : SBA_ERR_CUDA;
 }
 
 size_t sba_pool_select_lse_workspace_size(int B, int H, int Npad, int D, int block, int nsub) {

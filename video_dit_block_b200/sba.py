@@ -51,6 +51,10 @@ def lib() -> ctypes.CDLL:
         L.sba_pool_select_lse.restype = i32
         L.sba_pool_select_lse.argtypes = [vp, vp, i32, i32, i32, i32, vp, i32, i32, f64, i32, i32, vp, vp, vp,
                                           sz, vp]
+        L.sba_qk_norm_rope_pool.restype = i32
+        L.sba_qk_norm_rope_pool.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, i32, i32, f64, f32, vp, vp, vp]
+        L.sba_pool_select_means.restype = i32
+        L.sba_pool_select_means.argtypes = [vp, vp, i32, i32, i32, i32, vp, i32, f64, i32, vp, vp, vp, sz, vp]
         L.sba_block_means.restype = i32
         L.sba_block_means.argtypes = [vp, i32, i32, i32, i32, vp, i32, vp, vp]
         L.sba_attention.restype = i32
@@ -175,6 +179,51 @@ def pool_select_lse(q, k, valid_len=None, sparsity: float = 0.0, nsub: int = 4, 
                                      float(sparsity), int(budget), int(kmax), _ptr(kv_idx), _ptr(kv_cnt),
                                      _ptr(workspace), workspace.numel() * workspace.element_size(),
                                      _stream(stream)), "sba_pool_select_lse")
+    return kv_idx, kv_cnt
+
+
+def qk_norm_rope_pool(x, weight, pos, valid_len=None, rope_dim: int = 96, rope_base: float = 10000.0,
+                      eps: float = 1e-6, out=None, means=None, want_means: bool = True, block: int = BLOCK,
+                      stream=None):
+    """QK RMSNorm + 3D RoPE (see include/sba.h), with the block means of the output.
+    weight: bf16 [D]; pos: int32 [B, Npad, 3].  Returns (out bf16, means fp64 or None)."""
+    B, H, Npad, D = _qkv(x)
+    if not (weight.is_cuda and weight.dtype == torch.bfloat16 and weight.shape == (D,) and weight.is_contiguous()):
+        raise ValueError("weight must be a contiguous bf16 CUDA tensor [D]")
+    if not (pos.is_cuda and pos.dtype == torch.int32 and pos.shape == (B, Npad, 3) and pos.is_contiguous()):
+        raise ValueError("pos must be a contiguous int32 CUDA tensor [B, Npad, 3]")
+    if out is None:
+        out = torch.empty_like(x)
+    if means is None and want_means:
+        means = torch.empty((B, H, Npad // block, D), dtype=torch.float64, device=x.device)
+    _check(lib().sba_qk_norm_rope_pool(_ptr(x), _ptr(weight), _ptr(pos), B, H, Npad, D,
+                                       _ptr(_valid_len(valid_len, x.device)), block, int(rope_dim),
+                                       float(rope_base), float(eps), _ptr(out), _ptr(means), _stream(stream)),
+           "sba_qk_norm_rope_pool")
+    return out, means
+
+
+def pool_select_means(qmean, kmean, valid_len=None, sparsity: float = 0.0, kmax: int | None = None,
+                      block: int = BLOCK, kv_idx=None, kv_cnt=None, workspace=None, stream=None):
+    """Routing from given fp64 block means [B, H, Npad/64, D] (no pass over Q and K)."""
+    B, H, nB, D = qmean.shape
+    for t in (qmean, kmean):
+        if not (t.is_cuda and t.dtype == torch.float64 and t.is_contiguous() and t.shape == (B, H, nB, D)):
+            raise ValueError("qmean / kmean must be contiguous fp64 CUDA tensors [B, H, Npad/64, D]")
+    Npad = nB * block
+    vl = _valid_len(valid_len, qmean.device)
+    if kmax is None:
+        kmax = kmax_for(Npad, sparsity, block)
+    if kv_idx is None:
+        kv_idx = torch.empty((B, H, nB, kmax), dtype=torch.int32, device=qmean.device)
+    if kv_cnt is None:
+        kv_cnt = torch.empty((B, H, nB), dtype=torch.int32, device=qmean.device)
+    if workspace is None:
+        workspace = torch.empty(workspace_size(B, H, Npad, D, block), dtype=torch.uint8, device=qmean.device)
+    _check(lib().sba_pool_select_means(_ptr(qmean), _ptr(kmean), B, H, Npad, D, _ptr(vl), block, float(sparsity),
+                                       int(kmax), _ptr(kv_idx), _ptr(kv_cnt), _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(), _stream(stream)),
+           "sba_pool_select_means")
     return kv_idx, kv_cnt
 
 

@@ -69,6 +69,9 @@ class Workload:
     block: int = BLOCK
     grid: tuple = ()
     seed: int = 0
+    # int32 [B, Npad, 3]: (t, y, x) latent-grid position of each kept token (raster
+    # order n = (t*Hg + y)*Wg + x before pruning); padding rows are (0, 0, 0)
+    positions: np.ndarray | None = None
 
     @property
     def B(self):
@@ -167,8 +170,20 @@ def _build(name, B, H, D, grid, sparsity, sigma, per_head_freq, drop_rate, seed,
     # every job owns its own generators, so the result does not depend on scheduling.
     with concurrent.futures.ThreadPoolExecutor(max_workers=min(len(jobs), os.cpu_count() or 1)) as ex:
         list(ex.map(one, jobs))
+    pos = np.zeros((B, Npad, 3), dtype=np.int32)
+    for b in range(B):
+        r = keep_rows[b]
+        pos[b, :len(r)] = np.stack([r // (Hg * Wg), (r // Wg) % Hg, r % Wg], axis=1)
     return Workload(name=name, q=out["q"], k=out["k"], v=out["v"], valid_len=valid_len,
-                    sparsity=float(sparsity), grid=tuple(grid), seed=seed)
+                    sparsity=float(sparsity), grid=tuple(grid), seed=seed, positions=pos)
+
+
+def make_norm_weights(D: int, seed: int = 7):
+    """Per-channel RMSNorm weights for Q and K: bf16 bits [D] each, drawn from
+    U[0.5, 1.5) (learned QK-norm scales sit near 1)."""
+    wq = f64_to_bf16_bits(_rng(seed, 11).uniform(0.5, 1.5, size=D))
+    wk = f64_to_bf16_bits(_rng(seed, 12).uniform(0.5, 1.5, size=D))
+    return wq, wk
 
 
 def make_workload(name: str, heads: int | None = None, pad_value: float = 0.0) -> Workload:
