@@ -10,7 +10,10 @@ sba_attention_paired over the kept blocks.  Prints ONE JSON line (rank 0).
 
 `--router lse` routes with the sub-block log-sum-exp score (sba_pool_select_lse,
 16-token sub-blocks) and `--budget` rounds its kept count up to a multiple of B
-blocks; the default is the block-mean router with no rounding.
+blocks; the default is the block-mean router with no rounding.  `--producer` treats
+the workload's Q and K as the pre-norm projections: each step first applies QK
+RMSNorm + 3D RoPE with the block pooling fused (sba_qk_norm_rope_pool), then routes
+from those means (sba_pool_select_means) and attends over the normalised Q and K.
 
 Metric: effective TFLOP/s on the kept blocks, counted as
 4 * D * sum_{b,h,I} c_I * sum_{J kept} c_J (c = valid tokens of a block), divided by
@@ -52,6 +55,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--router", default="mean", choices=["mean", "lse"])
     ap.add_argument("--budget", type=int, default=1)
+    ap.add_argument("--producer", action="store_true")
     return ap.parse_args()
 
 
@@ -161,7 +165,7 @@ def whole_job_value(kept_flops_per_rank, ms_per_step, world):
     return world * kept_flops_per_rank / (ms_per_step * 1e-3) / 1e12
 
 
-def oracle_sample(w, target_s=10.0, seed=0, router="mean", budget=1):
+def oracle_sample(w, target_s=10.0, seed=0, router="mean", budget=1, producer=False):
     """Time the fp64 oracle, as it stands, on a bounded sample of the workload: the
     full routing of head (b=0, h=0) and the attention of a seeded subset of that head's
     query blocks, sized to about `target_s` seconds.
@@ -173,6 +177,13 @@ def oracle_sample(w, target_s=10.0, seed=0, router="mean", budget=1):
     q1, k1, v1 = (np.ascontiguousarray(x[:1, :1]) for x in (w.q, w.k, w.v))
     vl1 = np.ascontiguousarray(w.valid_len[:1])
     t0 = time.perf_counter()
+    if producer:
+        from workloads import make_norm_weights
+        wq, wk = make_norm_weights(w.q.shape[3])
+        pos1 = np.ascontiguousarray(w.positions[:1])
+        rd = 3 * w.q.shape[3] // 4  # 96 for D = 128 (the page's setting), 48 for D = 64
+        q1 = oracle.qk_norm_rope(q1, wq, pos1, rope_dim=rd)
+        k1 = oracle.qk_norm_rope(k1, wk, pos1, rope_dim=rd)
     if router == "lse":
         idx, cnt = oracle.select_lse(q1, k1, vl1, w.sparsity, budget=budget)
     else:
@@ -216,9 +227,11 @@ def workload_config(w, extra=None):
 
 
 def router_config(args):
-    if args.router == "mean":
-        return {"router": "block mean"}
-    return {"router": "sub-block log-sum-exp (4 x 16 tokens)", "budget": args.budget}
+    c = {"router": "block mean"} if args.router == "mean" else {
+        "router": "sub-block log-sum-exp (4 x 16 tokens)", "budget": args.budget}
+    if args.producer:
+        c["producer"] = "QK RMSNorm + 3D RoPE (rope_dim 3D/4, base 1e4, eps 1e-6) with fused block pooling"
+    return c
 
 
 def run_reference(args):
@@ -230,7 +243,8 @@ def run_reference(args):
     per = []
     target = max(2.0, 60.0 / max(1, args.steps + args.warmup))
     for i in range(args.warmup + args.steps):
-        s = oracle_sample(w, target_s=target, seed=i, router=args.router, budget=args.budget)
+        s = oracle_sample(w, target_s=target, seed=i, router=args.router, budget=args.budget,
+                          producer=args.producer)
         if i >= args.warmup:
             per.append(s)
     value = statistics.mean(s["value"] for s in per)
@@ -285,21 +299,40 @@ def run_ours(args):
     pws = torch.empty(int(sba.lib().sba_pair_workspace_size(B, H, Npad, 64)), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def route(qq=q, kk=k, vll=vl):
+    if args.producer:
         if lse_router:
+            raise SystemExit("--producer routes from block means: use the block-mean router")
+        from workloads import make_norm_weights
+        wq, wk = (t(x) for x in make_norm_weights(D))
+        pos = torch.from_numpy(w.positions).to(dev)
+        q_n, k_n = torch.empty_like(q), torch.empty_like(k)
+        q_m = torch.empty((B, H, Npad // 64, D), dtype=torch.float64, device=dev)
+        k_m = torch.empty_like(q_m)
+
+    def route(qq=q, kk=k, vll=vl):
+        """Routing (and, with --producer, the norm + RoPE before it); returns the Q, K
+        the attention reads."""
+        if args.producer:
+            sba.qk_norm_rope_pool(qq, wq, pos, vll, rope_dim=3 * D // 4, out=q_n, means=q_m, stream=stream)
+            sba.qk_norm_rope_pool(kk, wk, pos, vll, rope_dim=3 * D // 4, out=k_n, means=k_m, stream=stream)
+            sba.pool_select_means(q_m, k_m, vll, w.sparsity, kmax, kv_idx=kv_idx, kv_cnt=kv_cnt, workspace=ws,
+                                  stream=stream)
+            qq, kk = q_n, k_n
+        elif lse_router:
             sba.pool_select_lse(qq, kk, vll, w.sparsity, budget=args.budget, kmax=kmax, kv_idx=kv_idx,
                                 kv_cnt=kv_cnt, workspace=ws, stream=stream)
         else:
             sba.pool_select(qq, kk, vll, w.sparsity, kmax, kv_idx=kv_idx, kv_cnt=kv_cnt, workspace=ws,
                             stream=stream)
         sba.pair_query_blocks(kv_idx, kv_cnt, vll, pair_order=pair_order, workspace=pws, stream=stream)
+        return qq, kk
 
     def attend(qq=q, kk=k, vv=v, vll=vl):
         sba.attention_paired(qq, kk, vv, kv_idx, kv_cnt, pair_order, vll, out=o, lse=lse, stream=stream)
 
     def step(qq=q, kk=k, vv=v):
-        route(qq, kk)
-        attend(qq, kk, vv)
+        qa, ka = route(qq, kk)
+        attend(qa, ka, vv)
 
     def barrier():
         if dist is not None:
@@ -323,9 +356,9 @@ def run_ours(args):
     time.sleep(0.3)
     for i in range(K):
         ev[i][0].record(stream)
-        route()
+        qa, ka = route()
         ev[i][1].record(stream)
-        attend()
+        attend(qa, ka)
         ev[i][2].record(stream)
     torch.cuda.synchronize(dev)
     clk = clocks.stop()
@@ -357,8 +390,8 @@ def run_ours(args):
             kd.copy_(kh, non_blocking=True)
             vd.copy_(vh, non_blocking=True)
             vld.copy_(vlh, non_blocking=True)
-            route(qd, kd, vld)
-            attend(qd, kd, vd, vld)
+            qa, ka = route(qd, kd, vld)
+            attend(qa, ka, vd, vld)
             oh.copy_(o, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize(dev)
@@ -392,14 +425,15 @@ def run_ours(args):
                      "traffic": traffic},
         # per step: routing = 2 pooling + key-norm maximum + screen (only when blocks are
         # dropped) + top-k; pairing = bitmaps + 4 x (propose, resolve) + emit; 1 attention
-        "gpu_launches": (4 + (1 if w.sparsity > 0 else 0) + 10 + 1) * K,
+        # (--producer: 2 producer launches and 2 splits of the given means replace pooling)
+        "gpu_launches": (4 + (1 if w.sparsity > 0 else 0) + (2 if args.producer else 0) + 10 + 1) * K,
         "clocks": clk,
     }
     if e2e is not None:
         line["e2e"] = e2e
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_from(oracle_sample(w, target_s=15.0, router=args.router,
-                                                               budget=args.budget))
+                                                               budget=args.budget, producer=args.producer))
     print(json.dumps(line), flush=True)
     if dist is not None:
         dist.destroy_process_group()
