@@ -327,8 +327,8 @@ def run_ours(args):
         sba.pair_query_blocks(kv_idx, kv_cnt, vll, pair_order=pair_order, workspace=pws, stream=stream)
         return qq, kk
 
-    def attend(qq=q, kk=k, vv=v, vll=vl):
-        sba.attention_paired(qq, kk, vv, kv_idx, kv_cnt, pair_order, vll, out=o, lse=lse, stream=stream)
+    def attend(qq=q, kk=k, vv=v, vll=vl, out=o):
+        sba.attention_paired(qq, kk, vv, kv_idx, kv_cnt, pair_order, vll, out=out, lse=lse, stream=stream)
 
     def step(qq=q, kk=k, vv=v):
         qa, ka = route(qq, kk)
@@ -372,33 +372,60 @@ def run_ours(args):
     ms_step = total_ms / K
     value = whole_job_value(f_step, ms_step, world)
 
-    # ---- end to end through the public API with host buffers
+    # ---- end to end through the public API with host buffers: every step uploads its
+    # inputs from pinned host memory and downloads its output.  The steps are pipelined
+    # the way a serving loop would run them: inputs and outputs are double-buffered on
+    # the device, uploads run on one stream, compute on the launching stream and
+    # downloads on a third, ordered by events, so step i+1's upload and step i-1's
+    # download overlap step i's compute.  Timed from the first upload to the last
+    # download.
     e2e = None
     if not args.no_e2e:
         qh, kh, vh = (x.cpu().pin_memory() for x in (q, k, v))
         vlh = vl.cpu().pin_memory()
         oh = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-        qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-        vld = torch.empty_like(vl)
-        Ke = max(2, K // 2)
+        bufs = [(torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(vl))
+                for _ in range(2)]
+        outs = [o, torch.empty_like(o)]
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        in_done = [torch.cuda.Event() for _ in range(2)]
+        comp_done = [torch.cuda.Event() for _ in range(2)]
+        out_done = [torch.cuda.Event() for _ in range(2)]
+        Ke = max(4, K)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier()
         torch.cuda.synchronize(dev)
-        e0.record(stream)
-        for _ in range(Ke):
-            qd.copy_(qh, non_blocking=True)
-            kd.copy_(kh, non_blocking=True)
-            vd.copy_(vh, non_blocking=True)
-            vld.copy_(vlh, non_blocking=True)
+        e0.record(s_in)
+        for i in range(Ke):
+            bi_ = i % 2
+            qd, kd, vd, vld = bufs[bi_]
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(comp_done[bi_])   # step i-2 has finished reading this buffer
+                qd.copy_(qh, non_blocking=True)
+                kd.copy_(kh, non_blocking=True)
+                vd.copy_(vh, non_blocking=True)
+                vld.copy_(vlh, non_blocking=True)
+                in_done[bi_].record(s_in)
+            stream.wait_event(in_done[bi_])
+            if i >= 2:
+                stream.wait_event(out_done[bi_])      # step i-2's output has been downloaded
             qa, ka = route(qd, kd, vld)
-            attend(qa, ka, vd, vld)
-            oh.copy_(o, non_blocking=True)
-        e1.record(stream)
+            attend(qa, ka, vd, vld, out=outs[bi_])
+            comp_done[bi_].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(comp_done[bi_])
+                oh.copy_(outs[bi_], non_blocking=True)
+                out_done[bi_].record(s_out)
+        e1.record(s_out)
         torch.cuda.synchronize(dev)
+        if sba.device_status(stream) != 0:
+            raise RuntimeError("device status error in the end-to-end loop")
         e_ms = max_over_ranks([e0.elapsed_time(e1) / Ke], dist, dev)[0]
         bi = 3 * q.numel() * 2 + vl.numel() * 4
         e2e = {"value": whole_job_value(f_step, e_ms, world), "unit": "TFLOP/s",
-               "ms_per_step": e_ms, "h2d_bytes_per_step": bi, "d2h_bytes_per_step": o.numel() * 2}
+               "ms_per_step": e_ms, "h2d_bytes_per_step": bi, "d2h_bytes_per_step": o.numel() * 2,
+               "steps": Ke, "mode": "pipelined: double-buffered uploads, compute and downloads on three streams"}
 
     if rank != 0:
         if dist is not None:
