@@ -55,6 +55,9 @@ def _load():
                                            vp, vp]
         _lib.oracle_qk_norm_rope.restype = i32
         _lib.oracle_qk_norm_rope.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, f64, f64, vp, vp]
+        _lib.oracle_attention_compensated.restype = i32
+        _lib.oracle_attention_compensated.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, i32, vp, vp, i32,
+                                                      f64, vp, i32, vp, vp]
         _lib.oracle_attention.restype = i32
         _lib.oracle_attention.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, i32, vp, vp, i32,
                                           f64, vp, i32, vp, vp]
@@ -222,6 +225,26 @@ def attention(q, k, v, kv_idx, kv_cnt, valid_len=None, scale: float = 0.0, block
     st = _load().oracle_attention(_p(q), _p(k), _p(v), B, H, Npad, D, _p(vl), block, _p(kv_idx),
                                   _p(kv_cnt), kmax, float(scale), _p(qb),
                                   0 if qb is None else len(qb), _p(o), _p(lse))
+    if st != 0:
+        raise ValueError("routing entry outside the sample's blocks")
+    return o, lse
+
+
+def attention_compensated(q, k, v, kv_idx, kv_cnt, valid_len=None, scale: float = 0.0, block: int = 64,
+                          qblocks=None):
+    """Block-sparse attention with each dropped block compensated by its (bf16) mean key
+    and value, weighted by its token count.  Returns (o, lse) like `attention`."""
+    q, k, v = _bf16(q), _bf16(k), _bf16(v)
+    B, H, Npad, D = q.shape
+    vl = _vl(valid_len, B, Npad)
+    kv_idx = np.ascontiguousarray(kv_idx, dtype=np.int32)
+    kv_cnt = np.ascontiguousarray(kv_cnt, dtype=np.int32)
+    o = np.full((B, H, Npad, D), np.nan)
+    lse = np.full((B, H, Npad), np.nan)
+    qb = None if qblocks is None else np.ascontiguousarray(qblocks, dtype=np.int32)
+    st = _load().oracle_attention_compensated(_p(q), _p(k), _p(v), B, H, Npad, D, _p(vl), block, _p(kv_idx),
+                                              _p(kv_cnt), kv_idx.shape[3], float(scale), _p(qb),
+                                              0 if qb is None else len(qb), _p(o), _p(lse))
     if st != 0:
         raise ValueError("routing entry outside the sample's blocks")
     return o, lse

@@ -499,3 +499,121 @@ int oracle_qk_norm_rope(const uint16_t* x, const uint16_t* w, const int32_t* pos
         }
     return 0;
 }
+
+/* ---------------------------------------------------------------------------
+ * Block-sparse attention with compensation of the dropped blocks.  PISA, as the
+ * page "Sol Video Inference Engine" (sjmshsh.github.io) describes it in section
+ * 4.2.2 (Sparse Attention), computes the critical blocks exactly and compensates
+ * the others by a first-order Taylor approximation.  Expanding exp(s q.k_j) about the mean key kbar_J
+ * of a dropped block J, the sum over its tokens is c_J exp(s q.kbar_J) to first
+ * order (the linear term sums to zero about the mean); the numerator's
+ * zeroth-order term is exp(s q.kbar_J) sum_j v_j = c_J exp(s q.kbar_J) vbar_J.
+ * So each dropped block enters the softmax as one entry of logit
+ * s q.kbar_J + log(c_J) carrying the value vbar_J:
+ *   o_i = [sum_{j kept} e^{s q.k_j} v_j + sum_{J dropped} c_J e^{s q.kbar_J} vbar_J]
+ *         / [sum_{j kept} e^{s q.k_j} + sum_{J dropped} c_J e^{s q.kbar_J}]
+ * with kbar_J, vbar_J the means of the valid tokens of block J (token order,
+ * fp64) rounded to bf16, c_J their count; "dropped" = the sample's blocks not in
+ * the row's kept list.  Exact when keys are constant within every dropped block.
+ * Same arguments and outputs as oracle_attention. */
+int oracle_attention_compensated(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int H,
+                                 int Npad, int D, const int32_t* valid_len, int block, const int32_t* kv_idx,
+                                 const int32_t* kv_cnt, int kmax, double scale, const int32_t* qblocks,
+                                 int n_qblocks, double* o, double* lse) {
+    const int nBmax = Npad / block;
+    const int nq = qblocks ? n_qblocks : nBmax;
+    if (scale <= 0.0) scale = 1.0 / sqrt((double)D);
+    const size_t nm = (size_t)B * H * nBmax * D;
+    double* km = (double*)malloc(sizeof(double) * nm);
+    double* vm = (double*)malloc(sizeof(double) * nm);
+    oracle_pool(k, B, H, Npad, D, valid_len, block, km);
+    oracle_pool(v, B, H, Npad, D, valid_len, block, vm);
+    for (size_t t = 0; t < nm; ++t) {   /* the means, rounded to bf16 */
+        km[t] = bf16_to_f64(bf16_rne(km[t]));
+        vm[t] = bf16_to_f64(bf16_rne(vm[t]));
+    }
+    int status = 0;
+#pragma omp parallel
+    {
+        int32_t* tok = (int32_t*)malloc(sizeof(int32_t) * (size_t)Npad);
+        double* lg = (double*)malloc(sizeof(double) * (size_t)(Npad + nBmax));
+        char* kept = (char*)malloc((size_t)(nBmax > 0 ? nBmax : 1));
+#pragma omp for collapse(3) schedule(dynamic)
+        for (int b = 0; b < B; ++b)
+            for (int h = 0; h < H; ++h)
+                for (int qi = 0; qi < nq; ++qi) {
+                    const int I = qblocks ? qblocks[qi] : qi;
+                    const int L = valid_len[b], nB = n_blocks_of(L, block);
+                    const size_t bh = (size_t)b * H + h;
+                    const uint16_t* ks = k + bh * (size_t)Npad * D;
+                    const uint16_t* vs = v + bh * (size_t)Npad * D;
+                    const double* kmb = km + bh * (size_t)nBmax * D;
+                    const double* vmb = vm + bh * (size_t)nBmax * D;
+                    const size_t r = bh * nBmax + I;
+                    int n = kept_tokens(kv_idx + r * kmax, kv_cnt[r], nB, L, block, tok);
+                    if (n < 0) {
+#pragma omp atomic write
+                        status = -1;
+                        n = 0;
+                    }
+                    for (int J = 0; J < nBmax; ++J) kept[J] = 0;
+                    if (n > 0)
+                        for (int t = 0; t < kv_cnt[r]; ++t) kept[kv_idx[r * kmax + t]] = 1;
+                    for (int i = I * block; i < (I + 1) * block; ++i) {
+                        double* orow = o + (bh * Npad + i) * D;
+                        double* l = lse + bh * Npad + i;
+                        for (int d = 0; d < D; ++d) orow[d] = 0.0;
+                        if (i >= L || I >= nB) {
+                            *l = -INFINITY;
+                            continue;
+                        }
+                        const uint16_t* qr = q + (bh * Npad + i) * D;
+                        /* logits: kept tokens, then one entry per dropped block */
+                        double m = -INFINITY;
+                        int ne = 0;
+                        for (int t = 0; t < n; ++t) {
+                            const uint16_t* kr = ks + (size_t)tok[t] * D;
+                            double s = 0.0;
+                            for (int d = 0; d < D; ++d) s += bf16_to_f64(qr[d]) * bf16_to_f64(kr[d]);
+                            lg[ne] = scale * s;
+                            if (lg[ne] > m) m = lg[ne];
+                            ++ne;
+                        }
+                        for (int J = 0; J < nB; ++J) {
+                            if (kept[J]) continue;
+                            int c = L - J * block;
+                            c = c > block ? block : c;
+                            double s = 0.0;
+                            for (int d = 0; d < D; ++d) s += bf16_to_f64(qr[d]) * kmb[(size_t)J * D + d];
+                            lg[ne] = scale * s + log((double)c);
+                            if (lg[ne] > m) m = lg[ne];
+                            ++ne;
+                        }
+                        if (ne == 0) {
+                            *l = -INFINITY;
+                            continue;
+                        }
+                        double Z = 0.0;
+                        for (int e = 0; e < ne; ++e) { lg[e] = exp(lg[e] - m); Z += lg[e]; }
+                        int e = 0;
+                        for (int t = 0; t < n; ++t, ++e) {
+                            const uint16_t* vr = vs + (size_t)tok[t] * D;
+                            const double w = lg[e] / Z;
+                            for (int d = 0; d < D; ++d) orow[d] += w * bf16_to_f64(vr[d]);
+                        }
+                        for (int J = 0; J < nB; ++J) {
+                            if (kept[J]) continue;
+                            const double w = lg[e++] / Z;
+                            for (int d = 0; d < D; ++d) orow[d] += w * vmb[(size_t)J * D + d];
+                        }
+                        *l = m + log(Z);
+                    }
+                }
+        free(tok);
+        free(lg);
+        free(kept);
+    }
+    free(km);
+    free(vm);
+    return status;
+}
