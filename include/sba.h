@@ -165,6 +165,31 @@ sba_status sba_pool_select_means(const double* qmean, const double* kmean, int B
                                  int kmax, int32_t* kv_idx, int32_t* kv_cnt, void* workspace,
                                  size_t workspace_bytes, void* stream);
 
+/* Bytes of device workspace sba_attention_compensated needs (0 on bad arguments):
+ * the bf16 block means of K and V. */
+size_t sba_compensation_workspace_size(int B, int H, int Npad, int D, int block);
+
+/* Block-sparse attention with compensation of the dropped blocks.  PISA, as the page
+ * "Sol Video Inference Engine" (sjmshsh.github.io), section 4.2.2, describes it,
+ * computes the critical blocks exactly and compensates the others by a first-order
+ * Taylor approximation; about a dropped block's mean key the expansion gives the
+ * block one softmax entry (the normaliser's linear term sums to zero):
+ *   o_i = [sum_{j kept} e^{s q.k_j} v_j + sum_{J dropped} c_J e^{s q.kbar_J} vbar_J]
+ *         / [sum_{j kept} e^{s q.k_j} + sum_{J dropped} c_J e^{s q.kbar_J}]
+ *   lse_i = log of the denominator
+ * where "dropped" are the sample's blocks J < nB_b missing from the row's kept list,
+ * kbar_J / vbar_J are the means of the valid tokens of block J (fp64 sums, rounded
+ * to bf16) and c_J their count.  Exact when keys are constant within each dropped
+ * block.  Arguments as sba_attention_paired (pair_order may be NULL for adjacent
+ * tiles), plus a workspace of at least sba_compensation_workspace_size bytes
+ * (16-byte aligned; contents on entry ignored).  Cost: the kept blocks plus
+ * ceil(nB/64) further 64-column steps per tile. */
+sba_status sba_attention_compensated(const void* q, const void* k, const void* v, void* o, float* lse,
+                                     int B, int H, int Npad, int D, const int32_t* valid_len, int block,
+                                     const int32_t* kv_idx, const int32_t* kv_cnt, int kmax,
+                                     const int32_t* pair_order, float softmax_scale, void* workspace,
+                                     size_t workspace_bytes, void* stream);
+
 /* Block means of x as fp64 values [B, H, Npad/block, D] (inspection helper;
  * blocks past nB_b are written as 0).  `out` is device memory. */
 sba_status sba_block_means(const void* x, int B, int H, int Npad, int D,

@@ -172,3 +172,14 @@ def test_pool_select_means_rejects(lib):
     assert f(kmax=7) == 1 and f(s=1.0) == 1 and f(wsb=16) == 1
     assert f(D=80) == 2
     assert f(qm=MIS) == 3
+
+
+def test_compensated_rejects(lib):
+    f = lambda q=A, v=A, idx=A, cnt=A, kmax=8, D=128, ws=A, wsb=1 << 30, po=NULL: lib.sba_attention_compensated(
+        q, A, v, A, A, 1, 2, 1024, D, NULL, 64, idx, cnt, kmax, po, 0.0, ws, wsb, S)
+    assert lib.sba_compensation_workspace_size(1, 2, 1024, 128, 64) > 0
+    assert lib.sba_compensation_workspace_size(1, 2, 1000, 128, 64) == 0
+    assert f(q=NULL) == 1 and f(v=NULL) == 1 and f(idx=NULL) == 1 and f(cnt=NULL) == 1
+    assert f(ws=NULL) == 1 and f(wsb=16) == 1 and f(kmax=0) == 1
+    assert f(D=96) == 2
+    assert f(ws=MIS) == 3 and f(po=ctypes.c_void_p(0x10002)) == 3

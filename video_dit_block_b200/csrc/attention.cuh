@@ -31,6 +31,14 @@
 //
 // Every wait is bounded: on expiry the CTA records SBA_ERR_TIMEOUT, unwinds all
 // roles, drains its own TMA loads and MMAs and frees its TMEM.
+//
+// COMP = true adds the compensation of the dropped blocks (the first-order
+// expansion of their exponentials about their mean key): after the union walk, the
+// tile walks the rows of kbar / vbar (the bf16 block means, [BH][nBpad][D]) as
+// further 64-column steps, column c of step b standing for block J = 64 b + c with
+// logit s q.kbar_J + log(c_J); a column is masked for a half whose query block
+// keeps J, and past the sample's blocks.  The online softmax then merges the two
+// parts exactly as it merges key blocks.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -88,10 +96,11 @@ __device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, uint64
     return true;
 }
 
-template <int D, int NS>
-__global__ void __launch_bounds__(192, 2)
-    attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+// The body of both kernels below; the tensor maps are the kernels' own __grid_constant__
+// parameters, passed by address (the plain kernel keeps its three-map signature).
+template <int D, int NS, bool COMP>
+__device__ __forceinline__ void attn_body(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                                          const CUtensorMap& tmKb, const CUtensorMap& tmVb, const AttnParams& p) {
     using SM = AttnSmem<D, NS>;
     constexpr int NCH = D / 64;                 // 128-byte column chunks per row
     constexpr uint32_t kIdescS = idesc_bf16_f32(128, 64, 0, 0);
@@ -209,12 +218,16 @@ __global__ void __launch_bounds__(192, 2)
     tc_fence_after();
     const uint32_t tmem = ctl[0];
     const int n = static_cast<int>(ctl[2]);
+    // with compensation, the block-mean steps follow the union (none for a tile whose
+    // two slots both lie past the sample)
+    const bool any_slot = (qb[0] >= 0 && qb[0] < nB) || (qb[1] >= 0 && qb[1] < nB);
+    const int n_all = COMP && any_slot ? n + (nB + 63) / 64 : n;
     const uint64_t lim = p.wait_limit;
     int issued_k = 0, issued_v = 0;  // K / V blocks whose loads the producer has issued
 
     if (warp == 4) {
         // ------------------------------------------------------------ TMA producer
-        if (lane == 0 && n > 0) {
+        if (lane == 0 && n_all > 0) {
             tma_prefetch_desc(&tmQ);
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
@@ -227,36 +240,38 @@ __global__ void __launch_bounds__(192, 2)
                     tma_load_3d(sQ + c * (128 * 128) + h2 * (64 * 128), &tmQ, bar_q, c * 64, qb[h2] * 64, bh);
             // K runs one block ahead of V: K(j) is released as soon as S(j) is done,
             // V(j) only after PV(j).  Issue order K0, K1, V0, K2, V1, ...
-            for (int j = 0; j <= n; ++j) {
-                if (j < n) {
+            for (int j = 0; j <= n_all; ++j) {
+                if (j < n_all) {
                     const int st = j % NS;
                     if (j >= NS && !wait_bounded(bar_ke(st), ((j / NS) - 1) & 1, abort_flag, lim)) break;
-                    const int J = ulist[j];
+                    const bool mean_step = COMP && j >= n;
+                    const int row = mean_step ? (j - n) * 64 : ulist[j] * 64;
                     mbar_arrive_expect_tx(bar_kf(st), SM::kKVBytes);
                     for (int c = 0; c < NCH; ++c)
-                        tma_load_3d(sK + st * SM::kKVBytes + c * (64 * 128), &tmK, bar_kf(st), c * 64,
-                                    J * 64, bh);
+                        tma_load_3d(sK + st * SM::kKVBytes + c * (64 * 128), mean_step ? &tmKb : &tmK, bar_kf(st),
+                                    c * 64, row, bh);
                     issued_k = j + 1;
                 }
                 if (j >= 1) {
                     const int jv = j - 1, st = jv % NS;
                     if (jv >= NS && !wait_bounded(bar_ve(st), ((jv / NS) - 1) & 1, abort_flag, lim)) break;
-                    const int J = ulist[jv];
+                    const bool mean_step = COMP && jv >= n;
+                    const int row = mean_step ? (jv - n) * 64 : ulist[jv] * 64;
                     mbar_arrive_expect_tx(bar_vf(st), SM::kKVBytes);
                     for (int c = 0; c < NCH; ++c)
-                        tma_load_3d(sV + st * SM::kKVBytes + c * (64 * 128), &tmV, bar_vf(st), c * 64,
-                                    J * 64, bh);
+                        tma_load_3d(sV + st * SM::kKVBytes + c * (64 * 128), mean_step ? &tmVb : &tmV, bar_vf(st),
+                                    c * 64, row, bh);
                     issued_v = jv + 1;
                 }
             }
         }
     } else if (warp == 5) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0 && n > 0) {
+        if (lane == 0 && n_all > 0) {
             bool ok = wait_bounded(bar_q, 0, abort_flag, lim);
             tc_fence_after();
-            for (int j = 0; ok && j <= n; ++j) {
-                if (j < n) {
+            for (int j = 0; ok && j <= n_all; ++j) {
+                if (j < n_all) {
                     const int st = j % NS;
                     if (!wait_bounded(bar_kf(st), (j / NS) & 1, abort_flag, lim)) { ok = false; break; }
                     tc_fence_after();
@@ -298,11 +313,34 @@ __global__ void __launch_bounds__(192, 2)
         const float sc = p.scale_log2;
         float m = -INFINITY, l = 0.f;
         bool ok = true;
-        for (int j = 0; j < n; ++j) {
-            const int J = ulist[j];
-            const bool kept = (bmh[J >> 5] >> (J & 31)) & 1u;  // uniform over the warp
-            int ncol = kept ? L - J * 64 : 0;
-            ncol = ncol > 64 ? 64 : ncol;
+        for (int j = 0; j < n_all; ++j) {
+            bool kept;                 // this half has weight in the step (uniform over the warp)
+            int ncol;
+            uint64_t cmask = ~0ull;    // mean steps: the columns that carry weight for this half
+            float off_full = 0.f, off_last = 0.f;
+            int last_col = -1;
+            if (COMP && j >= n) {
+                // columns 0..63 stand for blocks J = 64 pb + c: the half's dropped blocks
+                // of the sample, each with logit offset log2(c_J) (folded in as / sc)
+                const int pb = j - n;
+                const uint64_t kb = (uint64_t)bmh[2 * pb] | ((uint64_t)bmh[2 * pb + 1] << 32);
+                const int nv = nB - 64 * pb;
+                const uint64_t inb = nv >= 64 ? ~0ull : ((1ull << nv) - 1ull);
+                const bool half_ok = qb[half] >= 0 && qb[half] < nB;
+                cmask = half_ok ? (~kb & inb) : 0ull;
+                kept = cmask != 0ull;
+                ncol = 64;
+                off_full = 6.0f / sc;  // log2(64)
+                if (nv <= 64) {
+                    last_col = nv - 1;
+                    off_last = log2f((float)(L - 64 * (nB - 1))) / sc;
+                }
+            } else {
+                const int J = ulist[j];
+                kept = (bmh[J >> 5] >> (J & 31)) & 1u;
+                ncol = kept ? L - J * 64 : 0;
+                ncol = ncol > 64 ? 64 : ncol;
+            }
             if (!warp_wait_bounded(bar_sf(j & 1), (j >> 1) & 1, abort_flag, lim)) { ok = false; break; }
             tc_fence_after();
             const uint32_t sbuf = tl + (j & 1) * 64;
@@ -332,6 +370,13 @@ __global__ void __launch_bounds__(192, 2)
             if (ncol < 64) {  // ragged tail block of the sample
 #pragma unroll
                 for (int i = 0; i < 64; ++i) x[i] = i < ncol ? x[i] : -INFINITY;
+            }
+            if constexpr (COMP) {
+                if (j >= n) {
+#pragma unroll
+                    for (int i = 0; i < 64; ++i)
+                        x[i] = ((cmask >> i) & 1ull) ? x[i] + (i == last_col ? off_last : off_full) : -INFINITY;
+                }
             }
             float mx0 = x[0], mx1 = x[1];
 #pragma unroll
@@ -392,7 +437,7 @@ __global__ void __launch_bounds__(192, 2)
         }
 
         // ------------------------------------------------------------ epilogue
-        if (ok && n > 0) ok = warp_wait_bounded(bar_pv((n - 1) & 1), ((n - 1) >> 1) & 1, abort_flag, lim);
+        if (ok && n_all > 0) ok = warp_wait_bounded(bar_pv((n_all - 1) & 1), ((n_all - 1) >> 1) & 1, abort_flag, lim);
         tc_fence_after();
         const bool in_range = qb[half] >= 0 && qb[half] < nQ;
         const bool valid = tok < L && l > 0.f;
@@ -402,7 +447,7 @@ __global__ void __launch_bounds__(192, 2)
 #pragma unroll
             for (int ch = 0; ch < D / 32; ++ch) {
                 uint32_t o[32];
-                if (n > 0) {
+                if (n_all > 0) {
                     tmem_ld32(tl + 128 + ch * 32, o);
                     tmem_wait_ld();
                 }
@@ -410,8 +455,8 @@ __global__ void __launch_bounds__(192, 2)
                     uint32_t pk[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        const float o0 = (n > 0 && valid) ? __uint_as_float(o[2 * i]) * inv_l : 0.f;
-                        const float o1 = (n > 0 && valid) ? __uint_as_float(o[2 * i + 1]) * inv_l : 0.f;
+                        const float o0 = (n_all > 0 && valid) ? __uint_as_float(o[2 * i]) * inv_l : 0.f;
+                        const float o1 = (n_all > 0 && valid) ? __uint_as_float(o[2 * i + 1]) * inv_l : 0.f;
                         __nv_bfloat162 h2 = __floats2bfloat162_rn(o0, o1);
                         pk[i] = *reinterpret_cast<uint32_t*>(&h2);
                     }
@@ -433,7 +478,7 @@ __global__ void __launch_bounds__(192, 2)
     if (*abort_flag) {
         // An aborted CTA still lets its own TMA copies land and its MMAs finish
         // before it frees TMEM and exits.
-        if (warp == 4 && lane == 0 && n > 0) {
+        if (warp == 4 && lane == 0 && n_all > 0) {
             wait_drain(bar_q, 0);
             for (int j = issued_k > NS ? issued_k - NS : 0; j < issued_k; ++j)
                 wait_drain(bar_kf(j % NS), (j / NS) & 1);
@@ -450,6 +495,22 @@ __global__ void __launch_bounds__(192, 2)
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
+}
+
+template <int D, int NS>
+__global__ void __launch_bounds__(192, 2)
+    attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+    attn_body<D, NS, false>(tmQ, tmK, tmV, tmK, tmV, p);
+}
+
+// With compensation of the dropped blocks: kbar / vbar maps over [BH][nBpad][D].
+template <int D, int NS>
+__global__ void __launch_bounds__(192, 2)
+    attn_comp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKb,
+                     const __grid_constant__ CUtensorMap tmVb, const AttnParams p) {
+    attn_body<D, NS, true>(tmQ, tmK, tmV, tmKb, tmVb, p);
 }
 
 }  // namespace sba

@@ -17,6 +17,7 @@
 #include "score_lse.cuh"
 #include "pair.cuh"
 #include "producer.cuh"
+#include "compensation.cuh"
 
 namespace {
 
@@ -24,6 +25,7 @@ constexpr uint64_t kDefaultWaitLimit = 1ull << 32;  // clock cycles, ~2 s at 2 G
 uint64_t g_wait_limit = kDefaultWaitLimit;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t align_up_256(size_t x) { return (x + 255) & ~size_t(255); }
 
 sba_status check_shape(int B, int H, int Npad, int D, int block) {
     if (B <= 0 || H <= 0 || Npad <= 0) return SBA_ERR_INVALID_ARG;
@@ -70,19 +72,27 @@ bool make_map(CUtensorMap* map, const void* base, int BH, int Npad, int D, int b
     return r == CUDA_SUCCESS;
 }
 
-template <int D, int NS>
+// kbar / vbar (COMP only): bf16 [BH][nBpad][D] block means for the compensation steps.
+template <int D, int NS, bool COMP = false>
 sba_status launch_attention(const void* q, const void* k, const void* v, void* o, float* lse,
                             int B, int H, int Npad, const int32_t* valid_len,
                             const int32_t* kv_idx, const int32_t* kv_cnt, int kmax, int dense,
-                            const int32_t* pair_order, float softmax_scale, cudaStream_t stream) {
+                            const int32_t* pair_order, float softmax_scale, cudaStream_t stream,
+                            const void* kbar = nullptr, const void* vbar = nullptr, int nBpad = 0) {
     using SM = sba::AttnSmem<D, NS>;
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, tkb, tvb;
     const int BH = B * H;
     if (!make_map(&tq, q, BH, Npad, D, 64) || !make_map(&tk, k, BH, Npad, D, 64) ||
         !make_map(&tv, v, BH, Npad, D, 64))
         return SBA_ERR_CUDA;
-    if (cudaFuncSetAttribute(sba::attn_kernel<D, NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             SM::kAlloc) != cudaSuccess)
+    if (COMP) {
+        if (!make_map(&tkb, kbar, BH, nBpad, D, 64) || !make_map(&tvb, vbar, BH, nBpad, D, 64)) return SBA_ERR_CUDA;
+    } else {
+        tkb = tk;
+        tvb = tv;
+    }
+    if (cudaFuncSetAttribute(COMP ? (const void*)sba::attn_comp_kernel<D, NS> : (const void*)sba::attn_kernel<D, NS>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kAlloc) != cudaSuccess)
         return SBA_ERR_CUDA;
     sba::AttnParams p;
     p.o = static_cast<__nv_bfloat16*>(o);
@@ -99,7 +109,10 @@ sba_status launch_attention(const void* q, const void* k, const void* v, void* o
     p.scale_log2 = scale * 1.4426950408889634f;
     p.wait_limit = g_wait_limit;
     dim3 grid((Npad / 64 + 1) / 2, H, B);
-    sba::attn_kernel<D, NS><<<grid, 192, SM::kAlloc, stream>>>(tq, tk, tv, p);
+    if (COMP)
+        sba::attn_comp_kernel<D, NS><<<grid, 192, SM::kAlloc, stream>>>(tq, tk, tv, tkb, tvb, p);
+    else
+        sba::attn_kernel<D, NS><<<grid, 192, SM::kAlloc, stream>>>(tq, tk, tv, p);
     return cudaGetLastError() == cudaSuccess ? SBA_OK : SBA_ERR_CUDA;
 }
 
@@ -314,7 +327,8 @@ static sba_status attention_common(const void* q, const void* k, const void* v, 
                                    int B, int H, int Npad, int D, const int32_t* valid_len,
                                    int block, const int32_t* kv_idx, const int32_t* kv_cnt,
                                    int kmax, int dense, const int32_t* pair_order,
-                                   float softmax_scale, void* stream) {
+                                   float softmax_scale, void* stream, void* comp_ws = nullptr,
+                                   size_t comp_ws_bytes = 0) {
     sba_status st = check_shape(B, H, Npad, D, block);
     if (st != SBA_OK) return st;
     if (!q || !k || !v || !o) return SBA_ERR_INVALID_ARG;
@@ -328,6 +342,36 @@ static sba_status attention_common(const void* q, const void* k, const void* v, 
         (pair_order && (reinterpret_cast<uintptr_t>(pair_order) & 3u)))
         return SBA_ERR_ALIGNMENT;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (comp_ws) {
+        // compensated: the bf16 block means of K and V, then the attention with the
+        // mean steps after the kept blocks
+        if (dense) return SBA_ERR_INVALID_ARG;
+        if (!aligned16(comp_ws)) return SBA_ERR_ALIGNMENT;
+        const int nBpad = (Npad / 64 + 63) / 64 * 64;
+        const size_t half = align_up_256((size_t)B * H * nBpad * D * 2);
+        if (comp_ws_bytes < 2 * half) return SBA_ERR_INVALID_ARG;
+        char* kbar = static_cast<char*>(comp_ws);
+        char* vbar = kbar + half;
+        const long long groups = (long long)B * H * nBpad;
+        const int gpc = 256 / (D / 8);
+        const unsigned mgrid = (unsigned)((groups + gpc - 1) / gpc);
+        if (D == 128) {
+            sba::block_mean_bf16_kernel<128><<<mgrid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(k), valid_len, H,
+                                                                    Npad, nBpad, reinterpret_cast<__nv_bfloat16*>(kbar),
+                                                                    groups);
+            sba::block_mean_bf16_kernel<128><<<mgrid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(v), valid_len, H,
+                                                                    Npad, nBpad, reinterpret_cast<__nv_bfloat16*>(vbar),
+                                                                    groups);
+            return launch_attention<128, 2, true>(q, k, v, o, lse, B, H, Npad, valid_len, kv_idx, kv_cnt, kmax, 0,
+                                                  pair_order, softmax_scale, s, kbar, vbar, nBpad);
+        }
+        sba::block_mean_bf16_kernel<64><<<mgrid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(k), valid_len, H, Npad,
+                                                               nBpad, reinterpret_cast<__nv_bfloat16*>(kbar), groups);
+        sba::block_mean_bf16_kernel<64><<<mgrid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(v), valid_len, H, Npad,
+                                                               nBpad, reinterpret_cast<__nv_bfloat16*>(vbar), groups);
+        return launch_attention<64, 4, true>(q, k, v, o, lse, B, H, Npad, valid_len, kv_idx, kv_cnt, kmax, 0,
+                                             pair_order, softmax_scale, s, kbar, vbar, nBpad);
+    }
     if (D == 128)
         return launch_attention<128, 2>(q, k, v, o, lse, B, H, Npad, valid_len, kv_idx, kv_cnt, kmax,
                                         dense, pair_order, softmax_scale, s);
@@ -357,6 +401,22 @@ sba_status sba_dense_attention(const void* q, const void* k, const void* v, void
                                float softmax_scale, void* stream) {
     return attention_common(q, k, v, o, lse, B, H, Npad, D, valid_len, 64, nullptr, nullptr, 0, 1,
                             nullptr, softmax_scale, stream);
+}
+
+size_t sba_compensation_workspace_size(int B, int H, int Npad, int D, int block) {
+    if (check_shape(B, H, Npad, D, block) != SBA_OK) return 0;
+    const int nBpad = (Npad / 64 + 63) / 64 * 64;
+    return 2 * align_up_256((size_t)B * H * nBpad * D * 2);
+}
+
+sba_status sba_attention_compensated(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                                     int H, int Npad, int D, const int32_t* valid_len, int block,
+                                     const int32_t* kv_idx, const int32_t* kv_cnt, int kmax,
+                                     const int32_t* pair_order, float softmax_scale, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+    if (!workspace) return SBA_ERR_INVALID_ARG;
+    return attention_common(q, k, v, o, lse, B, H, Npad, D, valid_len, block, kv_idx, kv_cnt, kmax, 0,
+                            pair_order, softmax_scale, stream, workspace, workspace_bytes);
 }
 
 sba_status sba_get_device_status(void* stream) {

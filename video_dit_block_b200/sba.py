@@ -55,6 +55,11 @@ def lib() -> ctypes.CDLL:
         L.sba_qk_norm_rope_pool.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, i32, i32, f64, f32, vp, vp, vp]
         L.sba_pool_select_means.restype = i32
         L.sba_pool_select_means.argtypes = [vp, vp, i32, i32, i32, i32, vp, i32, f64, i32, vp, vp, vp, sz, vp]
+        L.sba_compensation_workspace_size.restype = sz
+        L.sba_compensation_workspace_size.argtypes = [i32, i32, i32, i32, i32]
+        L.sba_attention_compensated.restype = i32
+        L.sba_attention_compensated.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, i32, vp, vp, i32, vp,
+                                                f32, vp, sz, vp]
         L.sba_block_means.restype = i32
         L.sba_block_means.argtypes = [vp, i32, i32, i32, i32, vp, i32, vp, vp]
         L.sba_attention.restype = i32
@@ -283,6 +288,26 @@ def attention_paired(q, k, v, kv_idx, kv_cnt, pair_order, valid_len=None, softma
                                       _ptr(_valid_len(valid_len, q.device)), block, _ptr(kv_idx),
                                       _ptr(kv_cnt), kv_idx.shape[-1], _ptr(pair_order), float(softmax_scale),
                                       _stream(stream)), "sba_attention_paired")
+    return out, lse
+
+
+def attention_compensated(q, k, v, kv_idx, kv_cnt, valid_len=None, pair_order=None, softmax_scale: float = 0.0,
+                          out=None, lse=None, want_lse: bool = True, workspace=None, block: int = BLOCK,
+                          stream=None):
+    """Block-sparse attention with each dropped block compensated by its mean key and
+    value (see include/sba.h).  Returns (o bf16, lse fp32 or None)."""
+    B, H, Npad, D = _qkv(q, k, v)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H, Npad), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(int(lib().sba_compensation_workspace_size(B, H, Npad, D, block)), dtype=torch.uint8,
+                                device=q.device)
+    _check(lib().sba_attention_compensated(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Npad, D,
+                                           _ptr(_valid_len(valid_len, q.device)), block, _ptr(kv_idx), _ptr(kv_cnt),
+                                           kv_idx.shape[-1], _ptr(pair_order), float(softmax_scale), _ptr(workspace),
+                                           workspace.numel(), _stream(stream)), "sba_attention_compensated")
     return out, lse
 
 
