@@ -14,6 +14,8 @@ blocks; the default is the block-mean router with no rounding.  `--producer` tre
 the workload's Q and K as the pre-norm projections: each step first applies QK
 RMSNorm + 3D RoPE with the block pooling fused (sba_qk_norm_rope_pool), then routes
 from those means (sba_pool_select_means) and attends over the normalised Q and K.
+`--compensate` attends with compensation of the dropped blocks
+(sba_attention_compensated); the metric still counts kept-block FLOPs only.
 
 Metric: effective TFLOP/s on the kept blocks, counted as
 4 * D * sum_{b,h,I} c_I * sum_{J kept} c_J (c = valid tokens of a block), divided by
@@ -56,14 +58,15 @@ def parse():
     ap.add_argument("--router", default="mean", choices=["mean", "lse"])
     ap.add_argument("--budget", type=int, default=1)
     ap.add_argument("--producer", action="store_true")
+    ap.add_argument("--compensate", action="store_true")
     return ap.parse_args()
 
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one attention launch,
 # from the ncu captures summarised in profiles/attn_kernel_*.md, and the hash
 # of the kernel sources it was taken with.  Reported only while the sources match.
-ATTN_TRAFFIC = {"480p_dense": (632697856 + 189443072, "f94215845bc4f30c"),
-                "720p": (3019749376 + 805242368, "f94215845bc4f30c")}
+ATTN_TRAFFIC = {"480p_dense": (633502720 + 188913920, "f6f66ea55d2d8d99"),
+                "720p": (3049651000 + 806195200, "f6f66ea55d2d8d99")}
 KERNEL_SOURCES = ("video_dit_block_b200/csrc/attention.cuh", "video_dit_block_b200/csrc/ptx.cuh",
                   "video_dit_block_b200/csrc/common.cuh")
 
@@ -165,7 +168,7 @@ def whole_job_value(kept_flops_per_rank, ms_per_step, world):
     return world * kept_flops_per_rank / (ms_per_step * 1e-3) / 1e12
 
 
-def oracle_sample(w, target_s=10.0, seed=0, router="mean", budget=1, producer=False):
+def oracle_sample(w, target_s=10.0, seed=0, router="mean", budget=1, producer=False, compensate=False):
     """Time the fp64 oracle, as it stands, on a bounded sample of the workload: the
     full routing of head (b=0, h=0) and the attention of a seeded subset of that head's
     query blocks, sized to about `target_s` seconds.
@@ -197,7 +200,8 @@ def oracle_sample(w, target_s=10.0, seed=0, router="mean", budget=1, producer=Fa
     n, t_attn = 1, 0.0
     while True:
         t0 = time.perf_counter()
-        oracle.attention(q1, k1, v1, idx, cnt, vl1, qblocks=order[:n])
+        (oracle.attention_compensated if compensate else oracle.attention)(q1, k1, v1, idx, cnt, vl1,
+                                                                           qblocks=order[:n])
         t_attn = time.perf_counter() - t0
         if t_attn >= target_s / 2 or n >= nB0:
             break
@@ -231,6 +235,8 @@ def router_config(args):
         "router": "sub-block log-sum-exp (4 x 16 tokens)", "budget": args.budget}
     if args.producer:
         c["producer"] = "QK RMSNorm + 3D RoPE (rope_dim 3D/4, base 1e4, eps 1e-6) with fused block pooling"
+    if args.compensate:
+        c["compensation"] = "dropped blocks by their bf16 mean key and value, weighted by token count"
     return c
 
 
@@ -244,7 +250,7 @@ def run_reference(args):
     target = max(2.0, 60.0 / max(1, args.steps + args.warmup))
     for i in range(args.warmup + args.steps):
         s = oracle_sample(w, target_s=target, seed=i, router=args.router, budget=args.budget,
-                          producer=args.producer)
+                          producer=args.producer, compensate=args.compensate)
         if i >= args.warmup:
             per.append(s)
     value = statistics.mean(s["value"] for s in per)
@@ -327,8 +333,16 @@ def run_ours(args):
         sba.pair_query_blocks(kv_idx, kv_cnt, vll, pair_order=pair_order, workspace=pws, stream=stream)
         return qq, kk
 
+    if args.compensate:
+        cws = torch.empty(int(sba.lib().sba_compensation_workspace_size(B, H, Npad, D, 64)), dtype=torch.uint8,
+                          device=dev)
+
     def attend(qq=q, kk=k, vv=v, vll=vl, out=o):
-        sba.attention_paired(qq, kk, vv, kv_idx, kv_cnt, pair_order, vll, out=out, lse=lse, stream=stream)
+        if args.compensate:
+            sba.attention_compensated(qq, kk, vv, kv_idx, kv_cnt, vll, pair_order=pair_order, out=out, lse=lse,
+                                      workspace=cws, stream=stream)
+        else:
+            sba.attention_paired(qq, kk, vv, kv_idx, kv_cnt, pair_order, vll, out=out, lse=lse, stream=stream)
 
     def step(qq=q, kk=k, vv=v):
         qa, ka = route(qq, kk)
@@ -433,7 +447,7 @@ def run_ours(args):
         return
     peaks, src = load_peaks()
     tr = ATTN_TRAFFIC.get(w.name)
-    traffic = tr[0] if tr is not None and tr[1] == kernel_source_hash() else None
+    traffic = tr[0] if tr is not None and tr[1] == kernel_source_hash() and not args.compensate else None
     peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
     achieved = f_step / (attn_ms * 1e-3) / 1e12
     line = {
@@ -446,21 +460,26 @@ def run_ours(args):
             "kmax": kmax, **router_config(args)}),
         "pct_of_spec_bf16_peak": 100.0 * value / world / SPEC_BF16_TFLOPS,
         "attn_ms": attn_ms, "select_ms": sel_ms, "kept_tflop_per_step": f_step / 1e12,
-        "roofline": {"bound": "tensor", "kernel": "attn_kernel<128,2>" if D == 128 else "attn_kernel<64,4>",
+        "roofline": {"bound": "tensor",
+                     "kernel": ("attn_comp_kernel" if args.compensate else "attn_kernel")
+                     + ("<128,2>" if D == 128 else "<64,4>"),
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_source": f"{src} bf16_tflops_sustained (kernel timed inside a seconds-long loop)",
                      "traffic": traffic},
         # per step: routing = 2 pooling + key-norm maximum + screen (only when blocks are
         # dropped) + top-k; pairing = bitmaps + 4 x (propose, resolve) + emit; 1 attention
         # (--producer: 2 producer launches and 2 splits of the given means replace pooling)
-        "gpu_launches": (4 + (1 if w.sparsity > 0 else 0) + (2 if args.producer else 0) + 10 + 1) * K,
+        # (--compensate: 2 block-mean launches before the attention)
+        "gpu_launches": (4 + (1 if w.sparsity > 0 else 0) + (2 if args.producer else 0) + 10 + 1
+                         + (2 if args.compensate else 0)) * K,
         "clocks": clk,
     }
     if e2e is not None:
         line["e2e"] = e2e
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_from(oracle_sample(w, target_s=15.0, router=args.router,
-                                                               budget=args.budget, producer=args.producer))
+                                                               budget=args.budget, producer=args.producer,
+                                                               compensate=args.compensate))
     print(json.dumps(line), flush=True)
     if dist is not None:
         dist.destroy_process_group()
