@@ -49,7 +49,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--config", default="480p_dense")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -100,21 +100,25 @@ def kept_flops(kv_idx, kv_cnt, valid_len, D, block=64):
 
 
 class ClockSampler:
-    """nvidia-smi every 200 ms while the timed region runs."""
+    """nvidia-smi every 100 ms, started before the warm-up so that it is sampling when
+    the timed region begins; each line is stamped on arrival, and only the samples
+    that arrive within the timed window (widened by one interval) are summarised."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    INTERVAL_MS = 100
 
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
         self.lines = []
+        self.window = None
 
     def start(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", str(self.INTERVAL_MS)],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
@@ -123,7 +127,11 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.monotonic(), line.strip()))
+
+    def mark(self, t0, t1):
+        """The timed region, in time.monotonic() seconds."""
+        self.window = (t0, t1)
 
     def stop(self):
         if self.proc is None:
@@ -134,9 +142,12 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.thread.join(timeout=5)
+        pad = self.INTERVAL_MS * 1e-3
+        lines = [ln for (t, ln) in self.lines
+                 if self.window is None or self.window[0] - pad <= t <= self.window[1] + pad]
         sm, smax, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for ln in lines:
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 9:
                 continue
@@ -352,6 +363,8 @@ def run_ours(args):
         if dist is not None:
             dist.barrier()
 
+    clocks = ClockSampler(local)
+    clocks.start()  # sampling already when the timed region begins
     for _ in range(args.warmup):
         step()
     status = sba.device_status(stream)
@@ -363,11 +376,9 @@ def run_ours(args):
     K = args.steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
            torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    clocks = ClockSampler(local)
     barrier()
     torch.cuda.synchronize(dev)
-    clocks.start()
-    time.sleep(0.3)
+    t_begin = time.monotonic()
     for i in range(K):
         ev[i][0].record(stream)
         qa, ka = route()
@@ -375,6 +386,7 @@ def run_ours(args):
         attend(qa, ka)
         ev[i][2].record(stream)
     torch.cuda.synchronize(dev)
+    clocks.mark(t_begin, time.monotonic())
     clk = clocks.stop()
     barrier()
     total_ms = ev[0][0].elapsed_time(ev[-1][2])
