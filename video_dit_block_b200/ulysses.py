@@ -1,0 +1,78 @@
+"""Head sharding with a Ulysses all-to-all around the block-sparse path.
+
+A video DiT run with sequence parallelism holds, on each of P ranks, a contiguous
+1/P of the token sequence for all heads.  Attention needs the whole sequence, so
+the page "MiniMax-H3 on 8xH200 benchmark" runs it under SP/Ulysses-8: one
+all-to-all turns [B, H, N/P, D] per rank into [B, H/P, N, D] (every token, a
+1/P share of the heads), attention runs per head unchanged -- routing and the
+kernels see whole sequences -- and a second all-to-all turns the output back.
+
+The exchange is torch.distributed's all_to_all_single (NCCL between GPUs, gloo on
+CPU); the tensors travel as int32 pairs of bf16 bit patterns, so the exchange is
+exact and works on either backend.  Token range r * N/P .. (r+1) * N/P lives on
+rank r; heads p * H/P .. (p+1) * H/P are attended on rank p.
+"""
+from __future__ import annotations
+
+import torch
+import torch.distributed as dist
+
+
+def _as_words(x):
+    """A [.., D] bf16 (or int16) tensor viewed as int32 pairs, D even."""
+    return x.contiguous().view(torch.int32)
+
+
+def seq_to_heads(x, group=None):
+    """[B, H, N_local, D] on every rank -> [B, H/P, P * N_local, D] (this rank's heads,
+    the whole sequence).  H must be a multiple of P."""
+    P = dist.get_world_size(group)
+    B, H, Nl, D = x.shape
+    if H % P != 0:
+        raise ValueError(f"{H} heads do not split over {P} ranks")
+    w = _as_words(x)                                   # [B, H, Nl, D/2]
+    send = w.reshape(B, P, H // P, Nl, D // 2).transpose(0, 1).contiguous()  # [P dst, B, H/P, Nl, D/2]
+    recv = torch.empty_like(send)                      # [P src, B, H/P, Nl, D/2]
+    dist.all_to_all_single(recv, send, group=group)
+    out = recv.permute(1, 2, 0, 3, 4).reshape(B, H // P, P * Nl, D // 2)
+    return out.contiguous().view(x.dtype)
+
+
+def heads_to_seq(y, group=None):
+    """The inverse: [B, H/P, N, D] on every rank -> [B, H, N/P, D]."""
+    P = dist.get_world_size(group)
+    B, Hl, N, D = y.shape
+    if N % P != 0:
+        raise ValueError(f"{N} tokens do not split over {P} ranks")
+    Nl = N // P
+    w = _as_words(y)
+    send = w.reshape(B, Hl, P, Nl, D // 2).permute(2, 0, 1, 3, 4).contiguous()  # [P dst, B, Hl, Nl, D/2]
+    recv = torch.empty_like(send)                      # [P src (head group), B, Hl, Nl, D/2]
+    dist.all_to_all_single(recv, send, group=group)
+    out = recv.transpose(0, 1).reshape(B, P * Hl, Nl, D // 2)
+    return out.contiguous().view(y.dtype)
+
+
+def lse_heads_to_seq(lse, group=None):
+    """[B, H/P, N] fp32 -> [B, H, N/P]."""
+    P = dist.get_world_size(group)
+    B, Hl, N = lse.shape
+    Nl = N // P
+    send = lse.contiguous().view(torch.int32).reshape(B, Hl, P, Nl).permute(2, 0, 1, 3).contiguous()
+    recv = torch.empty_like(send)
+    dist.all_to_all_single(recv, send, group=group)
+    return recv.transpose(0, 1).reshape(B, P * Hl, Nl).contiguous().view(lse.dtype)
+
+
+def ulysses_attention(q, k, v, valid_len=None, sparsity: float = 0.75, group=None, attention=None, **kwargs):
+    """Sequence-sharded block-sparse attention.  q, k, v: this rank's [B, H, N/P, D]
+    token range (N the padded length, a multiple of 64 P); valid_len: the samples'
+    full lengths.  `attention(q, k, v, valid_len, sparsity, **kwargs) -> (o, lse, ...)`
+    runs on the gathered [B, H/P, N, D] tensors; by default the library's
+    sparse_attention.  Returns this rank's (o [B, H, N/P, D], lse [B, H, N/P])."""
+    if attention is None:
+        from .sba import sparse_attention as attention
+    qh, kh, vh = (seq_to_heads(t, group) for t in (q, k, v))
+    res = attention(qh, kh, vh, valid_len, sparsity, **kwargs)
+    o_h, lse_h = res[0], res[1]
+    return heads_to_seq(o_h, group), lse_heads_to_seq(lse_h, group)
