@@ -249,6 +249,23 @@ sba_status sba_get_device_status(void* stream);
  * default.  Meant for tests of the timeout path. */
 void sba_set_wait_limit(uint64_t cycles);
 
+/* Which attention kernel sba_attention, sba_attention_paired and sba_dense_attention
+ * run for D = 128 (the compensated path and D = 64 always use the first):
+ *   SBA_ATTN_KERNEL_QUERY_PAIRS  one SM per tile of two query blocks, walking the union
+ *                                of their kept lists (64 keys per step);
+ *   SBA_ATTN_KERNEL_CTA_PAIR     a 2-SM cluster per tile of four adjacent query blocks
+ *                                (tcgen05 MMAs of M = 256 across the pair, 128 keys per
+ *                                step), walking the union of their four lists;
+ *                                pair_order is not used;
+ *   SBA_ATTN_KERNEL_AUTO         (default) the query pairs, the faster of the two on
+ *                                every workload measured on B200.
+ * Outputs agree up to floating-point accumulation order.  Process-wide; returns
+ * SBA_ERR_INVALID_ARG for another value. */
+#define SBA_ATTN_KERNEL_AUTO 0
+#define SBA_ATTN_KERNEL_QUERY_PAIRS 1
+#define SBA_ATTN_KERNEL_CTA_PAIR 2
+sba_status sba_set_attention_kernel(int which);
+
 /* Routing for callers that cannot allocate device memory.
  *
  * No counterpart on the pages: this is a library convenience.  Some callers may

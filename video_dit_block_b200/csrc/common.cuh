@@ -16,12 +16,28 @@ __device__ __forceinline__ void raise_device_error(int code) {
     atomicCAS(&g_device_error, 0, code);
 }
 
+// Limits below this are for tests of the timeout path: those waits only poll (a
+// try_wait may suspend the thread for tens of microseconds, longer than such a limit).
+constexpr uint64_t kPollOnlyLimit = 1ull << 20;
+
 // Wait for phase `parity` of mbarrier `bar`, giving up when another thread of
 // the CTA has set *abort, or after `limit` clock cycles (then the error word is
 // set and *abort raised so every role of the CTA unwinds).  Returns true when
 // the phase completed.
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
                                              volatile uint32_t* abort, uint64_t limit) {
+    if (limit < kPollOnlyLimit) {
+        const long long t0 = clock64();
+        while (!mbar_test_wait(bar, parity)) {
+            if (*abort) return false;
+            if ((uint64_t)(clock64() - t0) > limit) {
+                raise_device_error(kErrTimeout);
+                *abort = 1u;
+                return false;
+            }
+        }
+        return true;
+    }
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {

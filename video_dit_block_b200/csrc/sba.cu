@@ -11,6 +11,7 @@
 
 #include "../../include/sba.h"
 #include "attention.cuh"
+#include "attention2.cuh"
 #include "common.cuh"
 #include "select.cuh"
 #include "score_mma.cuh"
@@ -23,6 +24,7 @@ namespace {
 
 constexpr uint64_t kDefaultWaitLimit = 1ull << 32;  // clock cycles, ~2 s at 2 GHz
 uint64_t g_wait_limit = kDefaultWaitLimit;
+int g_attn_kernel = SBA_ATTN_KERNEL_AUTO;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 size_t align_up_256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -113,6 +115,41 @@ sba_status launch_attention(const void* q, const void* k, const void* v, void* o
         sba::attn_comp_kernel<D, NS><<<grid, 192, SM::kAlloc, stream>>>(tq, tk, tv, tkb, tvb, p);
     else
         sba::attn_kernel<D, NS><<<grid, 192, SM::kAlloc, stream>>>(tq, tk, tv, p);
+    return cudaGetLastError() == cudaSuccess ? SBA_OK : SBA_ERR_CUDA;
+}
+
+// The CTA-pair kernel (D = 128): four query blocks per 2-SM cluster, two key blocks
+// per step.
+template <int NS>
+sba_status launch_attention_pair(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                                 int Npad, const int32_t* valid_len, const int32_t* kv_idx, const int32_t* kv_cnt,
+                                 int kmax, int dense, float softmax_scale, cudaStream_t stream) {
+    using SM = sba::Attn2Smem<NS>;
+    CUtensorMap tq, tk, tv;
+    const int BH = B * H;
+    if (!make_map(&tq, q, BH, Npad, 128, 64) || !make_map(&tk, k, BH, Npad, 128, 64) ||
+        !make_map(&tv, v, BH, Npad, 128, 64))
+        return SBA_ERR_CUDA;
+    if (cudaFuncSetAttribute(sba::attn_pair_kernel<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kAlloc) !=
+        cudaSuccess)
+        return SBA_ERR_CUDA;
+    sba::AttnParams p;
+    p.o = static_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.valid_len = valid_len;
+    p.kv_idx = kv_idx;
+    p.kv_cnt = kv_cnt;
+    p.pair_order = nullptr;
+    p.H = H;
+    p.Npad = Npad;
+    p.kmax = kmax;
+    p.dense = dense;
+    const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(128.0f);
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.wait_limit = g_wait_limit;
+    const int nQ = Npad / 64;
+    dim3 grid(2 * ((nQ + 3) / 4), H, B);
+    sba::attn_pair_kernel<NS><<<grid, 320, SM::kAlloc, stream>>>(tq, tk, tv, p);
     return cudaGetLastError() == cudaSuccess ? SBA_OK : SBA_ERR_CUDA;
 }
 
@@ -372,6 +409,11 @@ static sba_status attention_common(const void* q, const void* k, const void* v, 
         return launch_attention<64, 4, true>(q, k, v, o, lse, B, H, Npad, valid_len, kv_idx, kv_cnt, kmax, 0,
                                              pair_order, softmax_scale, s, kbar, vbar, nBpad);
     }
+    // the CTA-pair kernel only when chosen: on B200 it is slower than the query pairs on
+    // every workload measured, dense included
+    if (D == 128 && g_attn_kernel == SBA_ATTN_KERNEL_CTA_PAIR)
+        return launch_attention_pair<4>(q, k, v, o, lse, B, H, Npad, valid_len, kv_idx, kv_cnt, kmax, dense,
+                                        softmax_scale, s);
     if (D == 128)
         return launch_attention<128, 2>(q, k, v, o, lse, B, H, Npad, valid_len, kv_idx, kv_cnt, kmax,
                                         dense, pair_order, softmax_scale, s);
@@ -431,6 +473,13 @@ sba_status sba_get_device_status(void* stream) {
 }
 
 void sba_set_wait_limit(uint64_t cycles) { g_wait_limit = cycles ? cycles : kDefaultWaitLimit; }
+
+sba_status sba_set_attention_kernel(int which) {
+    if (which != SBA_ATTN_KERNEL_AUTO && which != SBA_ATTN_KERNEL_QUERY_PAIRS && which != SBA_ATTN_KERNEL_CTA_PAIR)
+        return SBA_ERR_INVALID_ARG;
+    g_attn_kernel = which;
+    return SBA_OK;
+}
 
 const char* sba_strerror(sba_status status) {
     switch (status) {

@@ -77,6 +77,8 @@ def lib() -> ctypes.CDLL:
         L.sba_get_device_status.argtypes = [vp]
         L.sba_set_wait_limit.restype = None
         L.sba_set_wait_limit.argtypes = [ctypes.c_uint64]
+        L.sba_set_attention_kernel.restype = i32
+        L.sba_set_attention_kernel.argtypes = [i32]
         L.sba_pool_select_noalloc.restype = i32
         L.sba_pool_select_noalloc.argtypes = [vp, vp, i32, i32, i32, i32, vp, i32, f64, i32, vp, vp, vp]
         L.sba_noalloc_scratch_bytes.restype = sz
@@ -349,3 +351,15 @@ def device_status(stream=None) -> int:
 
 def set_wait_limit(cycles: int) -> None:
     lib().sba_set_wait_limit(int(cycles))
+
+
+_ATTN_KERNELS = {"auto": 0, "query_pairs": 1, "cta_pair": 2}
+
+
+def set_attention_kernel(which: str) -> None:
+    """Which D = 128 attention kernel the attention calls run (process-wide):
+    "query_pairs" (one SM per two query blocks), "cta_pair" (a 2-SM cluster per four
+    query blocks) or "auto" (the query pairs, the faster one on B200)."""
+    if which not in _ATTN_KERNELS:
+        raise ValueError(f"unknown attention kernel {which!r}; one of {sorted(_ATTN_KERNELS)}")
+    _check(lib().sba_set_attention_kernel(_ATTN_KERNELS[which]), "sba_set_attention_kernel")
