@@ -65,8 +65,8 @@ def parse():
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one attention launch,
 # from the ncu captures summarised in profiles/attn_kernel_*.md, and the hash
 # of the kernel sources it was taken with.  Reported only while the sources match.
-ATTN_TRAFFIC = {"480p_dense": (633502720 + 188913920, "f6f66ea55d2d8d99"),
-                "720p": (3049651000 + 806195200, "f6f66ea55d2d8d99")}
+ATTN_TRAFFIC = {"480p_dense": (631184384 + 187226112, "bec59ccee166ae67"),
+                "720p": (2970393000 + 804928000, "bec59ccee166ae67")}
 KERNEL_SOURCES = ("video_dit_block_b200/csrc/attention.cuh", "video_dit_block_b200/csrc/ptx.cuh",
                   "video_dit_block_b200/csrc/common.cuh")
 

@@ -267,39 +267,55 @@ __device__ __forceinline__ void attn_body(const CUtensorMap& tmQ, const CUtensor
         }
     } else if (warp == 5) {
         // ------------------------------------------------------------ MMA issuer
+        // The tensor pipe queues only a few MMAs, so this thread issues without stalls:
+        // descriptors are precomputed (a shared-memory descriptor steps by adding
+        // (byte offset >> 4) to its start-address field), the barriers of the next
+        // group are tested (non-blocking) before the current group issues and read
+        // after it, and a pending one is waited for by polling.
         if (lane == 0 && n_all > 0) {
-            bool ok = wait_bounded(bar_q, 0, abort_flag, lim);
+            bool ok = poll_bounded(bar_q, 0, abort_flag, lim);
             tc_fence_after();
+            uint64_t dq[D / 16], dk[D / 16], dv[4];
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                dq[kk] = smem_desc_sw128(sQ + (kk / 4) * (128 * 128) + (kk % 4) * 32, 16, 1024);
+                dk[kk] = smem_desc_sw128(sK + (kk / 4) * (64 * 128) + (kk % 4) * 32, 16, 1024);
+            }
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) dv[kk] = smem_desc_sw128(sV + kk * (16 * 128), 64 * 128, 1024);
+            constexpr uint64_t kStep = SM::kKVBytes >> 4;
+            bool k_pre = false;  // K(j) seen ready during the previous PV group
             for (int j = 0; ok && j <= n_all; ++j) {
+                bool p_ok = false, v_ok = false;
+                const int jj = j - 1, sv = jj >= 0 ? jj % NS : 0;
                 if (j < n_all) {
                     const int st = j % NS;
-                    if (!wait_bounded(bar_kf(st), (j / NS) & 1, abort_flag, lim)) { ok = false; break; }
+                    if (!k_pre && !poll_bounded(bar_kf(st), (j / NS) & 1, abort_flag, lim)) { ok = false; break; }
                     tc_fence_after();
+                    if (jj >= 0) {
+                        p_ok = mbar_test_wait(bar_pf(jj & 1), (jj >> 1) & 1);
+                        v_ok = mbar_test_wait(bar_vf(sv), (jj / NS) & 1);
+                    }
                     const uint32_t dS = tmem + (j & 1) * 64;
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint64_t a = smem_desc_sw128(sQ + (kk / 4) * (128 * 128) + (kk % 4) * 32, 16, 1024);
-                        const uint64_t bd = smem_desc_sw128(
-                            sK + st * SM::kKVBytes + (kk / 4) * (64 * 128) + (kk % 4) * 32, 16, 1024);
-                        mma_bf16_ss(dS, a, bd, kIdescS, kk > 0 ? 1u : 0u);
-                    }
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        mma_bf16_ss(dS, dq[kk], dk[kk] + st * kStep, kIdescS, kk > 0 ? 1u : 0u);
                     mma_commit(bar_sf(j & 1));
                     mma_commit(bar_ke(st));
                 }
-                if (j >= 1) {
-                    const int jj = j - 1, st = jj % NS;
-                    if (!wait_bounded(bar_pf(jj & 1), (jj >> 1) & 1, abort_flag, lim)) { ok = false; break; }
-                    if (!wait_bounded(bar_vf(st), (jj / NS) & 1, abort_flag, lim)) { ok = false; break; }
+                k_pre = false;
+                if (jj >= 0) {
+                    if (!p_ok && !poll_bounded(bar_pf(jj & 1), (jj >> 1) & 1, abort_flag, lim)) { ok = false; break; }
+                    if (!v_ok && !poll_bounded(bar_vf(sv), (jj / NS) & 1, abort_flag, lim)) { ok = false; break; }
                     tc_fence_after();
+                    const int jn = j + 1;
+                    if (jn < n_all) k_pre = mbar_test_wait(bar_kf(jn % NS), (jn / NS) & 1);
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const uint64_t bd = smem_desc_sw128(sV + st * SM::kKVBytes + kk * (16 * 128),
-                                                            64 * 128, 1024);
-                        mma_bf16_ts(tmem + 128, tmem + (jj & 1) * 64 + kk * 8, bd, kIdescPV,
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16_ts(tmem + 128, tmem + (jj & 1) * 64 + kk * 8, dv[kk] + sv * kStep, kIdescPV,
                                     (jj > 0 || kk > 0) ? 1u : 0u);
-                    }
                     mma_commit(bar_pv(jj & 1));
-                    mma_commit(bar_ve(st));
+                    mma_commit(bar_ve(sv));
                 }
             }
         }

@@ -81,23 +81,6 @@ struct Attn2Smem {
     static constexpr int kAlloc = kTotal + 1024;
 };
 
-// Bounded wait by polling (the thread is never suspended, so it resumes as soon as the
-// phase completes).  For the MMA thread, whose every stall idles the tensor pipe.
-__device__ __forceinline__ bool poll_bounded(uint32_t bar, uint32_t parity, volatile uint32_t* abort,
-                                             uint64_t limit) {
-    if (mbar_test_wait(bar, parity)) return true;
-    const long long t0 = clock64();
-    while (true) {
-        if (mbar_test_wait(bar, parity)) return true;
-        if (*abort) return false;
-        if ((uint64_t)(clock64() - t0) > limit) {
-            raise_device_error(kErrTimeout);
-            *abort = 1u;
-            return false;
-        }
-    }
-}
-
 // 2^y for two values on the FMA pipe.  y = j + f with j = round(y), |f| <= 1/2; 2^f is
 // a degree-3 polynomial with constant term 1 fitted for least maximum relative error
 // on [-1/2, 1/2] (about 1.0e-4, below the bf16 rounding that P then takes), and j is

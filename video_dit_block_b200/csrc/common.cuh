@@ -51,6 +51,23 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
     }
 }
 
+// Bounded wait by polling (the thread is never suspended, so it resumes as soon as the
+// phase completes).  For the MMA thread, whose every stall idles the tensor pipe.
+__device__ __forceinline__ bool poll_bounded(uint32_t bar, uint32_t parity, volatile uint32_t* abort,
+                                             uint64_t limit) {
+    if (mbar_test_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (mbar_test_wait(bar, parity)) return true;
+        if (*abort) return false;
+        if ((uint64_t)(clock64() - t0) > limit) {
+            raise_device_error(kErrTimeout);
+            *abort = 1u;
+            return false;
+        }
+    }
+}
+
 // Warp-collective form: every lane waits, and all lanes agree on the outcome,
 // so warp-synchronous tcgen05 loads that follow are never reached by part of a warp.
 __device__ __forceinline__ bool warp_wait_bounded(uint32_t bar, uint32_t parity,
