@@ -232,6 +232,28 @@ sba_status sba_attention_paired(const void* q, const void* k, const void* v, voi
                                 const int32_t* kv_idx, const int32_t* kv_cnt, int kmax,
                                 const int32_t* pair_order, float softmax_scale, void* stream);
 
+/* sba_attention_paired with the output stored straight into sequence shards: the
+ * exchange back from head sharding to sequence sharding of the page "MiniMax-H3 on
+ * 8xH200 benchmark", which runs attention under SP/Ulysses.  The caller holds, for its
+ * H heads h_first .. h_first + H - 1 of h_total, the whole sequence (q, k, v as in
+ * sba_attention); the sequence is split into n_shards equal ranges of
+ * shard_len = Npad / n_shards tokens, range s owned by shard s.
+ *   o_shards:   host array of n_shards device pointers, bf16 [B][h_total][shard_len][D];
+ *               token n of head h_first + h goes to shard n / shard_len, row n % shard_len.
+ *               Other GPUs' memory (peer pointers, e.g. symmetric memory) is allowed: the
+ *               stores cross NVLink once per element, in place of an all-to-all.
+ *   lse_shards: NULL, or a host array of n_shards device pointers, fp32 [B][h_total][shard_len].
+ * Only the caller's heads are written; rows past a sample's valid length get 0 / -inf.
+ * pair_order may be NULL (adjacent pairs).  1 <= n_shards <= 8 and Npad % n_shards == 0,
+ * else SBA_ERR_INVALID_ARG; a shard pointer not 16-byte (o) or 4-byte (lse) aligned gives
+ * SBA_ERR_ALIGNMENT.  Stream-ordered; the shards' owners must synchronise with this
+ * stream before reading. */
+sba_status sba_attention_to_shards(const void* q, const void* k, const void* v, void* const* o_shards,
+                                   float* const* lse_shards, int n_shards, int h_total, int h_first, int B,
+                                   int H, int Npad, int D, const int32_t* valid_len, int block,
+                                   const int32_t* kv_idx, const int32_t* kv_cnt, int kmax,
+                                   const int32_t* pair_order, float softmax_scale, void* stream);
+
 /* Dense attention over all valid tokens of each sample (the sparsity = 0 case
  * without a routing), same layouts as sba_attention. */
 sba_status sba_dense_attention(const void* q, const void* k, const void* v, void* o, float* lse,

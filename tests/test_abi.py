@@ -183,3 +183,21 @@ def test_compensated_rejects(lib):
     assert f(ws=NULL) == 1 and f(wsb=16) == 1 and f(kmax=0) == 1
     assert f(D=96) == 2
     assert f(ws=MIS) == 3 and f(po=ctypes.c_void_p(0x10002)) == 3
+
+
+def test_attention_to_shards_rejects(lib):
+    def f(n=2, ptrs=None, lptrs=None, h_total=4, h_first=2, H=2, Npad=1024, D=128, q=A, idx=A):
+        arr = (ctypes.c_void_p * max(n, 1))(*(ptrs if ptrs is not None else [A.value] * max(n, 1)))
+        larr = None if lptrs is None else (ctypes.c_void_p * max(n, 1))(*lptrs)
+        return lib.sba_attention_to_shards(q, A, A, ctypes.cast(arr, ctypes.c_void_p),
+                                           None if larr is None else ctypes.cast(larr, ctypes.c_void_p), n, h_total,
+                                           h_first, 1, H, Npad, D, NULL, 64, idx, A, 8, NULL, 0.0, S)
+    assert f(n=0) == 1 and f(n=9) == 1                    # 1 .. 8 shards
+    assert f(Npad=1024, n=3) == 1                          # Npad must split evenly
+    assert f(h_first=3) == 1 and f(h_first=-1) == 1        # heads outside h_total
+    assert f(ptrs=[A.value, None]) == 1                    # a missing shard
+    assert f(lptrs=[A.value, None]) == 1
+    assert f(ptrs=[A.value, MIS.value]) == 3               # o shards 16-byte aligned
+    assert f(lptrs=[A.value, 0x10002]) == 3                # lse shards 4-byte aligned
+    assert f(q=NULL) == 1 and f(idx=NULL) == 1
+    assert f(D=96) == 2

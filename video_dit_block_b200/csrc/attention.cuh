@@ -49,6 +49,7 @@
 namespace sba {
 
 constexpr int kMaxBlocks = 4096;  // SBA_MAX_NPAD / 64
+constexpr int kMaxShards = 8;
 
 struct AttnParams {
     __nv_bfloat16* o;
@@ -63,6 +64,18 @@ struct AttnParams {
     int dense;
     float scale_log2;  // softmax scale * log2(e)
     unsigned long long wait_limit;
+    // Output to sequence shards: the Ulysses exchange back to sequence sharding, done by
+    // the epilogue's stores.  With n_shards > 0, token n of this call's head h goes to
+    // shard s = n / shard_len, row (b * h_total + h_first + h) * shard_len + n - s * shard_len
+    // of o_shard[s] / lse_shard[s] ([B][h_total][shard_len][D] and [.][.][shard_len]);
+    // the shards may be other GPUs' memory (peer pointers), so each output element
+    // crosses NVLink once, in place of an all-to-all and its copy.
+    int n_shards = 0;
+    int shard_len = 0;
+    int h_total = 0;
+    int h_first = 0;
+    __nv_bfloat16* o_shard[kMaxShards] = {};
+    float* lse_shard[kMaxShards] = {};
 };
 
 template <int D, int NS>
@@ -457,7 +470,18 @@ __device__ __forceinline__ void attn_body(const CUtensorMap& tmQ, const CUtensor
         tc_fence_after();
         const bool in_range = qb[half] >= 0 && qb[half] < nQ;
         const bool valid = tok < L && l > 0.f;
-        __nv_bfloat16* orow = p.o + ((size_t)bh * p.Npad + tok) * D;
+        __nv_bfloat16* orow;
+        float* lrow;
+        if (p.n_shards > 0) {
+            int sh = tok / p.shard_len;
+            sh = sh < p.n_shards ? sh : p.n_shards - 1;  // rows outside the range are not stored
+            const size_t row = (size_t)(b * p.h_total + p.h_first + h) * p.shard_len + (tok - sh * p.shard_len);
+            orow = p.o_shard[sh] + row * D;
+            lrow = p.lse_shard[sh] ? p.lse_shard[sh] + row : nullptr;
+        } else {
+            orow = p.o + ((size_t)bh * p.Npad + tok) * D;
+            lrow = p.lse ? p.lse + (size_t)bh * p.Npad + tok : nullptr;
+        }
         if (ok) {
             const float inv_l = valid ? 1.f / l : 0.f;
 #pragma unroll
@@ -482,9 +506,7 @@ __device__ __forceinline__ void attn_body(const CUtensorMap& tmQ, const CUtensor
                         dst[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
                 }
             }
-            if (in_range && p.lse)
-                p.lse[(size_t)bh * p.Npad + tok] =
-                    valid ? (m + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
+            if (in_range && lrow) *lrow = valid ? (m + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
         }
     }
 

@@ -74,13 +74,23 @@ bool make_map(CUtensorMap* map, const void* base, int BH, int Npad, int D, int b
     return r == CUDA_SUCCESS;
 }
 
+// Where the epilogue stores the output when it goes straight to sequence shards.
+struct ShardOut {
+    int n;
+    int h_total;
+    int h_first;
+    void* const* o;
+    float* const* lse;  // NULL: no lse
+};
+
 // kbar / vbar (COMP only): bf16 [BH][nBpad][D] block means for the compensation steps.
 template <int D, int NS, bool COMP = false>
 sba_status launch_attention(const void* q, const void* k, const void* v, void* o, float* lse,
                             int B, int H, int Npad, const int32_t* valid_len,
                             const int32_t* kv_idx, const int32_t* kv_cnt, int kmax, int dense,
                             const int32_t* pair_order, float softmax_scale, cudaStream_t stream,
-                            const void* kbar = nullptr, const void* vbar = nullptr, int nBpad = 0) {
+                            const void* kbar = nullptr, const void* vbar = nullptr, int nBpad = 0,
+                            const ShardOut* shards = nullptr) {
     using SM = sba::AttnSmem<D, NS>;
     CUtensorMap tq, tk, tv, tkb, tvb;
     const int BH = B * H;
@@ -110,6 +120,16 @@ sba_status launch_attention(const void* q, const void* k, const void* v, void* o
     const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)D);
     p.scale_log2 = scale * 1.4426950408889634f;
     p.wait_limit = g_wait_limit;
+    if (shards) {
+        p.n_shards = shards->n;
+        p.shard_len = Npad / shards->n;
+        p.h_total = shards->h_total;
+        p.h_first = shards->h_first;
+        for (int i = 0; i < shards->n; ++i) {
+            p.o_shard[i] = static_cast<__nv_bfloat16*>(shards->o[i]);
+            p.lse_shard[i] = shards->lse ? shards->lse[i] : nullptr;
+        }
+    }
     dim3 grid((Npad / 64 + 1) / 2, H, B);
     if (COMP)
         sba::attn_comp_kernel<D, NS><<<grid, 192, SM::kAlloc, stream>>>(tq, tk, tv, tkb, tvb, p);
@@ -365,7 +385,7 @@ static sba_status attention_common(const void* q, const void* k, const void* v, 
                                    int block, const int32_t* kv_idx, const int32_t* kv_cnt,
                                    int kmax, int dense, const int32_t* pair_order,
                                    float softmax_scale, void* stream, void* comp_ws = nullptr,
-                                   size_t comp_ws_bytes = 0) {
+                                   size_t comp_ws_bytes = 0, const ShardOut* shards = nullptr) {
     sba_status st = check_shape(B, H, Npad, D, block);
     if (st != SBA_OK) return st;
     if (!q || !k || !v || !o) return SBA_ERR_INVALID_ARG;
@@ -409,6 +429,13 @@ static sba_status attention_common(const void* q, const void* k, const void* v, 
         return launch_attention<64, 4, true>(q, k, v, o, lse, B, H, Npad, valid_len, kv_idx, kv_cnt, kmax, 0,
                                              pair_order, softmax_scale, s, kbar, vbar, nBpad);
     }
+    if (shards) {
+        if (D == 128)
+            return launch_attention<128, 2>(q, k, v, o, lse, B, H, Npad, valid_len, kv_idx, kv_cnt, kmax, dense,
+                                            pair_order, softmax_scale, s, nullptr, nullptr, 0, shards);
+        return launch_attention<64, 4>(q, k, v, o, lse, B, H, Npad, valid_len, kv_idx, kv_cnt, kmax, dense,
+                                       pair_order, softmax_scale, s, nullptr, nullptr, 0, shards);
+    }
     // the CTA-pair kernel only when chosen: on B200 it is slower than the query pairs on
     // every workload measured, dense included
     if (D == 128 && g_attn_kernel == SBA_ATTN_KERNEL_CTA_PAIR)
@@ -443,6 +470,26 @@ sba_status sba_dense_attention(const void* q, const void* k, const void* v, void
                                float softmax_scale, void* stream) {
     return attention_common(q, k, v, o, lse, B, H, Npad, D, valid_len, 64, nullptr, nullptr, 0, 1,
                             nullptr, softmax_scale, stream);
+}
+
+sba_status sba_attention_to_shards(const void* q, const void* k, const void* v, void* const* o_shards,
+                                   float* const* lse_shards, int n_shards, int h_total, int h_first, int B,
+                                   int H, int Npad, int D, const int32_t* valid_len, int block,
+                                   const int32_t* kv_idx, const int32_t* kv_cnt, int kmax,
+                                   const int32_t* pair_order, float softmax_scale, void* stream) {
+    if (!o_shards || n_shards < 1 || n_shards > sba::kMaxShards) return SBA_ERR_INVALID_ARG;
+    if (Npad <= 0 || Npad % n_shards != 0 || h_first < 0 || H < 1 || h_total < h_first + H)
+        return SBA_ERR_INVALID_ARG;
+    for (int i = 0; i < n_shards; ++i) {
+        if (!o_shards[i] || (lse_shards && !lse_shards[i])) return SBA_ERR_INVALID_ARG;
+        if (!aligned16(o_shards[i]) || (lse_shards && (reinterpret_cast<uintptr_t>(lse_shards[i]) & 3u)))
+            return SBA_ERR_ALIGNMENT;
+    }
+    if ((long long)B * h_total * (Npad / n_shards) > (1ll << 31)) return SBA_ERR_UNSUPPORTED;
+    const ShardOut sh{n_shards, h_total, h_first, o_shards, lse_shards};
+    // o is not written; any 16-byte aligned pointer passes the common checks
+    return attention_common(q, k, v, o_shards[0], nullptr, B, H, Npad, D, valid_len, block, kv_idx, kv_cnt, kmax, 0,
+                            pair_order, softmax_scale, stream, nullptr, 0, &sh);
 }
 
 size_t sba_compensation_workspace_size(int B, int H, int Npad, int D, int block) {

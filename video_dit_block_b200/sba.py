@@ -73,6 +73,9 @@ def lib() -> ctypes.CDLL:
                                            f32, vp]
         L.sba_dense_attention.restype = i32
         L.sba_dense_attention.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, f32, vp]
+        L.sba_attention_to_shards.restype = i32
+        L.sba_attention_to_shards.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, i32,
+                                              vp, vp, i32, vp, f32, vp]
         L.sba_get_device_status.restype = i32
         L.sba_get_device_status.argtypes = [vp]
         L.sba_set_wait_limit.restype = None
@@ -291,6 +294,39 @@ def attention_paired(q, k, v, kv_idx, kv_cnt, pair_order, valid_len=None, softma
                                       _ptr(kv_cnt), kv_idx.shape[-1], _ptr(pair_order), float(softmax_scale),
                                       _stream(stream)), "sba_attention_paired")
     return out, lse
+
+
+def attention_to_shards(q, k, v, kv_idx, kv_cnt, o_shards, lse_shards=None, h_first: int = 0, h_total=None,
+                        valid_len=None, pair_order=None, softmax_scale: float = 0.0, block: int = BLOCK,
+                        stream=None):
+    """Attention for this caller's heads h_first .. h_first + H - 1 (q, k, v: [B, H, Npad, D],
+    the whole sequence), each output row stored straight into the sequence shard that owns
+    its token: o_shards[s] is bf16 [B, h_total, Npad / len(o_shards), D] (a tensor, or a raw
+    device pointer such as a peer's symmetric-memory buffer, then h_total is required);
+    lse_shards likewise fp32 [B, h_total, Npad / len(o_shards)] or None."""
+    B, H, Npad, D = _qkv(q, k, v)
+    n = len(o_shards)
+    if n < 1 or n > 8:
+        raise ValueError("between 1 and 8 output shards")
+    ptr = lambda t: int(t) if isinstance(t, int) else t.data_ptr()
+    if h_total is None:
+        if isinstance(o_shards[0], int):
+            raise ValueError("h_total is required with raw shard pointers")
+        h_total = o_shards[0].shape[1]
+    for t in list(o_shards) + list(lse_shards or []):
+        if not isinstance(t, int):
+            exp = torch.bfloat16 if t.dim() == 4 else torch.float32
+            shape = (B, h_total, Npad // n) + ((D,) if t.dim() == 4 else ())
+            if t.dtype != exp or tuple(t.shape) != shape or not t.is_contiguous() or t.device != q.device:
+                raise ValueError(f"shard of shape {tuple(t.shape)} / {t.dtype}; expected {shape} / {exp}, contiguous")
+    o_arr = (ctypes.c_void_p * n)(*[ptr(t) for t in o_shards])
+    l_arr = None if lse_shards is None else (ctypes.c_void_p * n)(*[ptr(t) for t in lse_shards])
+    _check(lib().sba_attention_to_shards(_ptr(q), _ptr(k), _ptr(v), ctypes.cast(o_arr, ctypes.c_void_p),
+                                         None if l_arr is None else ctypes.cast(l_arr, ctypes.c_void_p), n,
+                                         int(h_total), int(h_first), B, H, Npad, D,
+                                         _ptr(_valid_len(valid_len, q.device)), block, _ptr(kv_idx), _ptr(kv_cnt),
+                                         kv_idx.shape[-1], _ptr(pair_order), float(softmax_scale), _stream(stream)),
+           "sba_attention_to_shards")
 
 
 def attention_compensated(q, k, v, kv_idx, kv_cnt, valid_len=None, pair_order=None, softmax_scale: float = 0.0,

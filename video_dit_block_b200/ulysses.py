@@ -11,6 +11,12 @@ The exchange is torch.distributed's all_to_all_single (NCCL between GPUs, gloo o
 CPU); the tensors travel as int32 pairs of bf16 bit patterns, so the exchange is
 exact and works on either backend.  Token range r * N/P .. (r+1) * N/P lives on
 rank r; heads p * H/P .. (p+1) * H/P are attended on rank p.
+
+ulysses_attention_fused replaces the second exchange: the attention kernel's epilogue
+stores every output row straight into the sequence shard of the rank that owns its
+token (sba_attention_to_shards), so the output crosses the interconnect once, with no
+all-to-all and no copy after it.  The shard buffers are one per rank; across GPUs they
+are peer pointers (symmetric memory), which the caller provides.
 """
 from __future__ import annotations
 
@@ -76,3 +82,28 @@ def ulysses_attention(q, k, v, valid_len=None, sparsity: float = 0.75, group=Non
     res = attention(qh, kh, vh, valid_len, sparsity, **kwargs)
     o_h, lse_h = res[0], res[1]
     return heads_to_seq(o_h, group), lse_heads_to_seq(lse_h, group)
+
+
+def ulysses_attention_fused(q, k, v, valid_len, sparsity: float, o_shards, lse_shards=None, group=None,
+                            h_total=None, softmax_scale: float = 0.0):
+    """Sequence-sharded block-sparse attention with the output exchange fused into the
+    attention kernel.  q, k, v: this rank's [B, H, N/P, D] token range (N a multiple of
+    64 P); valid_len: the samples' full lengths.  o_shards[p] / lse_shards[p]: rank p's
+    output buffers, bf16 [B, H, N/P, D] / fp32 [B, H, N/P] (tensors on this GPU, or raw
+    device pointers to other ranks' memory, then h_total = H is required).  Every rank
+    writes its heads' rows into every rank's shard; the call ends with a barrier of the
+    group, after which each rank's own shard holds its token range for all heads."""
+    from .sba import attention_to_shards, pair_query_blocks, pool_select
+    P = dist.get_world_size(group)
+    r = dist.get_rank(group)
+    if len(o_shards) != P or (lse_shards is not None and len(lse_shards) != P):
+        raise ValueError(f"one output shard per rank ({P})")
+    qh, kh, vh = (seq_to_heads(t, group) for t in (q, k, v))
+    Hl = qh.shape[1]
+    idx, cnt = pool_select(qh, kh, valid_len, sparsity)
+    po = pair_query_blocks(idx, cnt, valid_len)
+    attention_to_shards(qh, kh, vh, idx, cnt, o_shards, lse_shards, h_first=r * Hl, h_total=h_total,
+                        valid_len=valid_len, pair_order=po, softmax_scale=softmax_scale)
+    # every rank's stores into the shards land before any rank reads its own
+    torch.cuda.current_stream().synchronize()
+    dist.barrier(group)
