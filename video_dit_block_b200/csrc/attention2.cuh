@@ -11,8 +11,10 @@
 // cta_group::2 MMA of M = 256, N = 128 splits A by rows (each SM reads its own 128
 // Q rows) and B by columns (each SM reads one 64-key block), so each SM reads 6 KB
 // per 16-deep K step for 64 tensor cycles instead of 6 KB per 32, and the step
-// mix (S: M256 N128 K128, then O += P V: M256 N128 K128, P from TMEM) runs at the
-// full tensor rate with room left for the TMA writes.
+// mix (S: M256 N128 K128, then O += P V: M256 N128 K128, P from TMEM), measured
+// alone, runs at the full tensor rate with room left for the TMA writes.  Inside
+// this kernel it runs at about half that rate; the softmax warps' TMEM stores and
+// barrier waits account for part of the gap.
 //
 // Tiling.  A cluster owns four adjacent 64-row query blocks 4c .. 4c+3 of one (b, h);
 // CTA r of the pair holds 2r and 2r+1 as its 128-row Q tile.  The pair walks the
@@ -41,7 +43,10 @@
 // Completion of an MMA group is multicast to the barrier of both CTAs; the P-ready
 // barrier in CTA 0 counts one arrival per softmax warp of both CTAs.  S is triple
 // buffered and the MMA warp issues S two steps ahead (S(t+2) before O += P(t) V(t)),
-// so the tensor core never waits on one step's softmax for the next scores.
+// so the next scores never wait on one step's softmax.  The epilogue waits on a
+// one-phase barrier committed after the last PV, not on the two-phase PV barrier,
+// whose parity a warp that keeps nothing in its last steps could read two phases
+// early.
 //
 // A quarter of the exponentials run on the FMA pipe (exp2_fma2) instead of the MUFU:
 // eight softmax warps exponentiate 128 x 128 scores per step, which at the MUFU's 16
