@@ -93,3 +93,25 @@ def test_sharded_attention_equals_single_process(case, world):
     o_ref, lse_ref, _, _ = oracle_attention(t(w.q), t(w.k), t(w.v), torch.from_numpy(w.valid_len), s)
     np.testing.assert_array_equal(o_full, o_ref.view(torch.int16).numpy())
     np.testing.assert_array_equal(lse_full, lse_ref.numpy())
+
+
+def test_fused_wrapper_rejects_wrong_shard_count():
+    """ulysses_attention_fused checks its shard list against the group before any exchange
+    or device work (one gloo rank on the CPU)."""
+    import socket
+
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    from video_dit_block_b200 import ulysses
+    with socket.socket() as so:
+        so.bind(("127.0.0.1", 0))
+        port = so.getsockname()[1]
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1)
+    try:
+        x = torch.zeros(1, 2, 64, 64, dtype=torch.bfloat16)
+        with pytest.raises(ValueError):
+            ulysses.ulysses_attention_fused(x, x, x, None, 0.5, [x, x])
+        with pytest.raises(ValueError):
+            ulysses.ulysses_attention_fused(x, x, x, None, 0.5, [x], lse_shards=[x, x])
+    finally:
+        dist.destroy_process_group()
