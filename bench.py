@@ -59,6 +59,8 @@ def parse():
     ap.add_argument("--budget", type=int, default=1)
     ap.add_argument("--producer", action="store_true")
     ap.add_argument("--compensate", action="store_true")
+    ap.add_argument("--attn-kernel", default="auto", choices=["auto", "query_pairs", "cta_pair"],
+                    help="D = 128 attention kernel: the default query pairs, or the opt-in CTA pair")
     return ap.parse_args()
 
 
@@ -298,6 +300,7 @@ def run_ours(args):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
 
+    sba.set_attention_kernel(args.attn_kernel)
     w = make_workload(args.config)
     t = lambda x: torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
     q, k, v = t(w.q), t(w.k), t(w.v)
@@ -459,7 +462,9 @@ def run_ours(args):
         return
     peaks, src = load_peaks()
     tr = ATTN_TRAFFIC.get(w.name)
-    traffic = tr[0] if tr is not None and tr[1] == kernel_source_hash() and not args.compensate else None
+    pair_kernel = args.attn_kernel == "cta_pair" and D == 128 and not args.compensate
+    traffic = (tr[0] if tr is not None and tr[1] == kernel_source_hash() and not args.compensate
+               and not pair_kernel else None)
     peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
     achieved = f_step / (attn_ms * 1e-3) / 1e12
     line = {
@@ -469,12 +474,13 @@ def run_ours(args):
         "data": "synthetic (seeded smooth field + noise, bf16; no weights involved)",
         "config": workload_config(w, {
             "l2": f"inputs {3 * q.numel() * 2 / 1e6:.0f} MB > 126 MB L2; no flush between steps",
-            "kmax": kmax, **router_config(args)}),
+            "kmax": kmax, **router_config(args),
+            **({"attention_kernel": "CTA pair (tcgen05 across two SMs)"} if pair_kernel else {})}),
         "pct_of_spec_bf16_peak": 100.0 * value / world / SPEC_BF16_TFLOPS,
         "attn_ms": attn_ms, "select_ms": sel_ms, "kept_tflop_per_step": f_step / 1e12,
         "roofline": {"bound": "tensor",
-                     "kernel": ("attn_comp_kernel" if args.compensate else "attn_kernel")
-                     + ("<128,2>" if D == 128 else "<64,4>"),
+                     "kernel": "attn_pair_kernel<4>" if pair_kernel else
+                     ("attn_comp_kernel" if args.compensate else "attn_kernel") + ("<128,2>" if D == 128 else "<64,4>"),
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_source": f"{src} bf16_tflops_sustained (kernel timed inside a seconds-long loop)",
                      "traffic": traffic},
