@@ -169,3 +169,42 @@ def test_bad_routing_flagged(sba):
         assert sba.device_status() == 0
     finally:
         sba.set_attention_kernel("auto")
+
+
+def test_max_length_sampled(sba, oracle_mod):
+    """The CTA pair at the length limit (262144 tokens, 4096 blocks), a ragged second
+    sample, s = 0.95; sampled query blocks against the oracle."""
+    w = make_custom(2, 1, 128, (4, 256, 256), 0.95, drop_rate=0.0, seed=41)
+    w.valid_len = np.array([262144, 200000], dtype=np.int32)
+    q, k, v, vl = to_device(w, DEV)
+    idx, cnt = sba.pool_select(q, k, vl, 0.95)
+    sba.set_attention_kernel("cta_pair")
+    try:
+        o, lse = sba.attention(q, k, v, idx, cnt, vl)
+        assert sba.device_status() == 0
+    finally:
+        sba.set_attention_kernel("auto")
+    qb = np.array([0, 1, 2047, 3124], dtype=np.int32)   # 3124 = last block of the second sample
+    for b in range(2):
+        sl = lambda x: np.ascontiguousarray(x[b:b + 1])
+        o_ref, lse_ref = oracle_mod.attention(sl(w.q), sl(w.k), sl(w.v), idx[b:b + 1].cpu().numpy(),
+                                              cnt[b:b + 1].cpu().numpy(), w.valid_len[b:b + 1], qblocks=qb)
+        rows = np.isfinite(lse_ref)
+        mx, mean = output_errors(o[b:b + 1].float().cpu().numpy(), o_ref, rows)
+        assert mx <= MAX_ABS and mean <= MEAN_ABS, (b, mx, mean)
+
+
+def test_d64_falls_back_to_query_pairs(sba, oracle_mod):
+    """The CTA pair is D = 128 only: chosen with D = 64, the query-pair kernel runs."""
+    w = make_custom(1, 2, 64, (2, 8, 24), 0.5, seed=55)
+    q, k, v, vl = to_device(w, DEV)
+    idx, cnt = sba.pool_select(q, k, vl, 0.5)
+    o_ref_gpu, _ = sba.attention(q, k, v, idx, cnt, vl)
+    sba.set_attention_kernel("cta_pair")
+    try:
+        o, lse = sba.attention(q, k, v, idx, cnt, vl)
+        assert sba.device_status() == 0
+    finally:
+        sba.set_attention_kernel("auto")
+    assert torch.equal(o.view(torch.int16), o_ref_gpu.view(torch.int16))
+    check(sba, oracle_mod, w, o, lse, idx.cpu().numpy(), cnt.cpu().numpy())
