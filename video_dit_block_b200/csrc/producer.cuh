@@ -48,12 +48,28 @@ __device__ __forceinline__ void sincos_reduced(float theta, float* s, float* c) 
     *c = __cosf(r);
 }
 
+// Packed fp32 product (mul.rn.f32x2), and the round trip of two fp32 values through
+// bf16 (round to nearest even, as __float2bfloat16_rn) in one packed conversion.
+__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t bf16_round2(uint64_t v) {
+    float a, b;
+    unpack2(v, a, b);
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return pack2(__low2float(h), __high2float(h));
+}
+
 // One CTA of 256 threads per (bh, 64-token block).  A half-warp handles a row (lane l
 // of the half owns channels [CPL l, CPL l + CPL), CPL = D / 16, an even count, so every
 // RoPE pair is within a lane); warp w takes rows w, w + 8, ... two at a time, and all
-// of its rows are loaded before any is processed.
+// of its rows are loaded before any is processed.  Each lane then works on two of its
+// rows at once in packed f32x2 arithmetic.  At D = 128 that takes up to 85 registers,
+// three CTAs per SM; measured 11% faster than one row at a time in 64 registers.
 template <int D>
-__global__ void __launch_bounds__(256, 4) qk_norm_rope_pool_kernel(
+__global__ void __launch_bounds__(256, D == 128 ? 3 : 4) qk_norm_rope_pool_kernel(
     const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ w, const int32_t* __restrict__ pos,
     const int32_t* __restrict__ valid_len, int H, int Npad, int rope_dim, const RopeFreqs freqs, float eps,
     __nv_bfloat16* __restrict__ out, double* __restrict__ means) {
@@ -95,47 +111,88 @@ __global__ void __launch_bounds__(256, 4) qk_norm_rope_pool_kernel(
         auto tof = [](int v) { return __fsub_rn(__int_as_float(0x4B000000 + v), 8388608.0f); };
         pp[j] = make_float3(tof(__ldg(q3)), tof(__ldg(q3 + 1)), tof(__ldg(q3 + 2)));
     }
+    // Rows are taken two at a time (j and j + 1 of this lane), their arithmetic in packed
+    // f32x2 operations: element by element the same operations, in the same order, as
+    // one row at a time, so the same results, for about half the FMA-pipe instructions.
+    const uint64_t kInv2Pi2 = pack2(0.15915494309189535f, 0.15915494309189535f);
+    const uint64_t kRound2 = pack2(12582912.0f, 12582912.0f), kNegRound2 = pack2(-12582912.0f, -12582912.0f);
+    const uint64_t kNeg2PiHi2 = pack2(-6.28125f, -6.28125f);
+    const uint64_t kNeg2PiLo2 = pack2(-1.9353071795864769e-3f, -1.9353071795864769e-3f);
 #pragma unroll
-    for (int j = 0; j < RPW; ++j) {
-        const int r = warp + 8 * (2 * j + sub);
-        const int n = I * kBlock + r;
-        float xv[CPL];
-        const uint32_t* u = reinterpret_cast<const uint32_t*>(&raw[j]);
+    for (int jj = 0; jj < RPW / 2; ++jj) {
+        const int ja = 2 * jj, jb = 2 * jj + 1;
+        float xa[CPL], xb[CPL];
+        {
+            const uint32_t* ua = reinterpret_cast<const uint32_t*>(&raw[ja]);
+            const uint32_t* ub = reinterpret_cast<const uint32_t*>(&raw[jb]);
 #pragma unroll
-        for (int e = 0; e < CPL / 2; ++e) {
-            const __nv_bfloat162 v2 = *reinterpret_cast<const __nv_bfloat162*>(&u[e]);
-            xv[2 * e] = __low2float(v2);
-            xv[2 * e + 1] = __high2float(v2);
+            for (int e = 0; e < CPL / 2; ++e) {
+                const __nv_bfloat162 va = *reinterpret_cast<const __nv_bfloat162*>(&ua[e]);
+                const __nv_bfloat162 vb = *reinterpret_cast<const __nv_bfloat162*>(&ub[e]);
+                xa[2 * e] = __low2float(va);
+                xa[2 * e + 1] = __high2float(va);
+                xb[2 * e] = __low2float(vb);
+                xb[2 * e + 1] = __high2float(vb);
+            }
         }
-        float ss = 0.f;
+        uint64_t ss2 = pack2(0.f, 0.f);
 #pragma unroll
-        for (int e = 0; e < CPL; ++e) ss = fmaf(xv[e], xv[e], ss);
+        for (int e = 0; e < CPL; ++e) {
+            const uint64_t x2 = pack2(xa[e], xb[e]);
+            ss2 = ffma2(x2, x2, ss2);
+        }
+        float ssa, ssb;
+        unpack2(ss2, ssa, ssb);
 #pragma unroll
-        for (int off = 8; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-        const float inv = rsqrtf(ss / (float)D + eps);
-        uint32_t o2[CPL / 2];
+        for (int off = 8; off > 0; off >>= 1) {
+            ssa += __shfl_xor_sync(0xffffffffu, ssa, off);
+            ssb += __shfl_xor_sync(0xffffffffu, ssb, off);
+        }
+        const uint64_t inv2 = pack2(rsqrtf(ssa / (float)D + eps), rsqrtf(ssb / (float)D + eps));
+        uint32_t oa[CPL / 2], ob[CPL / 2];
 #pragma unroll
         for (int e = 0; e < CPL; e += 2) {
-            // the norm, rounded to bf16 before the rotation
-            const float y0 = __bfloat162float(__float2bfloat16_rn(xv[e] * inv * wv[e]));
-            const float y1 = __bfloat162float(__float2bfloat16_rn(xv[e + 1] * inv * wv[e + 1]));
-            // every lane evaluates the rotation (no divergent branch); channels past
-            // rope_dim then keep y by a select
+            // the norm, rounded to bf16 before the rotation: y0 = channel e, y1 = e + 1,
+            // rows a and b in the two halves
+            const uint64_t t0 = fmul2(fmul2(pack2(xa[e], xb[e]), inv2), pack2(wv[e], wv[e]));
+            const uint64_t t1 = fmul2(fmul2(pack2(xa[e + 1], xb[e + 1]), inv2), pack2(wv[e + 1], wv[e + 1]));
+            const uint64_t y0 = bf16_round2(t0), y1 = bf16_round2(t1);
             const int a = ax[e / 2];
-            const float pa = a == 0 ? pp[j].x : (a == 1 ? pp[j].y : pp[j].z);
-            float sn, cs;
-            sincos_reduced(pa * fr[e / 2], &sn, &cs);
-            const float r0 = a >= 0 ? fmaf(y0, cs, -y1 * sn) : y0;
-            const float r1 = a >= 0 ? fmaf(y0, sn, y1 * cs) : y1;
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(r0, r1);
-            o2[e / 2] = *reinterpret_cast<uint32_t*>(&h2);
+            const float pa_a = a == 0 ? pp[ja].x : (a == 1 ? pp[ja].y : pp[ja].z);
+            const float pa_b = a == 0 ? pp[jb].x : (a == 1 ? pp[jb].y : pp[jb].z);
+            const uint64_t ang = fmul2(pack2(pa_a, pa_b), pack2(fr[e / 2], fr[e / 2]));
+            // sincos_reduced on both angles: the same Cody-Waite steps, packed
+            const uint64_t k = fadd2(ffma2(ang, kInv2Pi2, kRound2), kNegRound2);
+            uint64_t rr = ffma2(k, kNeg2PiHi2, ang);
+            rr = ffma2(k, kNeg2PiLo2, rr);
+            float ra, rb;
+            unpack2(rr, ra, rb);
+            const float sa = __sinf(ra), ca = __cosf(ra), sb = __sinf(rb), cb = __cosf(rb);
+            const uint64_t cs = pack2(ca, cb), sn = pack2(sa, sb);
+            const uint64_t r0 = ffma2(y0, cs, fmul2(y1, pack2(-sa, -sb)));
+            const uint64_t r1 = ffma2(y0, sn, fmul2(y1, cs));
+            float r0a, r0b, r1a, r1b, y0a, y0b, y1a, y1b;
+            unpack2(r0, r0a, r0b);
+            unpack2(r1, r1a, r1b);
+            unpack2(y0, y0a, y0b);
+            unpack2(y1, y1a, y1b);
+            // channels past rope_dim keep y (a select: every lane evaluates the rotation)
+            __nv_bfloat162 ha = __floats2bfloat162_rn(a >= 0 ? r0a : y0a, a >= 0 ? r1a : y1a);
+            __nv_bfloat162 hb = __floats2bfloat162_rn(a >= 0 ? r0b : y0b, a >= 0 ? r1b : y1b);
+            oa[e / 2] = *reinterpret_cast<uint32_t*>(&ha);
+            ob[e / 2] = *reinterpret_cast<uint32_t*>(&hb);
         }
-        Vec ov;
-        uint32_t* ou = reinterpret_cast<uint32_t*>(&ov);
 #pragma unroll
-        for (int e = 0; e < CPL / 2; ++e) ou[e] = o2[e];
-        *reinterpret_cast<Vec*>(out + ((size_t)bh * Npad + n) * D + c0) = ov;
-        if (means) *reinterpret_cast<Vec*>(tile + r * D + c0) = ov;
+        for (int h2 = 0; h2 < 2; ++h2) {
+            const int r = warp + 8 * (2 * (h2 ? jb : ja) + sub);
+            const int n = I * kBlock + r;
+            Vec ov;
+            uint32_t* ou = reinterpret_cast<uint32_t*>(&ov);
+#pragma unroll
+            for (int e = 0; e < CPL / 2; ++e) ou[e] = h2 ? ob[e] : oa[e];
+            *reinterpret_cast<Vec*>(out + ((size_t)bh * Npad + n) * D + c0) = ov;
+            if (means) *reinterpret_cast<Vec*>(tile + r * D + c0) = ov;
+        }
     }
     if (!means) return;
     __syncthreads();
