@@ -302,6 +302,7 @@ def run_ours(args):
 
     sba.set_attention_kernel(args.attn_kernel)
     w = make_workload(args.config)
+    pair_kernel = args.attn_kernel == "cta_pair" and w.D == 128 and not args.compensate
     t = lambda x: torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
     q, k, v = t(w.q), t(w.k), t(w.v)
     vl = torch.from_numpy(w.valid_len).to(dev)
@@ -344,7 +345,8 @@ def run_ours(args):
         else:
             sba.pool_select(qq, kk, vll, w.sparsity, kmax, kv_idx=kv_idx, kv_cnt=kv_cnt, workspace=ws,
                             stream=stream)
-        sba.pair_query_blocks(kv_idx, kv_cnt, vll, pair_order=pair_order, workspace=pws, stream=stream)
+        if not pair_kernel:  # the CTA-pair kernel tiles four adjacent query blocks itself
+            sba.pair_query_blocks(kv_idx, kv_cnt, vll, pair_order=pair_order, workspace=pws, stream=stream)
         return qq, kk
 
     if args.compensate:
@@ -462,7 +464,6 @@ def run_ours(args):
         return
     peaks, src = load_peaks()
     tr = ATTN_TRAFFIC.get(w.name)
-    pair_kernel = args.attn_kernel == "cta_pair" and D == 128 and not args.compensate
     traffic = (tr[0] if tr is not None and tr[1] == kernel_source_hash() and not args.compensate
                and not pair_kernel else None)
     peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
@@ -485,11 +486,12 @@ def run_ours(args):
                      "peak_source": f"{src} bf16_tflops_sustained (kernel timed inside a seconds-long loop)",
                      "traffic": traffic},
         # per step: routing = 2 pooling + key-norm maximum + screen (only when blocks are
-        # dropped) + top-k; pairing = bitmaps + 4 x (propose, resolve) + emit; 1 attention
+        # dropped) + top-k; pairing = bitmaps + 4 x (propose, resolve) + emit (not with the
+        # CTA-pair kernel); 1 attention
         # (--producer: 2 producer launches and 2 splits of the given means replace pooling)
         # (--compensate: 2 block-mean launches before the attention)
-        "gpu_launches": (4 + (1 if w.sparsity > 0 else 0) + (2 if args.producer else 0) + 10 + 1
-                         + (2 if args.compensate else 0)) * K,
+        "gpu_launches": (4 + (1 if w.sparsity > 0 else 0) + (2 if args.producer else 0)
+                         + (0 if pair_kernel else 10) + 1 + (2 if args.compensate else 0)) * K,
         "clocks": clk,
     }
     if e2e is not None:

@@ -113,5 +113,7 @@ def test_fused_wrapper_rejects_wrong_shard_count():
             ulysses.ulysses_attention_fused(x, x, x, None, 0.5, [x, x])
         with pytest.raises(ValueError):
             ulysses.ulysses_attention_fused(x, x, x, None, 0.5, [x], lse_shards=[x, x])
+        with pytest.raises(ValueError):
+            ulysses.ulysses_attention_fused(x, x, x, None, 0.5, [x], router="topk")
     finally:
         dist.destroy_process_group()

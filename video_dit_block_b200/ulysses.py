@@ -85,22 +85,28 @@ def ulysses_attention(q, k, v, valid_len=None, sparsity: float = 0.75, group=Non
 
 
 def ulysses_attention_fused(q, k, v, valid_len, sparsity: float, o_shards, lse_shards=None, group=None,
-                            h_total=None, softmax_scale: float = 0.0):
+                            h_total=None, softmax_scale: float = 0.0, router: str = "mean", budget: int = 1):
     """Sequence-sharded block-sparse attention with the output exchange fused into the
     attention kernel.  q, k, v: this rank's [B, H, N/P, D] token range (N a multiple of
     64 P); valid_len: the samples' full lengths.  o_shards[p] / lse_shards[p]: rank p's
     output buffers, bf16 [B, H, N/P, D] / fp32 [B, H, N/P] (tensors on this GPU, or raw
     device pointers to other ranks' memory, then h_total = H is required).  Every rank
     writes its heads' rows into every rank's shard; the call ends with a barrier of the
-    group, after which each rank's own shard holds its token range for all heads."""
-    from .sba import attention_to_shards, pair_query_blocks, pool_select
+    group, after which each rank's own shard holds its token range for all heads.  router /
+    budget as in sparse_attention."""
+    from .sba import attention_to_shards, pair_query_blocks, pool_select, pool_select_lse
     P = dist.get_world_size(group)
     r = dist.get_rank(group)
     if len(o_shards) != P or (lse_shards is not None and len(lse_shards) != P):
         raise ValueError(f"one output shard per rank ({P})")
+    if router not in ("mean", "lse"):
+        raise ValueError(f"unknown router {router!r}")
     qh, kh, vh = (seq_to_heads(t, group) for t in (q, k, v))
     Hl = qh.shape[1]
-    idx, cnt = pool_select(qh, kh, valid_len, sparsity)
+    if router == "mean":
+        idx, cnt = pool_select(qh, kh, valid_len, sparsity)
+    else:
+        idx, cnt = pool_select_lse(qh, kh, valid_len, sparsity, budget=budget)
     po = pair_query_blocks(idx, cnt, valid_len)
     attention_to_shards(qh, kh, vh, idx, cnt, o_shards, lse_shards, h_first=r * Hl, h_total=h_total,
                         valid_len=valid_len, pair_order=po, softmax_scale=softmax_scale)
