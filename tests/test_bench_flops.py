@@ -1,6 +1,8 @@
-"""The metric's FLOP count (bench.kept_flops): 4 D for every (query token, kept key token)
-pair of valid tokens.  Pinned by the dense closed form -- including the 480p dense figure of
-4 * 128 * 24 * 32760^2 = 1.319e13 FLOPs -- and by brute-force enumeration of token pairs."""
+"""bench.py's host arithmetic on the CPU.  The metric's FLOP count (kept_flops): 4 D for
+every (query token, kept key token) pair of valid tokens, pinned by the dense closed form --
+including the 480p dense figure of 4 * 128 * 24 * 32760^2 = 1.319e13 FLOPs -- and by
+brute-force enumeration of token pairs; the whole-job value; and the clock summary read
+from nvidia-smi lines."""
 import os
 import sys
 
@@ -58,3 +60,44 @@ def test_brute_force_token_pairs():
 def test_whole_job_value_sums_replicas():
     assert bench.whole_job_value(2e12, 4.0, 1) == 2e12 / 4e-3 / 1e12
     assert bench.whole_job_value(2e12, 4.0, 8) == 8 * 2e12 / 4e-3 / 1e12
+
+
+class _FakeProc:
+    def terminate(self):
+        pass
+
+    def wait(self, timeout=None):
+        return 0
+
+
+class _FakeThread:
+    def join(self, timeout=None):
+        pass
+
+
+def test_clock_sampler_window_and_reasons():
+    """Only samples inside the timed window (widened by one interval) count; throttle
+    reasons are read from their columns; malformed lines are skipped."""
+    cs = bench.ClockSampler(0)
+    cs.proc, cs.thread = _FakeProc(), _FakeThread()
+    active = "Active"
+    idle = "Not Active"
+    cs.lines = [
+        (0.50, f"0, 900, 1965, 400.0, 0x1, {active}, {idle}, {idle}, {idle}"),      # before the window
+        (1.00, f"0, 1965, 1965, 700.0, 0x4, {idle}, {idle}, {idle}, {active}"),
+        (1.05, f"0, 1800, 1965, 950.5, 0x4, {idle}, {idle}, {idle}, {active}"),
+        (1.08, "0, [N/A], 1965"),                                                    # malformed
+        (1.10, f"0, 1700, 1965, [N/A], 0x40, {idle}, {active}, {idle}, {idle}"),
+        (3.00, f"0, 500, 1965, 100.0, 0x8, {idle}, {idle}, {active}, {idle}"),     # after the window
+    ]
+    cs.mark(0.95, 1.05)
+    r = cs.stop()
+    assert r["samples"] == 3
+    assert r["sm_mhz"] == 1800.0 and r["sm_max_mhz"] == 1965.0
+    assert r["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
+
+
+def test_clock_sampler_without_nvidia_smi():
+    cs = bench.ClockSampler(0)
+    r = cs.stop()
+    assert r["sm_mhz"] is None and r["reasons"] == ["nvidia-smi unavailable"]
