@@ -201,3 +201,10 @@ def test_attention_to_shards_rejects(lib):
     assert f(lptrs=[A.value, 0x10002]) == 3                # lse shards 4-byte aligned
     assert f(q=NULL) == 1 and f(idx=NULL) == 1
     assert f(D=96) == 2
+
+
+def test_set_attention_kernel_values(lib):
+    for which in (0, 1, 2):
+        assert lib.sba_set_attention_kernel(which) == 0
+    assert lib.sba_set_attention_kernel(3) == 1 and lib.sba_set_attention_kernel(-1) == 1
+    assert lib.sba_set_attention_kernel(0) == 0        # back to the default
