@@ -57,7 +57,7 @@ def _load():
         _lib.oracle_qk_norm_rope.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, f64, f64, vp, vp]
         _lib.oracle_attention_compensated.restype = i32
         _lib.oracle_attention_compensated.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, i32, vp, vp, i32,
-                                                      f64, vp, i32, vp, vp]
+                                                      f64, i32, vp, i32, vp, vp]
         _lib.oracle_attention.restype = i32
         _lib.oracle_attention.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, i32, vp, vp, i32,
                                           f64, vp, i32, vp, vp]
@@ -231,9 +231,12 @@ def attention(q, k, v, kv_idx, kv_cnt, valid_len=None, scale: float = 0.0, block
 
 
 def attention_compensated(q, k, v, kv_idx, kv_cnt, valid_len=None, scale: float = 0.0, block: int = 64,
-                          qblocks=None):
-    """Block-sparse attention with each dropped block compensated by its (bf16) mean key
-    and value, weighted by its token count.  Returns (o, lse) like `attention`."""
+                          qblocks=None, order: int = 1):
+    """Block-sparse attention with the dropped blocks compensated by the first-order
+    expansion of their exponentials about each block's mean key (order=1: the count-
+    weighted mean value plus the moment term s q^T sum_j (k_j - kbar)v_j^T), or by the
+    mean key and value alone (order=0).  Means in fp64.  Returns (o, lse) like
+    `attention`."""
     q, k, v = _bf16(q), _bf16(k), _bf16(v)
     B, H, Npad, D = q.shape
     vl = _vl(valid_len, B, Npad)
@@ -243,11 +246,20 @@ def attention_compensated(q, k, v, kv_idx, kv_cnt, valid_len=None, scale: float 
     lse = np.full((B, H, Npad), np.nan)
     qb = None if qblocks is None else np.ascontiguousarray(qblocks, dtype=np.int32)
     st = _load().oracle_attention_compensated(_p(q), _p(k), _p(v), B, H, Npad, D, _p(vl), block, _p(kv_idx),
-                                              _p(kv_cnt), kv_idx.shape[3], float(scale), _p(qb),
+                                              _p(kv_cnt), kv_idx.shape[3], float(scale), int(order), _p(qb),
                                               0 if qb is None else len(qb), _p(o), _p(lse))
+    if st == -2:
+        raise ValueError("order must be 0 or 1")
     if st != 0:
         raise ValueError("routing entry outside the sample's blocks")
     return o, lse
+
+
+def attention_mean_compensated(q, k, v, kv_idx, kv_cnt, valid_len=None, scale: float = 0.0, block: int = 64,
+                               qblocks=None):
+    """The zeroth-order form: each dropped block is one softmax entry of logit
+    s q.kbar_J + log c_J carrying vbar_J (fp64 means)."""
+    return attention_compensated(q, k, v, kv_idx, kv_cnt, valid_len, scale, block, qblocks, order=0)
 
 
 def dense(q, k, v, valid_len=None, scale: float = 0.0):

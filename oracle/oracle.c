@@ -502,53 +502,86 @@ int oracle_qk_norm_rope(const uint16_t* x, const uint16_t* w, const int32_t* pos
 
 /* ---------------------------------------------------------------------------
  * Block-sparse attention with compensation of the dropped blocks.  PISA, as the
- * page "Sol Video Inference Engine" (sjmshsh.github.io) describes it in section
- * 4.2.2 (Sparse Attention), computes the critical blocks exactly and compensates
- * the others by a first-order Taylor approximation.  Expanding exp(s q.k_j) about the mean key kbar_J
- * of a dropped block J, the sum over its tokens is c_J exp(s q.kbar_J) to first
- * order (the linear term sums to zero about the mean); the numerator's
- * zeroth-order term is exp(s q.kbar_J) sum_j v_j = c_J exp(s q.kbar_J) vbar_J.
- * So each dropped block enters the softmax as one entry of logit
- * s q.kbar_J + log(c_J) carrying the value vbar_J:
- *   o_i = [sum_{j kept} e^{s q.k_j} v_j + sum_{J dropped} c_J e^{s q.kbar_J} vbar_J]
- *         / [sum_{j kept} e^{s q.k_j} + sum_{J dropped} c_J e^{s q.kbar_J}]
- * with kbar_J, vbar_J the means of the valid tokens of block J (token order,
- * fp64) rounded to bf16, c_J their count; "dropped" = the sample's blocks not in
- * the row's kept list.  Exact when keys are constant within every dropped block.
- * Same arguments and outputs as oracle_attention. */
+ * page "Sol Video Inference Engine" (sjmshsh.github.io) names it in section 4.2.2
+ * (Sparse Attention), computes the critical blocks exactly and compensates the
+ * other blocks by a first-order Taylor approximation.  Reading taken here: for a
+ * dropped block J, each token's exponential is expanded to first order about the
+ * block's mean key kbar_J,
+ *     exp(s q.k_j) ~ exp(s q.kbar_J) * (1 + s q.(k_j - kbar_J)).
+ * Summed over the c_J valid tokens j of J, the linear term vanishes from the
+ * normaliser (the deviations sum to zero about the mean) and leaves in the
+ * numerator the D x D moment
+ *     M_J[d][e] = sum_j (k_j[d] - kbar_J[d]) * v_j[e]:
+ *   Z_i = sum_{j kept} e^{x_ij} + sum_{J dropped} c_J e^{xbar_iJ}
+ *   N_i = sum_{j kept} e^{x_ij} v_j
+ *       + sum_{J dropped} e^{xbar_iJ} (c_J vbar_J + s * sum_d q_i[d] M_J[d][.])
+ *   o_i = N_i / Z_i,   lse_i = log Z_i
+ * with x_ij = s q_i.k_j, xbar_iJ = s q_i.kbar_J, kbar_J and vbar_J the means of the
+ * valid tokens of J in fp64 (token order), and "dropped" the sample's blocks
+ * J < nB_b missing from the row's kept list.  The exponentials are shifted by
+ * m = the largest of the kept x_ij and the dropped xbar_iJ.  The result is exact
+ * when keys are constant within every dropped block, and its error shrinks with
+ * the square of the keys' spread about their block means.
+ *
+ * order = 0 leaves the moment term out: each dropped block is then one softmax
+ * entry of logit xbar_iJ + log c_J carrying vbar_J (the mean-key form, whose error
+ * shrinks only linearly with the spread).
+ *
+ * Same arguments and outputs as oracle_attention, plus `order` (0 or 1).  Works
+ * one (b, h) at a time: the block means and moments of that head, then its rows. */
 int oracle_attention_compensated(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int H,
                                  int Npad, int D, const int32_t* valid_len, int block, const int32_t* kv_idx,
-                                 const int32_t* kv_cnt, int kmax, double scale, const int32_t* qblocks,
+                                 const int32_t* kv_cnt, int kmax, double scale, int order, const int32_t* qblocks,
                                  int n_qblocks, double* o, double* lse) {
     const int nBmax = Npad / block;
     const int nq = qblocks ? n_qblocks : nBmax;
     if (scale <= 0.0) scale = 1.0 / sqrt((double)D);
-    const size_t nm = (size_t)B * H * nBmax * D;
-    double* km = (double*)malloc(sizeof(double) * nm);
-    double* vm = (double*)malloc(sizeof(double) * nm);
-    oracle_pool(k, B, H, Npad, D, valid_len, block, km);
-    oracle_pool(v, B, H, Npad, D, valid_len, block, vm);
-    for (size_t t = 0; t < nm; ++t) {   /* the means, rounded to bf16 */
-        km[t] = bf16_to_f64(bf16_rne(km[t]));
-        vm[t] = bf16_to_f64(bf16_rne(vm[t]));
-    }
+    if (order != 0 && order != 1) return -2;
+    double* km = (double*)malloc(sizeof(double) * (size_t)nBmax * D);
+    double* vm = (double*)malloc(sizeof(double) * (size_t)nBmax * D);
+    double* M = order ? (double*)malloc(sizeof(double) * (size_t)nBmax * D * D) : NULL;
     int status = 0;
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H; ++h) {
+            const int L = valid_len[b], nB = n_blocks_of(L, block);
+            const size_t bh = (size_t)b * H + h;
+            const uint16_t* ks = k + bh * (size_t)Npad * D;
+            const uint16_t* vs = v + bh * (size_t)Npad * D;
+            /* block means of K and V over the valid tokens, and the moments */
+#pragma omp parallel for schedule(dynamic)
+            for (int J = 0; J < nB; ++J) {
+                const int j0 = J * block, j1 = (J + 1) * block < L ? (J + 1) * block : L;
+                const double c = (double)(j1 - j0);
+                for (int d = 0; d < D; ++d) {
+                    double sk = 0.0, sv = 0.0;
+                    for (int j = j0; j < j1; ++j) {
+                        sk += bf16_to_f64(ks[(size_t)j * D + d]);
+                        sv += bf16_to_f64(vs[(size_t)j * D + d]);
+                    }
+                    km[(size_t)J * D + d] = sk / c;
+                    vm[(size_t)J * D + d] = sv / c;
+                }
+                if (order) {
+                    double* MJ = M + (size_t)J * D * D;
+                    for (int d = 0; d < D; ++d)
+                        for (int e = 0; e < D; ++e) {
+                            double s = 0.0;
+                            for (int j = j0; j < j1; ++j)
+                                s += (bf16_to_f64(ks[(size_t)j * D + d]) - km[(size_t)J * D + d]) *
+                                     bf16_to_f64(vs[(size_t)j * D + e]);
+                            MJ[(size_t)d * D + e] = s;
+                        }
+                }
+            }
 #pragma omp parallel
-    {
-        int32_t* tok = (int32_t*)malloc(sizeof(int32_t) * (size_t)Npad);
-        double* lg = (double*)malloc(sizeof(double) * (size_t)(Npad + nBmax));
-        char* kept = (char*)malloc((size_t)(nBmax > 0 ? nBmax : 1));
-#pragma omp for collapse(3) schedule(dynamic)
-        for (int b = 0; b < B; ++b)
-            for (int h = 0; h < H; ++h)
+            {
+                int32_t* tok = (int32_t*)malloc(sizeof(int32_t) * (size_t)Npad);
+                double* lg = (double*)malloc(sizeof(double) * (size_t)(Npad + nBmax));
+                double* qm = (double*)malloc(sizeof(double) * (size_t)D);
+                char* kept = (char*)malloc((size_t)(nBmax > 0 ? nBmax : 1));
+#pragma omp for schedule(dynamic)
                 for (int qi = 0; qi < nq; ++qi) {
                     const int I = qblocks ? qblocks[qi] : qi;
-                    const int L = valid_len[b], nB = n_blocks_of(L, block);
-                    const size_t bh = (size_t)b * H + h;
-                    const uint16_t* ks = k + bh * (size_t)Npad * D;
-                    const uint16_t* vs = v + bh * (size_t)Npad * D;
-                    const double* kmb = km + bh * (size_t)nBmax * D;
-                    const double* vmb = vm + bh * (size_t)nBmax * D;
                     const size_t r = bh * nBmax + I;
                     int n = kept_tokens(kv_idx + r * kmax, kv_cnt[r], nB, L, block, tok);
                     if (n < 0) {
@@ -568,7 +601,7 @@ int oracle_attention_compensated(const uint16_t* q, const uint16_t* k, const uin
                             continue;
                         }
                         const uint16_t* qr = q + (bh * Npad + i) * D;
-                        /* logits: kept tokens, then one entry per dropped block */
+                        /* exponents: the kept tokens, then one per dropped block */
                         double m = -INFINITY;
                         int ne = 0;
                         for (int t = 0; t < n; ++t) {
@@ -581,11 +614,9 @@ int oracle_attention_compensated(const uint16_t* q, const uint16_t* k, const uin
                         }
                         for (int J = 0; J < nB; ++J) {
                             if (kept[J]) continue;
-                            int c = L - J * block;
-                            c = c > block ? block : c;
                             double s = 0.0;
-                            for (int d = 0; d < D; ++d) s += bf16_to_f64(qr[d]) * kmb[(size_t)J * D + d];
-                            lg[ne] = scale * s + log((double)c);
+                            for (int d = 0; d < D; ++d) s += bf16_to_f64(qr[d]) * km[(size_t)J * D + d];
+                            lg[ne] = scale * s;
                             if (lg[ne] > m) m = lg[ne];
                             ++ne;
                         }
@@ -594,26 +625,42 @@ int oracle_attention_compensated(const uint16_t* q, const uint16_t* k, const uin
                             continue;
                         }
                         double Z = 0.0;
-                        for (int e = 0; e < ne; ++e) { lg[e] = exp(lg[e] - m); Z += lg[e]; }
                         int e = 0;
                         for (int t = 0; t < n; ++t, ++e) {
+                            const double w = exp(lg[e] - m);
                             const uint16_t* vr = vs + (size_t)tok[t] * D;
-                            const double w = lg[e] / Z;
+                            Z += w;
                             for (int d = 0; d < D; ++d) orow[d] += w * bf16_to_f64(vr[d]);
                         }
                         for (int J = 0; J < nB; ++J) {
                             if (kept[J]) continue;
-                            const double w = lg[e++] / Z;
-                            for (int d = 0; d < D; ++d) orow[d] += w * vmb[(size_t)J * D + d];
+                            const int c = (L - J * block) < block ? (L - J * block) : block;
+                            const double w = exp(lg[e++] - m);
+                            Z += (double)c * w;
+                            for (int d = 0; d < D; ++d) orow[d] += w * (double)c * vm[(size_t)J * D + d];
+                            if (order) {
+                                /* s * q^T M_J, weighted like the block */
+                                const double* MJ = M + (size_t)J * D * D;
+                                for (int d = 0; d < D; ++d) qm[d] = 0.0;
+                                for (int dd = 0; dd < D; ++dd) {
+                                    const double qd = bf16_to_f64(qr[dd]);
+                                    for (int d = 0; d < D; ++d) qm[d] += qd * MJ[(size_t)dd * D + d];
+                                }
+                                for (int d = 0; d < D; ++d) orow[d] += w * scale * qm[d];
+                            }
                         }
+                        for (int d = 0; d < D; ++d) orow[d] /= Z;
                         *l = m + log(Z);
                     }
                 }
-        free(tok);
-        free(lg);
-        free(kept);
-    }
+                free(tok);
+                free(lg);
+                free(qm);
+                free(kept);
+            }
+        }
     free(km);
     free(vm);
+    free(M);
     return status;
 }
