@@ -63,6 +63,10 @@ def _load():
                                           f64, vp, i32, vp, vp]
         _lib.oracle_dense.restype = None
         _lib.oracle_dense.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, f64, vp, vp]
+        _lib.oracle_keep_tokens.restype = i32
+        _lib.oracle_keep_tokens.argtypes = [i32, f64]
+        _lib.oracle_token_prune.restype = i32
+        _lib.oracle_token_prune.argtypes = [vp, i32, i32, i32, vp, f64, i32, vp, vp, vp]
         _lib.oracle_probs.restype = i32
         _lib.oracle_probs.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, i32, vp, vp, i32, f64,
                                       i32, i32, i32, vp]
@@ -286,3 +290,31 @@ def probs(q, k, v, kv_idx, kv_cnt, b, h, i, valid_len=None, scale: float = 0.0, 
     if st != 0:
         raise ValueError("routing entry outside the sample's blocks")
     return p
+
+
+def keep_tokens(n_tokens: int, ratio: float) -> int:
+    """Tokens kept by saliency pruning: clamp(ceil(ratio * n - 1e-9), 1, n)."""
+    return int(_load().oracle_keep_tokens(int(n_tokens), float(ratio)))
+
+
+def token_prune(x, valid_len=None, ratio: float = 0.5, npad_out: int | None = None):
+    """Token pruning by feature-norm saliency (page "Sol Video Inference Engine", LTX-2.3
+    appendix, stage 2: keep 50% of the video tokens by feat_norm).  x: bf16 bits
+    [B, N, C].  Keeps the keep_tokens(L_b, ratio) tokens of largest squared norm
+    (channel-order fp64 sum), ties to the lower index, in their original order.
+    Returns (idx int32 [B, npad_out] ascending then -1, valid_out int32 [B],
+    norm2 fp64 [B, N])."""
+    x = np.ascontiguousarray(x)
+    assert x.dtype == np.uint16 and x.ndim == 3, "bf16 bit patterns [B, N, C] expected"
+    B, N, C = x.shape
+    vl = np.full(B, N, dtype=np.int32) if valid_len is None else np.ascontiguousarray(valid_len, dtype=np.int32)
+    if npad_out is None:
+        npad_out = max(keep_tokens(int(L), ratio) for L in vl)
+    idx = np.empty((B, npad_out), dtype=np.int32)
+    vout = np.empty(B, dtype=np.int32)
+    norm2 = np.empty((B, N))
+    st = _load().oracle_token_prune(_p(x), B, N, C, _p(vl), float(ratio), int(npad_out), _p(norm2), _p(idx),
+                                    _p(vout))
+    if st != 0:
+        raise ValueError("npad_out smaller than a kept count")
+    return idx, vout, norm2

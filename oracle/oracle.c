@@ -664,3 +664,65 @@ int oracle_attention_compensated(const uint16_t* q, const uint16_t* k, const uin
     free(M);
     return status;
 }
+
+/* ---------------------------------------------------------------------------
+ * Token pruning by feature-norm saliency.  The page "Sol Video Inference Engine"
+ * (sjmshsh.github.io), LTX-2.3 appendix, stage 2, keeps 50% of the video tokens by
+ * feat_norm saliency before the refinement transformer's first two calls.  Reading
+ * taken here: the saliency of token n of sample b is the Euclidean norm of its
+ * feature vector x[b][n][0..C); the kept tokens are the keep_tokens(L_b, ratio)
+ * most salient of the sample's L_b valid tokens, equal norms going to the lower
+ * token index, and they keep their original (raster) order, compacted to the front.
+ * The norm is ranked through its square, sum_c x_c^2 summed in channel order in
+ * fp64 (every square of a bf16 value is exact in fp64).
+ *
+ * keep_tokens(L, r) = clamp(ceil(r * L - 1e-9), 1, L) in fp64; 0 when L <= 0. */
+int32_t oracle_keep_tokens(int32_t n, double ratio) {
+    if (n <= 0) return 0;
+    double x = ceil(ratio * (double)n - 1e-9);
+    if (x < 1.0) x = 1.0;
+    if (x > (double)n) x = (double)n;
+    return (int32_t)x;
+}
+
+/* x: bf16 [B, N, C]; valid_len[b] <= N.  Writes norm2 [B, N] (0 past L_b),
+ * idx [B, Npad_out] (kept token indices ascending, then -1) and valid_out [B].
+ * Returns 0, or -1 when a kept count exceeds Npad_out. */
+int oracle_token_prune(const uint16_t* x, int B, int N, int C, const int32_t* valid_len, double ratio,
+                       int Npad_out, double* norm2, int32_t* idx, int32_t* valid_out) {
+    int status = 0;
+    for (int b = 0; b < B; ++b) {
+        const int L = valid_len[b];
+        double* nb = norm2 + (size_t)b * N;
+#pragma omp parallel for schedule(static)
+        for (int n = 0; n < N; ++n) {
+            double s = 0.0;
+            if (n < L) {
+                const uint16_t* row = x + ((size_t)b * N + n) * C;
+                for (int c = 0; c < C; ++c) {
+                    const double v = bf16_to_f64(row[c]);
+                    s += v * v;
+                }
+            }
+            nb[n] = s;
+        }
+        const int k = oracle_keep_tokens(L, ratio);
+        int32_t* ib = idx + (size_t)b * Npad_out;
+        for (int p = 0; p < Npad_out; ++p) ib[p] = -1;
+        valid_out[b] = k;
+        if (k > Npad_out) {
+            status = -1;
+            continue;
+        }
+        scored_block* row = (scored_block*)malloc(sizeof(scored_block) * (size_t)(L > 0 ? L : 1));
+        for (int n = 0; n < L; ++n) {
+            row[n].score = nb[n];
+            row[n].index = n;
+        }
+        qsort(row, (size_t)L, sizeof(scored_block), by_score_desc_index_asc);
+        for (int t = 0; t < k; ++t) ib[t] = row[t].index;
+        qsort(ib, (size_t)k, sizeof(int32_t), int_asc);
+        free(row);
+    }
+    return status;
+}
