@@ -65,10 +65,18 @@ typedef enum {
 /* Largest padded sequence length a call accepts (4096 blocks of 64 tokens). */
 #define SBA_MAX_NPAD 262144
 
-/* Kept key blocks per query block for n_blocks candidate blocks at sparsity s:
+/* Kept key blocks per query block for n_blocks candidate blocks at sparsity s
+ * (same page and section: `sparsity` is the fraction of key blocks dropped):
  * clamp(ceil((1 - s) * n_blocks - 1e-9), 1, n_blocks), evaluated in fp64; 0 when
  * n_blocks <= 0.  Pure host function. */
 int32_t sba_keep_count(int32_t n_blocks, double sparsity);
+
+/* The kept count of the sub-block router with its block budget (same page and
+ * section, which rounds the kept count to an 8-block budget without giving the rule):
+ * sba_keep_count(n_blocks, sparsity) rounded up to a multiple of `budget`, at most
+ * n_blocks.  budget = 1 gives sba_keep_count; budget < 1 returns 0.  Pure host
+ * function. */
+int32_t sba_keep_count_budget(int32_t n_blocks, double sparsity, int32_t budget);
 
 /* Bytes of device workspace sba_pool_select needs for this shape (0 on bad
  * arguments).  The workspace holds the pooled Q and K block means. */
@@ -165,30 +173,52 @@ sba_status sba_pool_select_means(const double* qmean, const double* kmean, int B
                                  int kmax, int32_t* kv_idx, int32_t* kv_cnt, void* workspace,
                                  size_t workspace_bytes, void* stream);
 
-/* Bytes of device workspace sba_attention_compensated needs (0 on bad arguments):
- * the bf16 block means of K and V. */
-size_t sba_compensation_workspace_size(int B, int H, int Npad, int D, int block);
-
 /* Block-sparse attention with compensation of the dropped blocks.  PISA, as the page
- * "Sol Video Inference Engine" (sjmshsh.github.io), section 4.2.2, describes it,
- * computes the critical blocks exactly and compensates the others by a first-order
- * Taylor approximation; about a dropped block's mean key the expansion gives the
- * block one softmax entry (the normaliser's linear term sums to zero):
- *   o_i = [sum_{j kept} e^{s q.k_j} v_j + sum_{J dropped} c_J e^{s q.kbar_J} vbar_J]
- *         / [sum_{j kept} e^{s q.k_j} + sum_{J dropped} c_J e^{s q.kbar_J}]
+ * "Sol Video Inference Engine" (sjmshsh.github.io), section 4.2.2 (Sparse Attention),
+ * describes it, computes the critical blocks exactly and compensates the others by a
+ * first-order Taylor approximation.  Each dropped block J's exponentials are expanded
+ * to first order about its mean key:
+ *   e^{s q.k_j} ~ e^{s q.kbar_J} (1 + s q.(k_j - kbar_J))   for the valid tokens j of J
+ * so that, with x_j = s q.k_j and xbar_J = s q.kbar_J,
+ *   o_i = [sum_{j kept} e^{x_j} v_j
+ *          + sum_{J dropped} e^{xbar_J} (c_J vbar_J + s q_i^T sum_{j in J} (k_j - kbar_J) v_j^T)]
+ *         / [sum_{j kept} e^{x_j} + sum_{J dropped} c_J e^{xbar_J}]
  *   lse_i = log of the denominator
  * where "dropped" are the sample's blocks J < nB_b missing from the row's kept list,
- * kbar_J / vbar_J are the means of the valid tokens of block J (fp64 sums, rounded
- * to bf16) and c_J their count.  Exact when keys are constant within each dropped
- * block.  Arguments as sba_attention_paired (pair_order may be NULL for adjacent
- * tiles), plus a workspace of at least sba_compensation_workspace_size bytes
- * (16-byte aligned; contents on entry ignored).  Cost: the kept blocks plus
- * ceil(nB/64) further 64-column steps per tile. */
+ * kbar_J / vbar_J the means of the valid tokens of J and c_J their count.  Exact when
+ * keys are constant within each dropped block; the error shrinks as the square of the
+ * keys' spread about their block means.
+ * The kernel evaluates the expansion token by token (the weight of token j of a
+ * dropped block is e^{xbar_J} (1 + x_j - xbar_J), xbar_J being the mean of the block's
+ * logits), so it walks every block of the sample: the cost is that of dense attention,
+ * with one exponential per dropped block instead of one per token.
+ * Arguments as sba_attention_paired (pair_order may be NULL for adjacent tiles); no
+ * workspace. */
 sba_status sba_attention_compensated(const void* q, const void* k, const void* v, void* o, float* lse,
                                      int B, int H, int Npad, int D, const int32_t* valid_len, int block,
                                      const int32_t* kv_idx, const int32_t* kv_cnt, int kmax,
-                                     const int32_t* pair_order, float softmax_scale, void* workspace,
-                                     size_t workspace_bytes, void* stream);
+                                     const int32_t* pair_order, float softmax_scale, void* stream);
+
+/* Bytes of device workspace sba_attention_mean_compensated needs (0 on bad
+ * arguments): the bf16 block means of K and V. */
+size_t sba_mean_compensation_workspace_size(int B, int H, int Npad, int D, int block);
+
+/* The cheaper, zeroth-order compensation: the expansion above without its moment
+ * term, so each dropped block enters the softmax as one entry of logit
+ * s q.kbar_J + log(c_J) carrying vbar_J:
+ *   o_i = [sum_{j kept} e^{x_j} v_j + sum_{J dropped} c_J e^{xbar_J} vbar_J]
+ *         / [sum_{j kept} e^{x_j} + sum_{J dropped} c_J e^{xbar_J}]
+ * Its error shrinks only linearly with the keys' spread.  The means are formed in
+ * fp64 and stored in bf16 (2^-9 relative), which moves each dropped block's logit by
+ * at most s sum_d |q_d kbar_d| 2^-9.  Arguments as sba_attention_compensated, plus a
+ * workspace of at least sba_mean_compensation_workspace_size bytes (16-byte aligned;
+ * contents on entry ignored).  Cost: the kept blocks plus ceil(nB/64) further
+ * 64-column steps per tile. */
+sba_status sba_attention_mean_compensated(const void* q, const void* k, const void* v, void* o, float* lse,
+                                          int B, int H, int Npad, int D, const int32_t* valid_len, int block,
+                                          const int32_t* kv_idx, const int32_t* kv_cnt, int kmax,
+                                          const int32_t* pair_order, float softmax_scale, void* workspace,
+                                          size_t workspace_bytes, void* stream);
 
 /* Block means of x as fp64 values [B, H, Npad/block, D] (inspection helper;
  * blocks past nB_b are written as 0).  `out` is device memory. */
@@ -254,6 +284,48 @@ sba_status sba_attention_to_shards(const void* q, const void* k, const void* v, 
                                    const int32_t* kv_idx, const int32_t* kv_cnt, int kmax,
                                    const int32_t* pair_order, float softmax_scale, void* stream);
 
+/* Token pruning by feature-norm saliency, the producer of a ragged, pruned sequence.
+ * The page "Sol Video Inference Engine" (sjmshsh.github.io), LTX-2.3 appendix, stage
+ * 2, keeps 50% of the video tokens by feat_norm saliency.  Per sample b, with L_b
+ * valid tokens:
+ *   saliency(n) = |x[b][n]|^2 = sum_c x[b][n][c]^2, summed in channel order in fp64
+ *                 (every square of a bf16 value is exact)
+ *   kept = the keep_tokens(L_b, keep_ratio) tokens of largest saliency, equal values
+ *          going to the lower index, listed in their original (raster) order
+ *   keep_tokens(L, r) = clamp(ceil(r * L - 1e-9), 1, L), fp64 (sba_keep_token_count).
+ *   x            bf16 [B, N, C] token features, C a multiple of 8 (else UNSUPPORTED),
+ *                16-byte aligned
+ *   valid_len    int32 [B] device (1 <= valid_len[b] <= N), or NULL (all N valid)
+ *   keep_ratio   in [0, 1]
+ *   Npad_out     row length of idx; must be >= keep_tokens(N, keep_ratio)
+ *   idx          int32 [B, Npad_out] (written): the kept token indices ascending,
+ *                then -1
+ *   valid_len_out int32 [B] (written): the kept counts (a valid_len for the pruned
+ *                sequence)
+ *   workspace    device buffer of sba_token_prune_workspace_size bytes, 16-byte
+ *                aligned; on return its first B * N fp64 values are the saliencies
+ *                (0 for padding tokens)
+ * HBM-bound: x is read once. */
+int32_t sba_keep_token_count(int32_t n_tokens, double keep_ratio);
+size_t sba_token_prune_workspace_size(int B, int N);
+sba_status sba_token_prune_select(const void* x, int B, int N, int C, const int32_t* valid_len,
+                                  double keep_ratio, int Npad_out, int32_t* idx, int32_t* valid_len_out,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* The pruned sequence's rows: dst[b][h][p] = src[b][h][idx[b][p]] for
+ * p < valid_len_out[b], zero rows for the rest of [0, Npad_out).  Companion of
+ * sba_token_prune_select for the per-token tensors that follow the pruning (Q, K, V
+ * [B, H, N, D], positions [B, N, 3] with H = 1, ...).
+ *   src          [B, H, N] rows of row_bytes bytes (row_bytes a multiple of 4, else
+ *                UNSUPPORTED); 16-byte aligned when row_bytes is a multiple of 16,
+ *                else 4-byte aligned (dst likewise)
+ *   idx, valid_len_out, Npad_out  as written by sba_token_prune_select (an index
+ *                outside [0, N) raises SBA_ERR_DEVICE_FLAG and copies row 0)
+ *   dst          [B, H, Npad_out] rows (written, every row)
+ * HBM-bound row copy. */
+sba_status sba_gather_tokens(const void* src, int B, int H, int N, int row_bytes, const int32_t* idx,
+                             const int32_t* valid_len_out, int Npad_out, void* dst, void* stream);
+
 /* Dense attention over all valid tokens of each sample (the sparsity = 0 case
  * without a routing), same layouts as sba_attention. */
 sba_status sba_dense_attention(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -279,6 +351,9 @@ void sba_set_wait_limit(uint64_t cycles);
  *                                (tcgen05 MMAs of M = 256 across the pair, 128 keys per
  *                                step), walking the union of their four lists;
  *                                pair_order is not used;
+ *   SBA_ATTN_KERNEL_KEY_PAIRS    the query pairs of SBA_ATTN_KERNEL_QUERY_PAIRS, walking
+ *                                their union two key blocks (128 keys) per step, which
+ *                                halves the shared-memory reads of Q per key;
  *   SBA_ATTN_KERNEL_AUTO         (default) the query pairs, the faster of the two on
  *                                every workload measured on B200.
  * Outputs agree up to floating-point accumulation order.  Process-wide; returns
@@ -286,6 +361,7 @@ void sba_set_wait_limit(uint64_t cycles);
 #define SBA_ATTN_KERNEL_AUTO 0
 #define SBA_ATTN_KERNEL_QUERY_PAIRS 1
 #define SBA_ATTN_KERNEL_CTA_PAIR 2
+#define SBA_ATTN_KERNEL_KEY_PAIRS 3
 sba_status sba_set_attention_kernel(int which);
 
 /* Routing for callers that cannot allocate device memory.
@@ -306,7 +382,8 @@ sba_status sba_set_attention_kernel(int which);
  *     calls no allocating library routine.
  *   - The first call on a device looks up the array's device address (once per
  *     device, under a lock) with cudaGetSymbolAddress; make that first call
- *     before any stream capture.
+ *     before any stream capture.  The address is kept for the life of the process,
+ *     so do not call this entry point on a device after cudaDeviceReset there.
  *   - All calls on a device share the one array and it keeps whatever the last
  *     call left in it.  That is harmless here, since every value a call reads
  *     from it was written earlier in the same call, so nothing has to start at

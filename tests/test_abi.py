@@ -175,14 +175,35 @@ def test_pool_select_means_rejects(lib):
 
 
 def test_compensated_rejects(lib):
-    f = lambda q=A, v=A, idx=A, cnt=A, kmax=8, D=128, ws=A, wsb=1 << 30, po=NULL: lib.sba_attention_compensated(
-        q, A, v, A, A, 1, 2, 1024, D, NULL, 64, idx, cnt, kmax, po, 0.0, ws, wsb, S)
-    assert lib.sba_compensation_workspace_size(1, 2, 1024, 128, 64) > 0
-    assert lib.sba_compensation_workspace_size(1, 2, 1000, 128, 64) == 0
+    f = lambda q=A, v=A, idx=A, cnt=A, kmax=8, D=128, po=NULL: lib.sba_attention_compensated(
+        q, A, v, A, A, 1, 2, 1024, D, NULL, 64, idx, cnt, kmax, po, 0.0, S)
+    assert f(q=NULL) == 1 and f(v=NULL) == 1 and f(idx=NULL) == 1 and f(cnt=NULL) == 1
+    assert f(kmax=0) == 1
+    assert f(D=96) == 2
+    assert f(q=MIS) == 3 and f(po=ctypes.c_void_p(0x10002)) == 3
+
+
+def test_mean_compensated_rejects(lib):
+    f = lambda q=A, v=A, idx=A, cnt=A, kmax=8, D=128, ws=A, wsb=1 << 30, po=NULL: \
+        lib.sba_attention_mean_compensated(q, A, v, A, A, 1, 2, 1024, D, NULL, 64, idx, cnt, kmax, po, 0.0, ws, wsb,
+                                           S)
+    assert lib.sba_mean_compensation_workspace_size(1, 2, 1024, 128, 64) > 0
+    assert lib.sba_mean_compensation_workspace_size(1, 2, 1000, 128, 64) == 0
     assert f(q=NULL) == 1 and f(v=NULL) == 1 and f(idx=NULL) == 1 and f(cnt=NULL) == 1
     assert f(ws=NULL) == 1 and f(wsb=16) == 1 and f(kmax=0) == 1
     assert f(D=96) == 2
     assert f(ws=MIS) == 3 and f(po=ctypes.c_void_p(0x10002)) == 3
+
+
+def test_keep_count_budget_export(lib):
+    """The budget rule is the library's: the binding only forwards to it."""
+    import video_dit_block_b200 as sba
+    assert lib.sba_keep_count_budget(1182, 0.8, 1) == lib.sba_keep_count(1182, 0.8) == 237
+    assert lib.sba_keep_count_budget(1182, 0.8, 8) == 240
+    assert lib.sba_keep_count_budget(10, 0.05, 8) == 10        # capped at n
+    assert lib.sba_keep_count_budget(10, 0.5, 0) == 0          # budget < 1
+    assert lib.sba_keep_count_budget(0, 0.5, 8) == 0
+    assert sba.keep_count_budget(1182, 0.8, 8) == 240
 
 
 def test_attention_to_shards_rejects(lib):
@@ -208,3 +229,28 @@ def test_set_attention_kernel_values(lib):
         assert lib.sba_set_attention_kernel(which) == 0
     assert lib.sba_set_attention_kernel(3) == 1 and lib.sba_set_attention_kernel(-1) == 1
     assert lib.sba_set_attention_kernel(0) == 0        # back to the default
+
+
+def test_token_prune_rejects(lib):
+    assert lib.sba_keep_token_count(63240, 0.5) == 31620
+    assert lib.sba_keep_token_count(10, 1.5) == 0
+    assert lib.sba_token_prune_workspace_size(2, 63240) >= 2 * 63240 * 8
+    assert lib.sba_token_prune_workspace_size(0, 5) == 0
+    f = lambda x=A, N=1000, C=64, r=0.5, npo=512, idx=A, vo=A, ws=A, wsb=1 << 20: lib.sba_token_prune_select(
+        x, 2, N, C, NULL, r, npo, idx, vo, ws, wsb, S)
+    assert f(x=NULL) == 1 and f(idx=NULL) == 1 and f(vo=NULL) == 1 and f(ws=NULL) == 1
+    assert f(r=1.5) == 1 and f(r=-0.1) == 1
+    assert f(npo=499) == 1                       # keep_tokens(1000, 0.5) = 500
+    assert f(wsb=1000) == 1
+    assert f(C=60) == 2                          # C % 8 != 0
+    assert f(x=MIS) == 3 and f(ws=MIS) == 3 and f(idx=ctypes.c_void_p(0x10002)) == 3
+
+
+def test_gather_tokens_rejects(lib):
+    f = lambda src=A, rb=256, idx=A, vo=A, dst=A, npo=64: lib.sba_gather_tokens(src, 2, 4, 1000, rb, idx, vo, npo,
+                                                                                 dst, S)
+    assert f(src=NULL) == 1 and f(dst=NULL) == 1 and f(idx=NULL) == 1 and f(vo=NULL) == 1
+    assert f(rb=0) == 1 and f(npo=0) == 1
+    assert f(rb=6) == 2                          # not a multiple of 4
+    assert f(src=MIS) == 3 and f(dst=MIS) == 3   # 16-byte units for 256-byte rows
+    assert f(rb=12, src=ctypes.c_void_p(0x10002)) == 3

@@ -57,3 +57,8 @@ def test_our_arm_line():
     assert isinstance(d["gpu_launches"], int) and d["gpu_launches"] > 0
     c = d["clocks"]
     assert "sm_mhz" in c and "sm_max_mhz" in c and isinstance(c["reasons"], list)
+    p = d["parity"]
+    assert p["mask_rows"] > 0 and p["mask_mismatch"] == 0 and p["ok"] is True
+    assert p["max_abs"] <= 2e-2 and p["mean_abs"] <= 2e-3 and p["out_rows"] > 0
+    m = d["median_ms"]
+    assert m["step"] > 0 and m["attn"] > 0 and m["select"] > 0

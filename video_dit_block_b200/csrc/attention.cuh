@@ -32,13 +32,26 @@
 // Every wait is bounded: on expiry the CTA records SBA_ERR_TIMEOUT, unwinds all
 // roles, drains its own TMA loads and MMAs and frees its TMEM.
 //
-// COMP = true adds the compensation of the dropped blocks (the first-order
-// expansion of their exponentials about their mean key): after the union walk, the
-// tile walks the rows of kbar / vbar (the bf16 block means, [BH][nBpad][D]) as
-// further 64-column steps, column c of step b standing for block J = 64 b + c with
-// logit s q.kbar_J + log(c_J); a column is masked for a half whose query block
-// keeps J, and past the sample's blocks.  The online softmax then merges the two
-// parts exactly as it merges key blocks.
+// MODE selects what the dropped key blocks contribute (the compensation of the
+// dropped blocks; page "Sol Video Inference Engine", section 4.2.2: PISA computes the
+// critical blocks exactly and compensates the others by a first-order Taylor
+// approximation):
+//   kPlain      nothing: the kept blocks only.
+//   kMeanComp   each dropped block as one softmax entry: after the union walk, the
+//               tile walks the rows of kbar / vbar (the bf16 block means,
+//               [BH][nBpad][D]) as further 64-column steps, column c of step b
+//               standing for block J = 64 b + c with logit s q.kbar_J + log(c_J); a
+//               column is masked for a half whose query block keeps J, and past the
+//               sample's blocks.  The online softmax merges the two parts exactly as
+//               it merges key blocks.
+//   kFirstOrder the first-order expansion of every dropped block's exponentials about
+//               its mean key: the tile walks all blocks of the sample; a block the
+//               half keeps gets weights e^{x_j}, a dropped one the tangent line
+//               e^{xbar} (1 + x_j - xbar), where x_j = s q.k_j and xbar = s q.kbar_J is
+//               the mean of the block's logits over its valid tokens, and adds
+//               c_J e^{xbar} to the normaliser.  Summed over the block this is
+//               e^{xbar} (c_J vbar_J + s q^T sum_j (k_j - kbar_J) v_j^T): the
+//               zeroth- and first-order terms, with no D x D moment ever formed.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -47,6 +60,8 @@
 #include "common.cuh"
 
 namespace sba {
+
+enum AttnMode : int { kPlain = 0, kMeanComp = 1, kFirstOrder = 2 };
 
 constexpr int kMaxBlocks = 4096;  // SBA_MAX_NPAD / 64
 constexpr int kMaxShards = 8;
@@ -111,7 +126,7 @@ __device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, uint64
 
 // The body of both kernels below; the tensor maps are the kernels' own __grid_constant__
 // parameters, passed by address (the plain kernel keeps its three-map signature).
-template <int D, int NS, bool COMP>
+template <int D, int NS, int MODE>
 __device__ __forceinline__ void attn_body(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                                           const CUtensorMap& tmKb, const CUtensorMap& tmVb, const AttnParams& p) {
     using SM = AttnSmem<D, NS>;
@@ -207,7 +222,12 @@ __device__ __forceinline__ void attn_body(const CUtensorMap& tmQ, const CUtensor
         int base = 0;
         for (int w0 = 0; w0 < W; w0 += 32) {
             const int w = w0 + lane;
-            const uint32_t u = w < W ? (bm[w] | bm[kMaxBlocks / 32 + w]) : 0u;
+            uint32_t u = w < W ? (bm[w] | bm[kMaxBlocks / 32 + w]) : 0u;
+            if (MODE == kFirstOrder) {
+                // every block of the sample: kept ones exactly, dropped ones by the expansion
+                const bool any = (qb[0] >= 0 && qb[0] < nB) || (qb[1] >= 0 && qb[1] < nB);
+                u = (w < W && any) ? ((w * 32 + 32 <= nB) ? 0xffffffffu : ((1u << (nB - w * 32)) - 1u)) : 0u;
+            }
             const int c = __popc(u);
             int incl = c;
 #pragma unroll
@@ -234,7 +254,7 @@ __device__ __forceinline__ void attn_body(const CUtensorMap& tmQ, const CUtensor
     // with compensation, the block-mean steps follow the union (none for a tile whose
     // two slots both lie past the sample)
     const bool any_slot = (qb[0] >= 0 && qb[0] < nB) || (qb[1] >= 0 && qb[1] < nB);
-    const int n_all = COMP && any_slot ? n + (nB + 63) / 64 : n;
+    const int n_all = MODE == kMeanComp && any_slot ? n + (nB + 63) / 64 : n;
     const uint64_t lim = p.wait_limit;
     int issued_k = 0, issued_v = 0;  // K / V blocks whose loads the producer has issued
 
@@ -257,7 +277,7 @@ __device__ __forceinline__ void attn_body(const CUtensorMap& tmQ, const CUtensor
                 if (j < n_all) {
                     const int st = j % NS;
                     if (j >= NS && !wait_bounded(bar_ke(st), ((j / NS) - 1) & 1, abort_flag, lim)) break;
-                    const bool mean_step = COMP && j >= n;
+                    const bool mean_step = MODE == kMeanComp && j >= n;
                     const int row = mean_step ? (j - n) * 64 : ulist[j] * 64;
                     mbar_arrive_expect_tx(bar_kf(st), SM::kKVBytes);
                     for (int c = 0; c < NCH; ++c)
@@ -268,7 +288,7 @@ __device__ __forceinline__ void attn_body(const CUtensorMap& tmQ, const CUtensor
                 if (j >= 1) {
                     const int jv = j - 1, st = jv % NS;
                     if (jv >= NS && !wait_bounded(bar_ve(st), ((jv / NS) - 1) & 1, abort_flag, lim)) break;
-                    const bool mean_step = COMP && jv >= n;
+                    const bool mean_step = MODE == kMeanComp && jv >= n;
                     const int row = mean_step ? (jv - n) * 64 : ulist[jv] * 64;
                     mbar_arrive_expect_tx(bar_vf(st), SM::kKVBytes);
                     for (int c = 0; c < NCH; ++c)
@@ -342,20 +362,21 @@ __device__ __forceinline__ void attn_body(const CUtensorMap& tmQ, const CUtensor
         const float sc = p.scale_log2;
         float m = -INFINITY, l = 0.f;
         bool ok = true;
+        const bool half_ok = qb[half] >= 0 && qb[half] < nB;
         for (int j = 0; j < n_all; ++j) {
-            bool kept;                 // this half has weight in the step (uniform over the warp)
+            bool kept;                 // exponential weights for this half (uniform over the warp)
+            bool tangent = false;      // first-order weights of a dropped block (kFirstOrder)
             int ncol;
             uint64_t cmask = ~0ull;    // mean steps: the columns that carry weight for this half
             float off_full = 0.f, off_last = 0.f;
             int last_col = -1;
-            if (COMP && j >= n) {
+            if (MODE == kMeanComp && j >= n) {
                 // columns 0..63 stand for blocks J = 64 pb + c: the half's dropped blocks
                 // of the sample, each with logit offset log2(c_J) (folded in as / sc)
                 const int pb = j - n;
                 const uint64_t kb = (uint64_t)bmh[2 * pb] | ((uint64_t)bmh[2 * pb + 1] << 32);
                 const int nv = nB - 64 * pb;
                 const uint64_t inb = nv >= 64 ? ~0ull : ((1ull << nv) - 1ull);
-                const bool half_ok = qb[half] >= 0 && qb[half] < nB;
                 cmask = half_ok ? (~kb & inb) : 0ull;
                 kept = cmask != 0ull;
                 ncol = 64;
@@ -367,13 +388,14 @@ __device__ __forceinline__ void attn_body(const CUtensorMap& tmQ, const CUtensor
             } else {
                 const int J = ulist[j];
                 kept = (bmh[J >> 5] >> (J & 31)) & 1u;
-                ncol = kept ? L - J * 64 : 0;
+                tangent = MODE == kFirstOrder && !kept && half_ok;
+                ncol = (kept || tangent) ? L - J * 64 : 0;
                 ncol = ncol > 64 ? 64 : ncol;
             }
             if (!warp_wait_bounded(bar_sf(j & 1), (j >> 1) & 1, abort_flag, lim)) { ok = false; break; }
             tc_fence_after();
             const uint32_t sbuf = tl + (j & 1) * 64;
-            if (!kept) {
+            if (!kept && !tangent) {
                 // the other query block of the tile keeps this key block: P = 0 for these rows
                 uint32_t z[32];
 #pragma unroll
@@ -396,25 +418,39 @@ __device__ __forceinline__ void attn_body(const CUtensorMap& tmQ, const CUtensor
                     x[32 + i] = __uint_as_float(c[i]);
                 }
             }
-            if (ncol < 64) {  // ragged tail block of the sample
+            float m_step;              // this step's largest exponent (log2 units)
+            float xbar = 0.f;          // tangent: mean logit of the block's valid tokens (q.k units)
+            if (MODE == kFirstOrder && tangent) {
+                uint64_t s2 = pack2(0.f, 0.f);
 #pragma unroll
-                for (int i = 0; i < 64; ++i) x[i] = i < ncol ? x[i] : -INFINITY;
-            }
-            if constexpr (COMP) {
-                if (j >= n) {
+                for (int i = 0; i < 32; ++i)
+                    s2 = fadd2(s2, pack2(2 * i < ncol ? x[2 * i] : 0.f, 2 * i + 1 < ncol ? x[2 * i + 1] : 0.f));
+                float s0, s1;
+                unpack2(s2, s0, s1);
+                xbar = (s0 + s1) / (float)ncol;
+                m_step = xbar * sc;
+            } else {
+                if (ncol < 64) {  // ragged tail block of the sample
 #pragma unroll
-                    for (int i = 0; i < 64; ++i)
-                        x[i] = ((cmask >> i) & 1ull) ? x[i] + (i == last_col ? off_last : off_full) : -INFINITY;
+                    for (int i = 0; i < 64; ++i) x[i] = i < ncol ? x[i] : -INFINITY;
                 }
-            }
-            float mx0 = x[0], mx1 = x[1];
+                if constexpr (MODE == kMeanComp) {
+                    if (j >= n) {
 #pragma unroll
-            for (int i = 2; i < 62; i += 4) {
-                mx0 = fmax3(mx0, x[i], x[i + 1]);
-                mx1 = fmax3(mx1, x[i + 2], x[i + 3]);
+                        for (int i = 0; i < 64; ++i)
+                            x[i] = ((cmask >> i) & 1ull) ? x[i] + (i == last_col ? off_last : off_full) : -INFINITY;
+                    }
+                }
+                float mx0 = x[0], mx1 = x[1];
+#pragma unroll
+                for (int i = 2; i < 62; i += 4) {
+                    mx0 = fmax3(mx0, x[i], x[i + 1]);
+                    mx1 = fmax3(mx1, x[i + 2], x[i + 3]);
+                }
+                mx0 = fmax3(mx0, x[62], x[63]);
+                m_step = fmaxf(mx0, mx1) * sc;
             }
-            mx0 = fmax3(mx0, x[62], x[63]);
-            const float m_new = fmaxf(m, fmaxf(mx0, mx1) * sc);
+            const float m_new = fmaxf(m, m_step);
             const bool grow = m_new > m + 8.f;
             if (j > 0 && __any_sync(0xffffffffu, grow)) {
                 // O holds sum P V with the old running max: move the max, rescale O and l.
@@ -438,22 +474,38 @@ __device__ __forceinline__ void attn_body(const CUtensorMap& tmQ, const CUtensor
             } else if (grow || j == 0) {
                 m = m_new;
             }
-            // p = 2^(s * scale * log2e - m), packed to bf16 pairs over the S columns just read
-            const float nm = (m == -INFINITY) ? 0.f : -m;
-            const uint64_t sc2 = pack2(sc, sc), nm2 = pack2(nm, nm);
-            uint64_t acc0 = pack2(0.f, 0.f), acc1 = acc0;
             uint32_t pk[32];
+            if (MODE == kFirstOrder && tangent) {
+                // w_j = e^{xbar} (1 + s (q.k_j - q.kbar)), relative to the running max:
+                // e = 2^(xbar sc - m), slope e ln2 sc; the normaliser gains c_J e
+                const float e = ex2_approx(m_step - m);
+                const float slope = e * (sc * 0.69314718055994530942f);
+                const uint64_t nx2 = pack2(-xbar, -xbar), sl2 = pack2(slope, slope), e2 = pack2(e, e);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                float y0, y1;
-                unpack2(ffma2(pack2(x[2 * i], x[2 * i + 1]), sc2, nm2), y0, y1);
-                const float p0 = ex2_approx(y0), p1 = ex2_approx(y1);
-                if (i & 1) acc1 = fadd2(acc1, pack2(p0, p1));
-                else acc0 = fadd2(acc0, pack2(p0, p1));
-                __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-                pk[i] = *reinterpret_cast<uint32_t*>(&h2);
-            }
-            {
+                for (int i = 0; i < 32; ++i) {
+                    float w0, w1;
+                    unpack2(ffma2(fadd2(pack2(x[2 * i], x[2 * i + 1]), nx2), sl2, e2), w0, w1);
+                    w0 = 2 * i < ncol ? w0 : 0.f;
+                    w1 = 2 * i + 1 < ncol ? w1 : 0.f;
+                    __nv_bfloat162 h2 = __floats2bfloat162_rn(w0, w1);
+                    pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+                }
+                l += (float)ncol * e;
+            } else {
+                // p = 2^(s * scale * log2e - m), packed to bf16 pairs over the S columns just read
+                const float nm = (m == -INFINITY) ? 0.f : -m;
+                const uint64_t sc2 = pack2(sc, sc), nm2 = pack2(nm, nm);
+                uint64_t acc0 = pack2(0.f, 0.f), acc1 = acc0;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    float y0, y1;
+                    unpack2(ffma2(pack2(x[2 * i], x[2 * i + 1]), sc2, nm2), y0, y1);
+                    const float p0 = ex2_approx(y0), p1 = ex2_approx(y1);
+                    if (i & 1) acc1 = fadd2(acc1, pack2(p0, p1));
+                    else acc0 = fadd2(acc0, pack2(p0, p1));
+                    __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+                    pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+                }
                 float a0, a1, b0, b1;
                 unpack2(acc0, a0, a1);
                 unpack2(acc1, b0, b1);
@@ -539,16 +591,24 @@ template <int D, int NS>
 __global__ void __launch_bounds__(192, 2)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
-    attn_body<D, NS, false>(tmQ, tmK, tmV, tmK, tmV, p);
+    attn_body<D, NS, kPlain>(tmQ, tmK, tmV, tmK, tmV, p);
 }
 
-// With compensation of the dropped blocks: kbar / vbar maps over [BH][nBpad][D].
+// Mean-key compensation of the dropped blocks: kbar / vbar maps over [BH][nBpad][D].
 template <int D, int NS>
 __global__ void __launch_bounds__(192, 2)
     attn_comp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKb,
                      const __grid_constant__ CUtensorMap tmVb, const AttnParams p) {
-    attn_body<D, NS, true>(tmQ, tmK, tmV, tmKb, tmVb, p);
+    attn_body<D, NS, kMeanComp>(tmQ, tmK, tmV, tmKb, tmVb, p);
+}
+
+// First-order compensation of the dropped blocks: every block of the sample is walked.
+template <int D, int NS>
+__global__ void __launch_bounds__(192, 2)
+    attn_first_order_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                            const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+    attn_body<D, NS, kFirstOrder>(tmQ, tmK, tmV, tmK, tmV, p);
 }
 
 }  // namespace sba

@@ -12,6 +12,7 @@
 #include "../../include/sba.h"
 #include "attention.cuh"
 #include "attention2.cuh"
+#include "attention3.cuh"
 #include "common.cuh"
 #include "select.cuh"
 #include "score_mma.cuh"
@@ -19,6 +20,7 @@
 #include "pair.cuh"
 #include "producer.cuh"
 #include "compensation.cuh"
+#include "prune.cuh"
 
 namespace {
 
@@ -74,6 +76,21 @@ bool make_map(CUtensorMap* map, const void* base, int BH, int Npad, int D, int b
     return r == CUDA_SUCCESS;
 }
 
+// Row-major [rows][cols] bf16 as a 2-D tensor; box = 64 columns (128 B) x box_rows,
+// 128-byte swizzle.
+bool make_map_2d(CUtensorMap* map, const void* base, long long rows, int cols, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // Where the epilogue stores the output when it goes straight to sequence shards.
 struct ShardOut {
     int n;
@@ -83,8 +100,8 @@ struct ShardOut {
     float* const* lse;  // NULL: no lse
 };
 
-// kbar / vbar (COMP only): bf16 [BH][nBpad][D] block means for the compensation steps.
-template <int D, int NS, bool COMP = false>
+// kbar / vbar (kMeanComp only): bf16 [BH][nBpad][D] block means for the compensation steps.
+template <int D, int NS, int MODE = sba::kPlain>
 sba_status launch_attention(const void* q, const void* k, const void* v, void* o, float* lse,
                             int B, int H, int Npad, const int32_t* valid_len,
                             const int32_t* kv_idx, const int32_t* kv_cnt, int kmax, int dense,
@@ -97,14 +114,16 @@ sba_status launch_attention(const void* q, const void* k, const void* v, void* o
     if (!make_map(&tq, q, BH, Npad, D, 64) || !make_map(&tk, k, BH, Npad, D, 64) ||
         !make_map(&tv, v, BH, Npad, D, 64))
         return SBA_ERR_CUDA;
-    if (COMP) {
+    if (MODE == sba::kMeanComp) {
         if (!make_map(&tkb, kbar, BH, nBpad, D, 64) || !make_map(&tvb, vbar, BH, nBpad, D, 64)) return SBA_ERR_CUDA;
     } else {
         tkb = tk;
         tvb = tv;
     }
-    if (cudaFuncSetAttribute(COMP ? (const void*)sba::attn_comp_kernel<D, NS> : (const void*)sba::attn_kernel<D, NS>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kAlloc) != cudaSuccess)
+    const void* fn = MODE == sba::kMeanComp      ? (const void*)sba::attn_comp_kernel<D, NS>
+                     : MODE == sba::kFirstOrder ? (const void*)sba::attn_first_order_kernel<D, NS>
+                                                : (const void*)sba::attn_kernel<D, NS>;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kAlloc) != cudaSuccess)
         return SBA_ERR_CUDA;
     sba::AttnParams p;
     p.o = static_cast<__nv_bfloat16*>(o);
@@ -131,10 +150,45 @@ sba_status launch_attention(const void* q, const void* k, const void* v, void* o
         }
     }
     dim3 grid((Npad / 64 + 1) / 2, H, B);
-    if (COMP)
+    if (MODE == sba::kMeanComp)
         sba::attn_comp_kernel<D, NS><<<grid, 192, SM::kAlloc, stream>>>(tq, tk, tv, tkb, tvb, p);
+    else if (MODE == sba::kFirstOrder)
+        sba::attn_first_order_kernel<D, NS><<<grid, 192, SM::kAlloc, stream>>>(tq, tk, tv, p);
     else
         sba::attn_kernel<D, NS><<<grid, 192, SM::kAlloc, stream>>>(tq, tk, tv, p);
+    return cudaGetLastError() == cudaSuccess ? SBA_OK : SBA_ERR_CUDA;
+}
+
+// The two-key-block kernel (D = 128): query pairs as attn_kernel, 128 keys per step.
+sba_status launch_attention128(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                               int Npad, const int32_t* valid_len, const int32_t* kv_idx, const int32_t* kv_cnt,
+                               int kmax, int dense, const int32_t* pair_order, float softmax_scale,
+                               cudaStream_t stream) {
+    using SM = sba::Attn3Smem;
+    CUtensorMap tq, tk, tv;
+    const int BH = B * H;
+    if (!make_map(&tq, q, BH, Npad, 128, 64) || !make_map(&tk, k, BH, Npad, 128, 64) ||
+        !make_map(&tv, v, BH, Npad, 128, 64))
+        return SBA_ERR_CUDA;
+    if (cudaFuncSetAttribute(sba::attn128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kAlloc) !=
+        cudaSuccess)
+        return SBA_ERR_CUDA;
+    sba::AttnParams p;
+    p.o = static_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.valid_len = valid_len;
+    p.kv_idx = kv_idx;
+    p.kv_cnt = kv_cnt;
+    p.pair_order = pair_order;
+    p.H = H;
+    p.Npad = Npad;
+    p.kmax = kmax;
+    p.dense = dense;
+    const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(128.0f);
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.wait_limit = g_wait_limit;
+    dim3 grid((Npad / 64 + 1) / 2, H, B);
+    sba::attn128_kernel<<<grid, 192, SM::kAlloc, stream>>>(tq, tk, tv, p);
     return cudaGetLastError() == cudaSuccess ? SBA_OK : SBA_ERR_CUDA;
 }
 
@@ -255,6 +309,11 @@ extern "C" {
 
 int32_t sba_keep_count(int32_t n_blocks, double sparsity) {
     return sba::keep_count(n_blocks, sparsity);
+}
+
+int32_t sba_keep_count_budget(int32_t n_blocks, double sparsity, int32_t budget) {
+    if (budget < 1) return 0;
+    return sba::keep_count_budget(n_blocks, sparsity, budget);
 }
 
 size_t sba_pool_select_workspace_size(int B, int H, int Npad, int D, int block) {
@@ -385,7 +444,8 @@ static sba_status attention_common(const void* q, const void* k, const void* v, 
                                    int block, const int32_t* kv_idx, const int32_t* kv_cnt,
                                    int kmax, int dense, const int32_t* pair_order,
                                    float softmax_scale, void* stream, void* comp_ws = nullptr,
-                                   size_t comp_ws_bytes = 0, const ShardOut* shards = nullptr) {
+                                   size_t comp_ws_bytes = 0, const ShardOut* shards = nullptr,
+                                   bool first_order = false) {
     sba_status st = check_shape(B, H, Npad, D, block);
     if (st != SBA_OK) return st;
     if (!q || !k || !v || !o) return SBA_ERR_INVALID_ARG;
@@ -419,15 +479,23 @@ static sba_status attention_common(const void* q, const void* k, const void* v, 
             sba::block_mean_bf16_kernel<128><<<mgrid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(v), valid_len, H,
                                                                     Npad, nBpad, reinterpret_cast<__nv_bfloat16*>(vbar),
                                                                     groups);
-            return launch_attention<128, 2, true>(q, k, v, o, lse, B, H, Npad, valid_len, kv_idx, kv_cnt, kmax, 0,
-                                                  pair_order, softmax_scale, s, kbar, vbar, nBpad);
+            return launch_attention<128, 2, sba::kMeanComp>(q, k, v, o, lse, B, H, Npad, valid_len, kv_idx, kv_cnt,
+                                                            kmax, 0, pair_order, softmax_scale, s, kbar, vbar, nBpad);
         }
         sba::block_mean_bf16_kernel<64><<<mgrid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(k), valid_len, H, Npad,
                                                                nBpad, reinterpret_cast<__nv_bfloat16*>(kbar), groups);
         sba::block_mean_bf16_kernel<64><<<mgrid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(v), valid_len, H, Npad,
                                                                nBpad, reinterpret_cast<__nv_bfloat16*>(vbar), groups);
-        return launch_attention<64, 4, true>(q, k, v, o, lse, B, H, Npad, valid_len, kv_idx, kv_cnt, kmax, 0,
-                                             pair_order, softmax_scale, s, kbar, vbar, nBpad);
+        return launch_attention<64, 4, sba::kMeanComp>(q, k, v, o, lse, B, H, Npad, valid_len, kv_idx, kv_cnt, kmax,
+                                                       0, pair_order, softmax_scale, s, kbar, vbar, nBpad);
+    }
+    if (first_order) {
+        if (dense) return SBA_ERR_INVALID_ARG;
+        if (D == 128)
+            return launch_attention<128, 2, sba::kFirstOrder>(q, k, v, o, lse, B, H, Npad, valid_len, kv_idx, kv_cnt,
+                                                              kmax, 0, pair_order, softmax_scale, s);
+        return launch_attention<64, 4, sba::kFirstOrder>(q, k, v, o, lse, B, H, Npad, valid_len, kv_idx, kv_cnt, kmax,
+                                                         0, pair_order, softmax_scale, s);
     }
     if (shards) {
         if (D == 128)
@@ -441,6 +509,9 @@ static sba_status attention_common(const void* q, const void* k, const void* v, 
     if (D == 128 && g_attn_kernel == SBA_ATTN_KERNEL_CTA_PAIR)
         return launch_attention_pair<4>(q, k, v, o, lse, B, H, Npad, valid_len, kv_idx, kv_cnt, kmax, dense,
                                         softmax_scale, s);
+    if (D == 128 && g_attn_kernel == SBA_ATTN_KERNEL_KEY_PAIRS)
+        return launch_attention128(q, k, v, o, lse, B, H, Npad, valid_len, kv_idx, kv_cnt, kmax, dense, pair_order,
+                                   softmax_scale, s);
     if (D == 128)
         return launch_attention<128, 2>(q, k, v, o, lse, B, H, Npad, valid_len, kv_idx, kv_cnt, kmax,
                                         dense, pair_order, softmax_scale, s);
@@ -492,20 +563,28 @@ sba_status sba_attention_to_shards(const void* q, const void* k, const void* v, 
                             pair_order, softmax_scale, stream, nullptr, 0, &sh);
 }
 
-size_t sba_compensation_workspace_size(int B, int H, int Npad, int D, int block) {
+size_t sba_mean_compensation_workspace_size(int B, int H, int Npad, int D, int block) {
     if (check_shape(B, H, Npad, D, block) != SBA_OK) return 0;
     const int nBpad = (Npad / 64 + 63) / 64 * 64;
     return 2 * align_up_256((size_t)B * H * nBpad * D * 2);
 }
 
-sba_status sba_attention_compensated(const void* q, const void* k, const void* v, void* o, float* lse, int B,
-                                     int H, int Npad, int D, const int32_t* valid_len, int block,
-                                     const int32_t* kv_idx, const int32_t* kv_cnt, int kmax,
-                                     const int32_t* pair_order, float softmax_scale, void* workspace,
-                                     size_t workspace_bytes, void* stream) {
+sba_status sba_attention_mean_compensated(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                                          int H, int Npad, int D, const int32_t* valid_len, int block,
+                                          const int32_t* kv_idx, const int32_t* kv_cnt, int kmax,
+                                          const int32_t* pair_order, float softmax_scale, void* workspace,
+                                          size_t workspace_bytes, void* stream) {
     if (!workspace) return SBA_ERR_INVALID_ARG;
     return attention_common(q, k, v, o, lse, B, H, Npad, D, valid_len, block, kv_idx, kv_cnt, kmax, 0,
                             pair_order, softmax_scale, stream, workspace, workspace_bytes);
+}
+
+sba_status sba_attention_compensated(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                                     int H, int Npad, int D, const int32_t* valid_len, int block,
+                                     const int32_t* kv_idx, const int32_t* kv_cnt, int kmax,
+                                     const int32_t* pair_order, float softmax_scale, void* stream) {
+    return attention_common(q, k, v, o, lse, B, H, Npad, D, valid_len, block, kv_idx, kv_cnt, kmax, 0,
+                            pair_order, softmax_scale, stream, nullptr, 0, nullptr, true);
 }
 
 sba_status sba_get_device_status(void* stream) {
@@ -522,7 +601,8 @@ sba_status sba_get_device_status(void* stream) {
 void sba_set_wait_limit(uint64_t cycles) { g_wait_limit = cycles ? cycles : kDefaultWaitLimit; }
 
 sba_status sba_set_attention_kernel(int which) {
-    if (which != SBA_ATTN_KERNEL_AUTO && which != SBA_ATTN_KERNEL_QUERY_PAIRS && which != SBA_ATTN_KERNEL_CTA_PAIR)
+    if (which != SBA_ATTN_KERNEL_AUTO && which != SBA_ATTN_KERNEL_QUERY_PAIRS && which != SBA_ATTN_KERNEL_CTA_PAIR &&
+        which != SBA_ATTN_KERNEL_KEY_PAIRS)
         return SBA_ERR_INVALID_ARG;
     g_attn_kernel = which;
     return SBA_OK;
@@ -543,6 +623,72 @@ const char* sba_strerror(sba_status status) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- token pruning
+extern "C" int32_t sba_keep_token_count(int32_t n_tokens, double keep_ratio) {
+    if (!(keep_ratio >= 0.0 && keep_ratio <= 1.0)) return 0;
+    return sba::keep_tokens(n_tokens, keep_ratio);
+}
+
+extern "C" size_t sba_token_prune_workspace_size(int B, int N) {
+    if (B <= 0 || N <= 0 || (long long)B * N > 0x7fffffffll) return 0;
+    return align_up_256((size_t)B * N * sizeof(double));
+}
+
+extern "C" sba_status sba_token_prune_select(const void* x, int B, int N, int C, const int32_t* valid_len,
+                                             double keep_ratio, int Npad_out, int32_t* idx, int32_t* valid_len_out,
+                                             void* workspace, size_t workspace_bytes, void* stream) {
+    if (B <= 0 || N <= 0 || C <= 0 || Npad_out <= 0) return SBA_ERR_INVALID_ARG;
+    if ((long long)B * N > 0x7fffffffll || B > 65535 || C > (1 << 20)) return SBA_ERR_UNSUPPORTED;
+    if (C % 8 != 0) return SBA_ERR_UNSUPPORTED;
+    if (!x || !idx || !valid_len_out || !workspace) return SBA_ERR_INVALID_ARG;
+    if (!(keep_ratio >= 0.0 && keep_ratio <= 1.0)) return SBA_ERR_INVALID_ARG;
+    if (Npad_out < sba::keep_tokens(N, keep_ratio)) return SBA_ERR_INVALID_ARG;
+    if (workspace_bytes < (size_t)B * N * sizeof(double)) return SBA_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(workspace) || !aligned16(valid_len) ||
+        (reinterpret_cast<uintptr_t>(idx) & 3u) || (reinterpret_cast<uintptr_t>(valid_len_out) & 3u))
+        return SBA_ERR_ALIGNMENT;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    CUtensorMap tx;
+    const long long rows = (long long)B * N;
+    if (!make_map_2d(&tx, x, rows, C, sba::kNormRows)) return SBA_ERR_CUDA;
+    if (cudaFuncSetAttribute(sba::token_norm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, sba::kNormSmem) !=
+        cudaSuccess)
+        return SBA_ERR_CUDA;
+    double* norm2 = static_cast<double*>(workspace);
+    const unsigned grid = (unsigned)((rows + sba::kNormRows - 1) / sba::kNormRows);
+    sba::token_norm_kernel<<<grid, 96, sba::kNormSmem, s>>>(tx, valid_len, N, C, rows, norm2, g_wait_limit);
+    sba::prune_select_kernel<<<(unsigned)B, 1024, 0, s>>>(norm2, valid_len, N, keep_ratio, Npad_out, idx,
+                                                           valid_len_out);
+    return cudaGetLastError() == cudaSuccess ? SBA_OK : SBA_ERR_CUDA;
+}
+
+extern "C" sba_status sba_gather_tokens(const void* src, int B, int H, int N, int row_bytes, const int32_t* idx,
+                                        const int32_t* valid_len_out, int Npad_out, void* dst, void* stream) {
+    if (B <= 0 || H <= 0 || N <= 0 || Npad_out <= 0 || row_bytes <= 0) return SBA_ERR_INVALID_ARG;
+    if (row_bytes % 4 != 0) return SBA_ERR_UNSUPPORTED;
+    if (!src || !dst || !idx || !valid_len_out) return SBA_ERR_INVALID_ARG;
+    const int unit = row_bytes % 16 == 0 ? 16 : 4;
+    const uintptr_t am = (uintptr_t)unit - 1;
+    if ((reinterpret_cast<uintptr_t>(src) & am) || (reinterpret_cast<uintptr_t>(dst) & am) ||
+        (reinterpret_cast<uintptr_t>(idx) & 3u) || (reinterpret_cast<uintptr_t>(valid_len_out) & 3u))
+        return SBA_ERR_ALIGNMENT;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const long long units = (long long)B * H * Npad_out * (row_bytes / unit);
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+        return SBA_ERR_CUDA;
+    const long long want = (units + 255) / 256;
+    const unsigned grid = (unsigned)(want < 8ll * sms ? want : 8ll * sms);
+    const auto* sp = static_cast<const unsigned char*>(src);
+    auto* dp = static_cast<unsigned char*>(dst);
+    if (unit == 16)
+        sba::gather_rows_kernel<16><<<grid, 256, 0, s>>>(sp, dp, idx, valid_len_out, H, N, row_bytes, Npad_out, units);
+    else
+        sba::gather_rows_kernel<4><<<grid, 256, 0, s>>>(sp, dp, idx, valid_len_out, H, N, row_bytes, Npad_out, units);
+    return cudaGetLastError() == cudaSuccess ? SBA_OK : SBA_ERR_CUDA;
+}
 
 // ---------------------------------------------------------------- query-block pairing
 extern "C" size_t sba_pair_workspace_size(int B, int H, int Npad, int block) {
@@ -588,8 +734,9 @@ extern "C" sba_status sba_pair_query_blocks(const int32_t* kv_idx, const int32_t
 
 // ---------------------------------------------------------------- routing without allocation
 // Scratch for sba_pool_select_noalloc: a fixed array in device memory that every
-// GPU loading this library holds until the process exits.  Its name is only a
-// host-side handle; the kernel gets the device address from cudaGetSymbolAddress.
+// GPU loading this library holds until the process exits.  In host code its name is
+// only a handle; host code resolves its device address with cudaGetSymbolAddress
+// and passes that address to sba_pool_select as the workspace.
 namespace {
 constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
@@ -598,7 +745,8 @@ constexpr int kMaxDevices = 64;
 void* g_noalloc_ptr[kMaxDevices] = {};
 std::mutex g_noalloc_mutex;
 
-// Device address of the scratch array on the current device, resolved on first use.
+// Device address of the scratch array on the current device, resolved once per device
+// (on the first call there, under the lock).
 sba_status noalloc_scratch(void** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SBA_ERR_CUDA;
@@ -619,8 +767,14 @@ extern "C" sba_status sba_pool_select_noalloc(const void* q, const void* k, int 
                                               int D, const int32_t* valid_len, int block,
                                               double sparsity, int kmax, int32_t* kv_idx,
                                               int32_t* kv_cnt, void* stream) {
+    // the argument checks of sba_pool_select first, so that a bad argument is reported
+    // as such whatever the problem size
     sba_status st = check_shape(B, H, Npad, D, block);
     if (st != SBA_OK) return st;
+    if (!q || !k || !kv_idx || !kv_cnt) return SBA_ERR_INVALID_ARG;
+    if (!(sparsity >= 0.0 && sparsity < 1.0)) return SBA_ERR_INVALID_ARG;
+    if (kmax < sba::keep_count(Npad / block, sparsity)) return SBA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(valid_len)) return SBA_ERR_ALIGNMENT;
     const size_t need = sba::select_workspace_bytes((size_t)B * H, (size_t)Npad / block, (size_t)D);
     if (need > kNoAllocScratchBytes) return SBA_ERR_SCRATCH_TOO_SMALL;
     void* scratch = nullptr;

@@ -11,8 +11,9 @@
 //
 // Exactness.  A block sum of 64 bf16 values is formed channel by channel in
 // token order in fp64; the mean is one correctly rounded division.  Scores are
-// first screened in fp32 (FFMA) with a proven bound delta on their error; only
-// candidates within 2*delta of the fp32 k-th value are re-scored in fp64, with
+// first screened on the tensor cores (score_mma_kernel: bf16 hi/lo splits of the
+// means, fp32 accumulation in TMEM) with a proven bound delta on their error; only
+// candidates within 2*delta of the screened k-th value are re-scored in fp64, with
 // a fixed summation order and explicit round-to-nearest operations, and the
 // selection among them is made on those fp64 values.  Everything above the
 // band is kept, everything below is dropped.

@@ -8,6 +8,7 @@ CUDA device, the call raises.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 
 import torch
@@ -55,11 +56,16 @@ def lib() -> ctypes.CDLL:
         L.sba_qk_norm_rope_pool.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, i32, i32, f64, f32, vp, vp, vp]
         L.sba_pool_select_means.restype = i32
         L.sba_pool_select_means.argtypes = [vp, vp, i32, i32, i32, i32, vp, i32, f64, i32, vp, vp, vp, sz, vp]
-        L.sba_compensation_workspace_size.restype = sz
-        L.sba_compensation_workspace_size.argtypes = [i32, i32, i32, i32, i32]
+        L.sba_keep_count_budget.restype = ctypes.c_int32
+        L.sba_keep_count_budget.argtypes = [ctypes.c_int32, f64, ctypes.c_int32]
+        L.sba_mean_compensation_workspace_size.restype = sz
+        L.sba_mean_compensation_workspace_size.argtypes = [i32, i32, i32, i32, i32]
+        L.sba_attention_mean_compensated.restype = i32
+        L.sba_attention_mean_compensated.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, i32, vp, vp, i32,
+                                                     vp, f32, vp, sz, vp]
         L.sba_attention_compensated.restype = i32
         L.sba_attention_compensated.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, i32, vp, vp, i32, vp,
-                                                f32, vp, sz, vp]
+                                                f32, vp]
         L.sba_block_means.restype = i32
         L.sba_block_means.argtypes = [vp, i32, i32, i32, i32, vp, i32, vp, vp]
         L.sba_attention.restype = i32
@@ -86,6 +92,14 @@ def lib() -> ctypes.CDLL:
         L.sba_pool_select_noalloc.argtypes = [vp, vp, i32, i32, i32, i32, vp, i32, f64, i32, vp, vp, vp]
         L.sba_noalloc_scratch_bytes.restype = sz
         L.sba_noalloc_scratch_bytes.argtypes = []
+        L.sba_keep_token_count.restype = ctypes.c_int32
+        L.sba_keep_token_count.argtypes = [ctypes.c_int32, f64]
+        L.sba_token_prune_workspace_size.restype = sz
+        L.sba_token_prune_workspace_size.argtypes = [i32, i32]
+        L.sba_token_prune_select.restype = i32
+        L.sba_token_prune_select.argtypes = [vp, i32, i32, i32, vp, f64, i32, vp, vp, vp, sz, vp]
+        L.sba_gather_tokens.restype = i32
+        L.sba_gather_tokens.argtypes = [vp, i32, i32, i32, i32, vp, vp, i32, vp, vp]
         L.sba_strerror.restype = ctypes.c_char_p
         L.sba_strerror.argtypes = [i32]
         _lib = L
@@ -158,11 +172,10 @@ def pool_select(q, k, valid_len=None, sparsity: float = 0.0, kmax: int | None = 
 
 
 def keep_count_budget(n_blocks: int, sparsity: float, budget: int = 1) -> int:
-    """keep(n, s) rounded up to a multiple of `budget`, at most n."""
-    k = keep_count(n_blocks, sparsity)
-    if budget > 1:
-        k = min(int(n_blocks), -(-k // budget) * budget)
-    return k
+    """keep(n, s) rounded up to a multiple of `budget`, at most n (sba_keep_count_budget)."""
+    if budget < 1:
+        raise ValueError("budget must be >= 1")
+    return int(lib().sba_keep_count_budget(int(n_blocks), float(sparsity), int(budget)))
 
 
 def lse_workspace_size(B: int, H: int, Npad: int, D: int, nsub: int = 4, block: int = BLOCK) -> int:
@@ -330,22 +343,43 @@ def attention_to_shards(q, k, v, kv_idx, kv_cnt, o_shards, lse_shards=None, h_fi
 
 
 def attention_compensated(q, k, v, kv_idx, kv_cnt, valid_len=None, pair_order=None, softmax_scale: float = 0.0,
-                          out=None, lse=None, want_lse: bool = True, workspace=None, block: int = BLOCK,
-                          stream=None):
-    """Block-sparse attention with each dropped block compensated by its mean key and
-    value (see include/sba.h).  Returns (o bf16, lse fp32 or None)."""
+                          out=None, lse=None, want_lse: bool = True, block: int = BLOCK, stream=None):
+    """Block-sparse attention with the dropped blocks compensated to first order about
+    their mean keys (see include/sba.h).  Returns (o bf16, lse fp32 or None)."""
+    B, H, Npad, D = _qkv(q, k, v)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H, Npad), dtype=torch.float32, device=q.device)
+    _check(lib().sba_attention_compensated(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Npad, D,
+                                           _ptr(_valid_len(valid_len, q.device)), block, _ptr(kv_idx), _ptr(kv_cnt),
+                                           kv_idx.shape[-1], _ptr(pair_order), float(softmax_scale),
+                                           _stream(stream)), "sba_attention_compensated")
+    return out, lse
+
+
+def mean_compensation_workspace_size(B: int, H: int, Npad: int, D: int, block: int = BLOCK) -> int:
+    return int(lib().sba_mean_compensation_workspace_size(B, H, Npad, D, block))
+
+
+def attention_mean_compensated(q, k, v, kv_idx, kv_cnt, valid_len=None, pair_order=None, softmax_scale: float = 0.0,
+                               out=None, lse=None, want_lse: bool = True, workspace=None, block: int = BLOCK,
+                               stream=None):
+    """Block-sparse attention with each dropped block as one softmax entry carrying its
+    mean key and value (the zeroth-order form; see include/sba.h).  Returns (o, lse)."""
     B, H, Npad, D = _qkv(q, k, v)
     if out is None:
         out = torch.empty_like(q)
     if lse is None and want_lse:
         lse = torch.empty((B, H, Npad), dtype=torch.float32, device=q.device)
     if workspace is None:
-        workspace = torch.empty(int(lib().sba_compensation_workspace_size(B, H, Npad, D, block)), dtype=torch.uint8,
+        workspace = torch.empty(mean_compensation_workspace_size(B, H, Npad, D, block), dtype=torch.uint8,
                                 device=q.device)
-    _check(lib().sba_attention_compensated(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Npad, D,
-                                           _ptr(_valid_len(valid_len, q.device)), block, _ptr(kv_idx), _ptr(kv_cnt),
-                                           kv_idx.shape[-1], _ptr(pair_order), float(softmax_scale), _ptr(workspace),
-                                           workspace.numel(), _stream(stream)), "sba_attention_compensated")
+    _check(lib().sba_attention_mean_compensated(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Npad, D,
+                                                _ptr(_valid_len(valid_len, q.device)), block, _ptr(kv_idx),
+                                                _ptr(kv_cnt), kv_idx.shape[-1], _ptr(pair_order),
+                                                float(softmax_scale), _ptr(workspace), workspace.numel(),
+                                                _stream(stream)), "sba_attention_mean_compensated")
     return out, lse
 
 
@@ -380,6 +414,54 @@ def sparse_attention(q, k, v, valid_len=None, sparsity: float = 0.75, softmax_sc
     return o, lse, kv_idx, kv_cnt
 
 
+def keep_token_count(n_tokens: int, ratio: float) -> int:
+    """Tokens saliency pruning keeps of n: clamp(ceil(ratio * n - 1e-9), 1, n)."""
+    return int(lib().sba_keep_token_count(int(n_tokens), float(ratio)))
+
+
+def token_prune(x, valid_len=None, ratio: float = 0.5, npad_out: int | None = None, idx=None, valid_out=None,
+                workspace=None, stream=None):
+    """Token pruning by feature-norm saliency (see include/sba.h).  x: bf16 [B, N, C]
+    token features.  Returns (idx int32 [B, npad_out]: the kept tokens' indices in
+    their original order, then -1; valid_out int32 [B]: the kept counts).  npad_out
+    defaults to the kept count of a full sample rounded up to a multiple of 64."""
+    if not (x.is_cuda and x.dtype == torch.bfloat16 and x.dim() == 3 and x.is_contiguous()):
+        raise ValueError("expected a contiguous bf16 CUDA tensor [B, N, C]")
+    B, N, C = x.shape
+    if npad_out is None:
+        npad_out = -(-keep_token_count(N, ratio) // BLOCK) * BLOCK
+    if idx is None:
+        idx = torch.empty((B, npad_out), dtype=torch.int32, device=x.device)
+    if valid_out is None:
+        valid_out = torch.empty((B,), dtype=torch.int32, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(int(lib().sba_token_prune_workspace_size(B, N)), dtype=torch.uint8,
+                                device=x.device)
+    _check(lib().sba_token_prune_select(_ptr(x), B, N, C, _ptr(_valid_len(valid_len, x.device)), float(ratio),
+                                        int(npad_out), _ptr(idx), _ptr(valid_out), _ptr(workspace),
+                                        workspace.numel(), _stream(stream)), "sba_token_prune_select")
+    return idx, valid_out
+
+
+def gather_tokens(src, idx, valid_out, out=None, stream=None):
+    """The kept rows of a per-token tensor, compacted: src [B, H, N, ...] or [B, N, ...]
+    (any dtype, a row of 4k bytes), idx / valid_out as token_prune returns them.  Rows
+    past a sample's kept count are zero.  Returns [B, H, npad_out, ...] / [B, npad_out, ...]."""
+    if not (src.is_cuda and src.is_contiguous() and src.dim() >= 3):
+        raise ValueError("expected a contiguous CUDA tensor [B, H, N, ...] or [B, N, ...]")
+    B, npad_out = idx.shape
+    heads = src.dim() == 4
+    H, N = (src.shape[1], src.shape[2]) if heads else (1, src.shape[1])
+    rest = src.shape[3:] if heads else src.shape[2:]
+    row_bytes = src.element_size() * math.prod(rest)
+    shape = (B, H, npad_out, *rest) if heads else (B, npad_out, *rest)
+    if out is None:
+        out = torch.empty(shape, dtype=src.dtype, device=src.device)
+    _check(lib().sba_gather_tokens(_ptr(src), B, H, N, row_bytes, _ptr(idx), _ptr(valid_out), int(npad_out),
+                                   _ptr(out), _stream(stream)), "sba_gather_tokens")
+    return out
+
+
 def device_status(stream=None) -> int:
     """Synchronise the stream; return and clear the device-side error word (an SBA_* code)."""
     return int(lib().sba_get_device_status(_stream(stream)))
@@ -389,7 +471,7 @@ def set_wait_limit(cycles: int) -> None:
     lib().sba_set_wait_limit(int(cycles))
 
 
-_ATTN_KERNELS = {"auto": 0, "query_pairs": 1, "cta_pair": 2}
+_ATTN_KERNELS = {"auto": 0, "query_pairs": 1, "cta_pair": 2, "key_pairs": 3}
 
 
 def set_attention_kernel(which: str) -> None:

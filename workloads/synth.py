@@ -178,6 +178,29 @@ def _build(name, B, H, D, grid, sparsity, sigma, per_head_freq, drop_rate, seed,
                     sparsity=float(sparsity), grid=tuple(grid), seed=seed, positions=pos)
 
 
+def make_hidden(B: int, grid, C: int, seed: int = 5, sigma: float = 0.5, chunk: int = 256) -> np.ndarray:
+    """Token feature vectors of the whole latent grid (before any pruning), the input
+    of saliency pruning: bf16 bits [B, T*Hg*Wg, C], each channel the same smooth field +
+    sigma N(0,1) recipe as Q, K and V, in raster order.  Channels are drawn in chunks of
+    `chunk` from generators of their own, so the result does not depend on threading."""
+    T, Hg, Wg = grid
+    N = T * Hg * Wg
+    out = np.empty((B, N, C), dtype=np.uint16)
+
+    def one(job):
+        b, c0 = job
+        c1 = min(C, c0 + chunk)
+        fr = _rng(seed, 21, b, c0).uniform(0.0, 3.0, size=(c1 - c0, 8, 3))
+        ph = _rng(seed, 22, b, c0).uniform(0.0, 2 * np.pi, size=(c1 - c0, 8))
+        eps = _rng(seed, 23, b, c0).standard_normal((N, c1 - c0), dtype=np.float32)
+        out[b, :, c0:c1] = f64_to_bf16_bits(_field(grid, fr, ph) + sigma * eps.astype(np.float64))
+
+    jobs = [(b, c0) for b in range(B) for c0 in range(0, C, chunk)]
+    with concurrent.futures.ThreadPoolExecutor(max_workers=min(len(jobs), os.cpu_count() or 1)) as ex:
+        list(ex.map(one, jobs))
+    return out
+
+
 def make_norm_weights(D: int, seed: int = 7):
     """Per-channel RMSNorm weights for Q and K: bf16 bits [D] each, drawn from
     U[0.5, 1.5) (learned QK-norm scales sit near 1)."""
