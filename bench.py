@@ -71,9 +71,8 @@ def parse():
     ap.add_argument("--budget", type=int, default=1)
     ap.add_argument("--producer", action="store_true")
     ap.add_argument("--compensate", default=None, choices=["first", "mean"])
-    ap.add_argument("--attn-kernel", default="auto", choices=["auto", "query_pairs", "cta_pair", "key_pairs"],
-                    help="D = 128 attention kernel: auto, the query pairs (64 keys per step), the CTA pair, "
-                         "or the query pairs with 128 keys per step")
+    ap.add_argument("--attn-kernel", default="auto", choices=["auto", "query_pairs", "cta_pair"],
+                    help="D = 128 attention kernel: the default query pairs, or the opt-in CTA pair")
     return ap.parse_args()
 
 

@@ -351,9 +351,6 @@ void sba_set_wait_limit(uint64_t cycles);
  *                                (tcgen05 MMAs of M = 256 across the pair, 128 keys per
  *                                step), walking the union of their four lists;
  *                                pair_order is not used;
- *   SBA_ATTN_KERNEL_KEY_PAIRS    the query pairs of SBA_ATTN_KERNEL_QUERY_PAIRS, walking
- *                                their union two key blocks (128 keys) per step, which
- *                                halves the shared-memory reads of Q per key;
  *   SBA_ATTN_KERNEL_AUTO         (default) the query pairs, the faster of the two on
  *                                every workload measured on B200.
  * Outputs agree up to floating-point accumulation order.  Process-wide; returns
@@ -361,7 +358,6 @@ void sba_set_wait_limit(uint64_t cycles);
 #define SBA_ATTN_KERNEL_AUTO 0
 #define SBA_ATTN_KERNEL_QUERY_PAIRS 1
 #define SBA_ATTN_KERNEL_CTA_PAIR 2
-#define SBA_ATTN_KERNEL_KEY_PAIRS 3
 sba_status sba_set_attention_kernel(int which);
 
 /* Routing for callers that cannot allocate device memory.

@@ -12,7 +12,6 @@
 #include "../../include/sba.h"
 #include "attention.cuh"
 #include "attention2.cuh"
-#include "attention3.cuh"
 #include "common.cuh"
 #include "select.cuh"
 #include "score_mma.cuh"
@@ -156,39 +155,6 @@ sba_status launch_attention(const void* q, const void* k, const void* v, void* o
         sba::attn_first_order_kernel<D, NS><<<grid, 192, SM::kAlloc, stream>>>(tq, tk, tv, p);
     else
         sba::attn_kernel<D, NS><<<grid, 192, SM::kAlloc, stream>>>(tq, tk, tv, p);
-    return cudaGetLastError() == cudaSuccess ? SBA_OK : SBA_ERR_CUDA;
-}
-
-// The two-key-block kernel (D = 128): query pairs as attn_kernel, 128 keys per step.
-sba_status launch_attention128(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-                               int Npad, const int32_t* valid_len, const int32_t* kv_idx, const int32_t* kv_cnt,
-                               int kmax, int dense, const int32_t* pair_order, float softmax_scale,
-                               cudaStream_t stream) {
-    using SM = sba::Attn3Smem;
-    CUtensorMap tq, tk, tv;
-    const int BH = B * H;
-    if (!make_map(&tq, q, BH, Npad, 128, 64) || !make_map(&tk, k, BH, Npad, 128, 64) ||
-        !make_map(&tv, v, BH, Npad, 128, 64))
-        return SBA_ERR_CUDA;
-    if (cudaFuncSetAttribute(sba::attn128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kAlloc) !=
-        cudaSuccess)
-        return SBA_ERR_CUDA;
-    sba::AttnParams p;
-    p.o = static_cast<__nv_bfloat16*>(o);
-    p.lse = lse;
-    p.valid_len = valid_len;
-    p.kv_idx = kv_idx;
-    p.kv_cnt = kv_cnt;
-    p.pair_order = pair_order;
-    p.H = H;
-    p.Npad = Npad;
-    p.kmax = kmax;
-    p.dense = dense;
-    const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(128.0f);
-    p.scale_log2 = scale * 1.4426950408889634f;
-    p.wait_limit = g_wait_limit;
-    dim3 grid((Npad / 64 + 1) / 2, H, B);
-    sba::attn128_kernel<<<grid, 192, SM::kAlloc, stream>>>(tq, tk, tv, p);
     return cudaGetLastError() == cudaSuccess ? SBA_OK : SBA_ERR_CUDA;
 }
 
@@ -509,9 +475,6 @@ static sba_status attention_common(const void* q, const void* k, const void* v, 
     if (D == 128 && g_attn_kernel == SBA_ATTN_KERNEL_CTA_PAIR)
         return launch_attention_pair<4>(q, k, v, o, lse, B, H, Npad, valid_len, kv_idx, kv_cnt, kmax, dense,
                                         softmax_scale, s);
-    if (D == 128 && g_attn_kernel == SBA_ATTN_KERNEL_KEY_PAIRS)
-        return launch_attention128(q, k, v, o, lse, B, H, Npad, valid_len, kv_idx, kv_cnt, kmax, dense, pair_order,
-                                   softmax_scale, s);
     if (D == 128)
         return launch_attention<128, 2>(q, k, v, o, lse, B, H, Npad, valid_len, kv_idx, kv_cnt, kmax,
                                         dense, pair_order, softmax_scale, s);
@@ -601,8 +564,7 @@ sba_status sba_get_device_status(void* stream) {
 void sba_set_wait_limit(uint64_t cycles) { g_wait_limit = cycles ? cycles : kDefaultWaitLimit; }
 
 sba_status sba_set_attention_kernel(int which) {
-    if (which != SBA_ATTN_KERNEL_AUTO && which != SBA_ATTN_KERNEL_QUERY_PAIRS && which != SBA_ATTN_KERNEL_CTA_PAIR &&
-        which != SBA_ATTN_KERNEL_KEY_PAIRS)
+    if (which != SBA_ATTN_KERNEL_AUTO && which != SBA_ATTN_KERNEL_QUERY_PAIRS && which != SBA_ATTN_KERNEL_CTA_PAIR)
         return SBA_ERR_INVALID_ARG;
     g_attn_kernel = which;
     return SBA_OK;

@@ -471,7 +471,7 @@ def set_wait_limit(cycles: int) -> None:
     lib().sba_set_wait_limit(int(cycles))
 
 
-_ATTN_KERNELS = {"auto": 0, "query_pairs": 1, "cta_pair": 2, "key_pairs": 3}
+_ATTN_KERNELS = {"auto": 0, "query_pairs": 1, "cta_pair": 2}
 
 
 def set_attention_kernel(which: str) -> None:
