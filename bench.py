@@ -71,6 +71,9 @@ def parse():
     ap.add_argument("--budget", type=int, default=1)
     ap.add_argument("--producer", action="store_true")
     ap.add_argument("--compensate", default=None, choices=["first", "mean"])
+    ap.add_argument("--prune", type=float, default=None, metavar="RATIO",
+                    help="prune each sample to RATIO of its tokens by feature-norm saliency at the start of "
+                         "every step (token features of width H*D), then gather Q, K, V")
     ap.add_argument("--attn-kernel", default="auto", choices=["auto", "query_pairs", "cta_pair"],
                     help="D = 128 attention kernel: the default query pairs, or the opt-in CTA pair")
     return ap.parse_args()
@@ -80,7 +83,8 @@ def parse():
 # from the ncu captures summarised in profiles/attn_kernel_*.md, and the hash
 # of the kernel sources it was taken with.  Reported only while the sources match.
 ATTN_TRAFFIC = {"480p_dense": (633137152 + 190604544, "97729a2a40a5b977"),
-                "720p": (2978964000 + 805915904, "97729a2a40a5b977")}
+                "720p": (2978964000 + 805915904, "97729a2a40a5b977"),
+                "long_clip": (2696579328 + 909271552, "46d3116201e64454")}
 KERNEL_SOURCES = ("video_dit_block_b200/csrc/attention.cuh", "video_dit_block_b200/csrc/ptx.cuh",
                   "video_dit_block_b200/csrc/common.cuh")
 
@@ -243,6 +247,37 @@ def oracle_sample(w, target_s=10.0, seed=0, router="mean", budget=1, producer=Fa
             "n_qblocks": n, "value": 1.0 / sec_per_flop / 1e12}
 
 
+def token_features(w, make_hidden):
+    """Token features of width H*D for the workload's tokens, in their order: the
+    smooth-field features of the whole latent grid (make_hidden), picked at each token's
+    (t, y, x) position; zero rows past each sample's length."""
+    B, H, Npad, D = w.q.shape
+    T, Hg, Wg = w.grid
+    hid = make_hidden(B, w.grid, H * D)
+    out = np.zeros((B, Npad, H * D), dtype=np.uint16)
+    for b in range(B):
+        L = int(w.valid_len[b])
+        p = w.positions[b, :L].astype(np.int64)
+        out[b, :L] = hid[b, (p[:, 0] * Hg + p[:, 1]) * Wg + p[:, 2]]
+    return out
+
+
+def pruned_workload(w, idx, valid_out, npad_out):
+    """The workload's Q, K, V compacted to the kept tokens (idx, as the oracle lists them)."""
+    import copy
+    B, H, _, D = w.q.shape
+    pw = copy.copy(w)
+    pw.q, pw.k, pw.v = (np.zeros((B, H, npad_out, D), dtype=np.uint16) for _ in range(3))
+    pw.positions = np.zeros((B, npad_out, 3), dtype=np.int32)
+    for b in range(B):
+        kb = int(valid_out[b])
+        for dst, src in ((pw.q, w.q), (pw.k, w.k), (pw.v, w.v)):
+            dst[b, :, :kb] = src[b][:, idx[b, :kb]]
+        pw.positions[b, :kb] = w.positions[b, idx[b, :kb]]
+    pw.valid_len = np.ascontiguousarray(valid_out, dtype=np.int32)
+    return pw
+
+
 TIE_REL = 1e-6   # score gap below which a routing difference is a tie (relative)
 
 
@@ -392,26 +427,52 @@ def run_ours(args):
     q, k, v = t(w.q), t(w.k), t(w.v)
     vl = torch.from_numpy(w.valid_len).to(dev)
     B, H, Npad, D = q.shape
+    stream = torch.cuda.current_stream(dev)
+    Npad_in = Npad
+    if args.prune is not None:
+        # token features of the workload's tokens (in their order), width H*D
+        from workloads import make_hidden
+        xf_host = token_features(w, make_hidden)
+        x = t(xf_host)
+        Npad = 64 * -(-sba.keep_token_count(Npad_in, args.prune) // 64)   # the pruned sequences' padded length
+        pr_idx = torch.empty((B, Npad), dtype=torch.int32, device=dev)
+        pr_vl = torch.empty((B,), dtype=torch.int32, device=dev)
+        pr_ws = torch.empty(int(sba.lib().sba_token_prune_workspace_size(B, Npad_in)), dtype=torch.uint8, device=dev)
+        qp, kp, vp = (torch.empty((B, H, Npad, D), dtype=torch.bfloat16, device=dev) for _ in range(3))
     lse_router = args.router == "lse"
     kmax = sba.keep_count_budget(Npad // 64, w.sparsity, args.budget) if lse_router else sba.kmax_for(Npad, w.sparsity)
     kv_idx = torch.empty((B, H, Npad // 64, kmax), dtype=torch.int32, device=dev)
     kv_cnt = torch.empty((B, H, Npad // 64), dtype=torch.int32, device=dev)
     wsz = sba.lse_workspace_size(B, H, Npad, D) if lse_router else sba.workspace_size(B, H, Npad, D)
     ws = torch.empty(wsz, dtype=torch.uint8, device=dev)
-    o = torch.empty_like(q)
+    o = torch.empty((B, H, Npad, D), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((B, H, Npad), dtype=torch.float32, device=dev)
     nQ = Npad // 64
     pair_order = torch.empty((B, H, 2 * ((nQ + 1) // 2)), dtype=torch.int32, device=dev)
     pws = torch.empty(int(sba.lib().sba_pair_workspace_size(B, H, Npad, 64)), dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream(dev)
+
+    def prep(qq=q, kk=k, vv=v, vll=vl, xx=None):
+        """With --prune: saliency pruning of the step's tokens, then the compacted Q, K, V
+        and valid lengths; otherwise the inputs as they are."""
+        if args.prune is None:
+            return qq, kk, vv, vll
+        sba.token_prune(x if xx is None else xx, vll, args.prune, npad_out=Npad, idx=pr_idx, valid_out=pr_vl,
+                        workspace=pr_ws, stream=stream)
+        for src, dst in ((qq, qp), (kk, kp), (vv, vp)):
+            sba.gather_tokens(src, pr_idx, pr_vl, out=dst, stream=stream)
+        if args.producer:
+            sba.gather_tokens(pos_src, pr_idx, pr_vl, out=pos, stream=stream)
+        return qp, kp, vp, pr_vl
 
     if args.producer:
         if lse_router:
             raise SystemExit("--producer routes from block means: use the block-mean router")
         from workloads import make_norm_weights
         wq, wk = (t(x) for x in make_norm_weights(D))
-        pos = torch.from_numpy(w.positions).to(dev)
-        q_n, k_n = torch.empty_like(q), torch.empty_like(k)
+        pos_src = torch.from_numpy(w.positions).to(dev)
+        # with --prune, the pruned tokens' positions, gathered by each step's pruning
+        pos = pos_src if args.prune is None else torch.empty((B, Npad, 3), dtype=torch.int32, device=dev)
+        q_n, k_n = (torch.empty((B, H, Npad, D), dtype=torch.bfloat16, device=dev) for _ in range(2))
         q_m = torch.empty((B, H, Npad // 64, D), dtype=torch.float64, device=dev)
         k_m = torch.empty_like(q_m)
 
@@ -447,9 +508,10 @@ def run_ours(args):
         else:
             sba.attention_paired(qq, kk, vv, kv_idx, kv_cnt, pair_order, vll, out=out, lse=lse, stream=stream)
 
-    def step(qq=q, kk=k, vv=v):
-        qa, ka = route(qq, kk)
-        attend(qa, ka, vv)
+    def step(qq=q, kk=k, vv=v, vll=vl, xx=None):
+        qq, kk, vv, vll = prep(qq, kk, vv, vll, xx)
+        qa, ka = route(qq, kk, vll)
+        attend(qa, ka, vv, vll)
 
     def barrier():
         if dist is not None:
@@ -462,20 +524,22 @@ def run_ours(args):
     status = sba.device_status(stream)
     if status != 0:
         raise RuntimeError(f"device status {status} after warm-up")
-    f_step = kept_flops(kv_idx.cpu().numpy(), kv_cnt.cpu().numpy(), w.valid_len, D)
+    vl_step = pr_vl.cpu().numpy() if args.prune is not None else w.valid_len
+    f_step = kept_flops(kv_idx.cpu().numpy(), kv_cnt.cpu().numpy(), vl_step, D)
 
     # ---- timed region: K steps, events on the launching stream
     K = args.steps
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(4)) for _ in range(K)]
     barrier()
     torch.cuda.synchronize(dev)
     t_begin = time.monotonic()
     for i in range(K):
         ev[i][0].record(stream)
-        qa, ka = route()
+        qq, kk, vv, vll = prep()
+        ev[i][3].record(stream)
+        qa, ka = route(qq, kk, vll)
         ev[i][1].record(stream)
-        attend(qa, ka)
+        attend(qa, ka, vv, vll)
         ev[i][2].record(stream)
     torch.cuda.synchronize(dev)
     clocks.mark(t_begin, time.monotonic())
@@ -487,10 +551,11 @@ def run_ours(args):
     med_step = statistics.median(e[0].elapsed_time(e[2]) for e in ev)
     med_sel = statistics.median(e[0].elapsed_time(e[1]) for e in ev)
     med_attn = statistics.median(e[1].elapsed_time(e[2]) for e in ev)
+    prune_ms = statistics.mean(e[0].elapsed_time(e[3]) for e in ev)
     if sba.device_status(stream) != 0:
         raise RuntimeError("device status error in the timed region")
-    total_ms, attn_ms, sel_ms, med_step, med_sel, med_attn = max_over_ranks(
-        [total_ms, attn_ms, sel_ms, med_step, med_sel, med_attn], dist, dev)
+    total_ms, attn_ms, sel_ms, med_step, med_sel, med_attn, prune_ms = max_over_ranks(
+        [total_ms, attn_ms, sel_ms, med_step, med_sel, med_attn, prune_ms], dist, dev)
     ms_step = total_ms / K
     value = whole_job_value(f_step, ms_step, world)
 
@@ -502,6 +567,7 @@ def run_ours(args):
                     [lse[b, h].cpu().numpy() for b, h in par_heads],
                     [kv_idx[b, h].cpu().numpy() for b, h in par_heads],
                     [kv_cnt[b, h].cpu().numpy() for b, h in par_heads])
+        par_prune = (pr_idx.cpu().numpy(), pr_vl.cpu().numpy()) if args.prune is not None else None
 
     # ---- end to end through the public API with host buffers: every step uploads its
     # inputs from pinned host memory and downloads its output.  The steps are pipelined
@@ -512,11 +578,12 @@ def run_ours(args):
     # download.
     e2e = None
     if not args.no_e2e:
-        qh, kh, vh = (x.cpu().pin_memory() for x in (q, k, v))
+        qh, kh, vh = (z.cpu().pin_memory() for z in (q, k, v))
         vlh = vl.cpu().pin_memory()
+        xh = x.cpu().pin_memory() if args.prune is not None else None
         oh = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-        bufs = [(torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(vl))
-                for _ in range(2)]
+        bufs = [(torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(vl),
+                 torch.empty_like(x) if args.prune is not None else None) for _ in range(2)]
         outs = [o, torch.empty_like(o)]
         s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
         in_done = [torch.cuda.Event() for _ in range(2)]
@@ -529,7 +596,7 @@ def run_ours(args):
         e0.record(s_in)
         for i in range(Ke):
             bi_ = i % 2
-            qd, kd, vd, vld = bufs[bi_]
+            qd, kd, vd, vld, xd = bufs[bi_]
             with torch.cuda.stream(s_in):
                 if i >= 2:
                     s_in.wait_event(comp_done[bi_])   # step i-2 has finished reading this buffer
@@ -537,12 +604,15 @@ def run_ours(args):
                 kd.copy_(kh, non_blocking=True)
                 vd.copy_(vh, non_blocking=True)
                 vld.copy_(vlh, non_blocking=True)
+                if xd is not None:
+                    xd.copy_(xh, non_blocking=True)
                 in_done[bi_].record(s_in)
             stream.wait_event(in_done[bi_])
             if i >= 2:
                 stream.wait_event(out_done[bi_])      # step i-2's output has been downloaded
-            qa, ka = route(qd, kd, vld)
-            attend(qa, ka, vd, vld, out=outs[bi_])
+            qq, kk, vv, vll = prep(qd, kd, vd, vld, xd)
+            qa, ka = route(qq, kk, vll)
+            attend(qa, ka, vv, vll, out=outs[bi_])
             comp_done[bi_].record(stream)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(comp_done[bi_])
@@ -553,7 +623,7 @@ def run_ours(args):
         if sba.device_status(stream) != 0:
             raise RuntimeError("device status error in the end-to-end loop")
         e_ms = max_over_ranks([e0.elapsed_time(e1) / Ke], dist, dev)[0]
-        bi = 3 * q.numel() * 2 + vl.numel() * 4
+        bi = 3 * q.numel() * 2 + vl.numel() * 4 + (x.numel() * 2 if args.prune is not None else 0)
         e2e = {"value": whole_job_value(f_step, e_ms, world), "unit": "TFLOP/s",
                "ms_per_step": e_ms, "h2d_bytes_per_step": bi, "d2h_bytes_per_step": o.numel() * 2,
                "steps": Ke, "mode": "pipelined: double-buffered uploads, compute and downloads on three streams"}
@@ -565,7 +635,7 @@ def run_ours(args):
     peaks, src = load_peaks()
     tr = ATTN_TRAFFIC.get(w.name)
     traffic = (tr[0] if tr is not None and tr[1] == kernel_source_hash() and not args.compensate
-               and not pair_kernel else None)
+               and not pair_kernel and args.prune is None else None)
     peak = float(peaks["bf16_tflops"])
     achieved = f_step / (attn_ms * 1e-3) / 1e12
     line = {
@@ -595,14 +665,31 @@ def run_ours(args):
         # CTA-pair kernel); 1 attention
         # (--producer: 2 producer launches and 2 splits of the given means replace pooling)
         # (--compensate mean: 2 block-mean launches before the attention)
+        # (--prune: norm + select + 3 gathers, and the positions' gather with --producer)
         "gpu_launches": (4 + (1 if w.sparsity > 0 else 0) + (2 if args.producer else 0)
-                         + (0 if pair_kernel else 10) + 1 + (2 if args.compensate == "mean" else 0)) * K,
+                         + (0 if pair_kernel else 10) + 1 + (2 if args.compensate == "mean" else 0)
+                         + (5 + (1 if args.producer else 0) if args.prune is not None else 0)) * K,
         "clocks": clk,
     }
     if e2e is not None:
         line["e2e"] = e2e
+    if args.prune is not None:
+        line["prune_ms"] = prune_ms
+        line["config"]["pruning"] = {"ratio": args.prune, "features": f"bf16 [B, N, {x.shape[2]}] (H*D channels)",
+                                     "valid_len_after": [int(z) for z in vl_step], "Npad_after": Npad}
+        # the norm kernel reads the features once: its share of the pruning stage's time
+        line["prune_feature_gbs"] = x.numel() * 2 / (prune_ms * 1e-3) / 1e9
     if par_data is not None:
-        line["parity"] = parity_check(args, w, par_heads, *par_data)
+        pw = w
+        if args.prune is not None:
+            import oracle
+            io, vo, _ = oracle.token_prune(xf_host, w.valid_len, args.prune, npad_out=Npad)
+            prune_exact = bool(np.array_equal(io, par_prune[0]) and np.array_equal(vo, par_prune[1]))
+            pw = pruned_workload(w, io, vo, Npad)
+        line["parity"] = parity_check(args, pw, par_heads, *par_data)
+        if args.prune is not None:
+            line["parity"]["prune_index_exact"] = prune_exact
+            line["parity"]["ok"] = line["parity"]["ok"] and prune_exact
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_from(oracle_sample(w, target_s=15.0, router=args.router,
                                                                budget=args.budget, producer=args.producer,

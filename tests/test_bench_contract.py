@@ -62,3 +62,15 @@ def test_our_arm_line():
     assert p["max_abs"] <= 2e-2 and p["mean_abs"] <= 2e-3 and p["out_rows"] > 0
     m = d["median_ms"]
     assert m["step"] > 0 and m["attn"] > 0 and m["select"] > 0
+
+
+@pytest.mark.gpu
+def test_our_arm_line_with_pruning():
+    """--prune: saliency pruning and the gathers inside every step; the parity block
+    also checks the pruned index lists against the oracle."""
+    d = _run(["--config", "tiny", "--steps", "3", "--warmup", "3", "--prune", "0.5", "--no-cpu-baseline"], 900)
+    _check_base(d)
+    assert d["prune_ms"] > 0 and d["config"]["pruning"]["ratio"] == 0.5
+    assert d["config"]["pruning"]["valid_len_after"] == [512]
+    p = d["parity"]
+    assert p["prune_index_exact"] is True and p["ok"] is True and p["mask_mismatch"] == 0

@@ -115,3 +115,22 @@ def test_valid_len_one(sba, oracle_mod):
     w = make_custom(2, 2, 128, (2, 8, 40), 0.5, seed=43)
     w.valid_len = np.array([1, 577], dtype=np.int32)
     check_routing(sba, oracle_mod, w)
+
+
+def test_fast_rows_and_handed_back_rows_in_one_call(sba, oracle_mod):
+    """The thread-per-row top-k hands rows it cannot settle within its window (all
+    scores equal, or a tie band wider than its cache) to the warp-per-row kernel; both
+    kinds of rows side by side in one call must match the oracle."""
+    rng = np.random.default_rng(23)
+    w = make_custom(1, 2, 128, (4, 16, 40), 0.75, seed=24)       # 40 blocks
+    q = w.q.copy()
+    q[:, :, 64 * 3:64 * 4] = f64_to_bf16_bits(np.zeros((1, 2, 64, 128)))   # block 3: all scores 0
+    w.q = q
+    k = w.k.copy()
+    # 24 identical key blocks: every query block sees a 24-way exact tie, wider than the
+    # band cache, wherever the k-th score falls among them
+    for J in range(1, 25):
+        k[:, 0, 64 * J:64 * (J + 1)] = k[:, 0, 0:64]
+    w.k = k
+    for s in (0.5, 0.75, 0.9):
+        check_routing(sba, oracle_mod, w, s)

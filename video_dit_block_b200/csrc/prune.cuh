@@ -13,13 +13,15 @@
 // squared norms are bit for bit the sequential fp64 sums; the selection on them is
 // then exact (a radix select on the order-preserving bits, ties to the lower index).
 //
-//   token_norm_kernel    HBM-bound: 64 tokens per CTA, their rows streamed through a
-//                        4-stage ring of TMA tiles (64 tokens x 128 channels, 128-byte
+//   token_norm_kernel    HBM-bound: 128 tokens per CTA, their rows streamed through a
+//                        4-stage ring of TMA tiles (128 tokens x 64 channels, 128-byte
 //                        swizzle, so the threads reading one 16-byte chunk each of
 //                        eight consecutive rows hit distinct banks); thread t sums
 //                        token t's channels in order.
-//   prune_select_kernel  one CTA per sample: 8-bit radix select of the k-th largest
-//                        squared norm, then an in-order compaction by block scans.
+//   prune_select_kernel  one CTA per sample: a bucket histogram over the sample's range
+//                        locates the k-th largest squared norm, a radix select among
+//                        that bucket's members finds it, an in-order compaction by
+//                        block scans lists the kept tokens.
 //   gather_rows_kernel   HBM-bound row copy dst[bh][p] = src[bh][idx[b][p]] (zero rows
 //                        past the kept count), 16-byte units.
 #pragma once
@@ -32,9 +34,9 @@
 
 namespace sba {
 
-constexpr int kNormRows = 64;       // tokens per CTA
+constexpr int kNormRows = 128;      // tokens per CTA
 constexpr int kNormBoxCols = 64;    // channels per TMA box (128 bytes)
-constexpr int kNormBoxes = 2;       // boxes per stage
+constexpr int kNormBoxes = 1;       // boxes per stage
 constexpr int kNormStages = 4;
 constexpr int kNormStageBytes = kNormBoxes * kNormRows * kNormBoxCols * 2;   // 16 KB
 constexpr int kNormSmem = kNormStages * kNormStageBytes + 1024 + 2 * kNormStages * 8 + 16;
@@ -53,10 +55,10 @@ __host__ __device__ inline int keep_tokens(int n, double r) {
     return (int)x;
 }
 
-// x viewed as rows [B*N][C] (tensor map tmX: box 64 channels x 64 rows, 128-byte
+// x viewed as rows [B*N][C] (tensor map tmX: box 64 channels x 128 rows, 128-byte
 // swizzle).  norm2[row] = sum_c x[row][c]^2 in channel order (0 for padding tokens).
-// 96 threads: warps 0-1 sum (thread t = token t of the tile), warp 2 lane 0 loads.
-__global__ void __launch_bounds__(96) token_norm_kernel(const __grid_constant__ CUtensorMap tmX,
+// 160 threads: warps 0-3 sum (thread t = token t of the tile), warp 4 lane 0 loads.
+__global__ void __launch_bounds__(160) token_norm_kernel(const __grid_constant__ CUtensorMap tmX,
                                                         const int32_t* __restrict__ valid_len, int N, int C,
                                                         long long rows, double* __restrict__ norm2,
                                                         unsigned long long wait_limit) {
@@ -82,7 +84,7 @@ __global__ void __launch_bounds__(96) token_norm_kernel(const __grid_constant__ 
     }
     __syncthreads();
     int issued = 0;
-    if (warp == 2) {
+    if (warp == 4) {
         if ((tid & 31) == 0) {
             tma_prefetch_desc(&tmX);
             for (int st = 0; st < n_steps; ++st) {
@@ -134,7 +136,7 @@ __global__ void __launch_bounds__(96) token_norm_kernel(const __grid_constant__ 
         }
     }
     __syncthreads();
-    if (*abort_flag && warp == 2 && (tid & 31) == 0) {
+    if (*abort_flag && warp == 4 && (tid & 31) == 0) {
         // let this CTA's own copies land before it exits
         for (int st = issued > kNormStages ? issued - kNormStages : 0; st < issued; ++st) {
             const long long t0 = clock64();
@@ -178,31 +180,32 @@ __device__ __forceinline__ int block_scan_1024(int v, int* scratch, int* total) 
 // One CTA of 1024 threads per sample b: keep the k = keep_tokens(L_b, ratio) tokens of
 // largest norm2 (ties to the lower index), idx[b][0..k) ascending, then -1 up to
 // Npad_out; valid_out[b] = k.
-__global__ void __launch_bounds__(1024) prune_select_kernel(const double* __restrict__ norm2,
-                                                            const int32_t* __restrict__ valid_len, int N,
-                                                            double ratio, int Npad_out, int32_t* __restrict__ idx,
-                                                            int32_t* __restrict__ valid_out) {
-    __shared__ uint32_t hist[256];
-    __shared__ int scan_scratch[33];
-    __shared__ uint32_t sel_digit, sel_above;
-    const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
-    int L = valid_len ? valid_len[b] : N;
-    if (L < 0 || L > N) {  // outside the documented range: flag it, never read past the sample
-        if (tid == 0) raise_device_error(kErrBadRouting);
-        L = L < 0 ? 0 : N;
-    }
-    const int k = keep_tokens(L, ratio);
-    const uint64_t* key = reinterpret_cast<const uint64_t*>(norm2 + (size_t)b * N);  // >= +0: bits are ordered
-    int32_t* out = idx + (size_t)b * Npad_out;
+//   1. the sample's smallest and largest squared norm;
+//   2. a kSelBuckets-bucket histogram between them; bucketing is monotone, so the k-th
+//      largest value tau lies in the bucket b* where the count from the top reaches k;
+//   3. tau exactly: a radix select (8-bit digits of the fp64 bits, which order
+//      non-negative values) over the members of b* only, gathered into shared memory;
+//      when b* holds more than kSelGather tokens (many equal norms), over the whole
+//      sample instead;
+//   4. an in-order compaction by block scans: every value above tau, and the first
+//      values equal to it, as many as the selection needs.
+constexpr int kSelBuckets = 2048;
+constexpr int kSelGather = 1024;
 
-    // ---- radix select of the k-th largest key, most significant byte first
+// Block-wide (1024 threads) k-th largest of the 64-bit keys key_of(i), i < n, among
+// those with pred(i); returns tau and, in *remaining, how many keys equal to tau the
+// k largest include.  hist: 256 words of shared memory.
+template <typename KeyOf>
+__device__ uint64_t block_radix_select(int n, uint32_t k, uint32_t* hist, uint32_t* sel, KeyOf key_of,
+                                       uint32_t* remaining_out) {
+    const int tid = threadIdx.x, lane = tid & 31;
     uint64_t prefix = 0, mask = 0;
-    uint32_t remaining = (uint32_t)k;
-    for (int shift = 56; shift >= 0 && k > 0; shift -= 8) {
+    uint32_t remaining = k;
+    for (int shift = 56; shift >= 0; shift -= 8) {
         for (int i = tid; i < 256; i += 1024) hist[i] = 0u;
         __syncthreads();
-        for (int n = tid; n < L; n += 1024) {
-            const uint64_t x = key[n];
+        for (int i = tid; i < n; i += 1024) {
+            const uint64_t x = key_of(i);
             if ((x & mask) == prefix) atomicAdd(&hist[(x >> shift) & 255u], 1u);
         }
         __syncthreads();
@@ -227,8 +230,8 @@ __global__ void __launch_bounds__(1024) prune_select_kernel(const double* __rest
                 uint32_t acc = excl;
                 for (int e = 0; e < 8; ++e) {
                     if (acc + c[e] >= remaining) {
-                        sel_digit = 255u - (8u * lane + e);
-                        sel_above = acc;
+                        sel[0] = 255u - (8u * lane + e);
+                        sel[1] = acc;
                         break;
                     }
                     acc += c[e];
@@ -236,13 +239,131 @@ __global__ void __launch_bounds__(1024) prune_select_kernel(const double* __rest
             }
         }
         __syncthreads();
-        prefix |= (uint64_t)sel_digit << shift;
+        prefix |= (uint64_t)sel[0] << shift;
         mask |= 0xFFull << shift;
-        remaining -= sel_above;
+        remaining -= sel[1];
         __syncthreads();
     }
-    // ---- in-order compaction: keys above tau, and the first `remaining` keys equal to it
-    const uint64_t tau = prefix;
+    *remaining_out = remaining;
+    return prefix;
+}
+
+__global__ void __launch_bounds__(1024) prune_select_kernel(const double* __restrict__ norm2,
+                                                            const int32_t* __restrict__ valid_len, int N,
+                                                            double ratio, int Npad_out, int32_t* __restrict__ idx,
+                                                            int32_t* __restrict__ valid_out) {
+    __shared__ uint32_t bhist[kSelBuckets];
+    __shared__ uint64_t gkey[kSelGather];
+    __shared__ uint32_t hist[256];
+    __shared__ uint32_t sel[4];
+    __shared__ double red[64];
+    __shared__ int scan_scratch[33];
+    const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    int L = valid_len ? valid_len[b] : N;
+    if (L < 0 || L > N) {  // outside the documented range: flag it, never read past the sample
+        if (tid == 0) raise_device_error(kErrBadRouting);
+        L = L < 0 ? 0 : N;
+    }
+    const int k = keep_tokens(L, ratio);
+    const double* val = norm2 + (size_t)b * N;
+    const uint64_t* key = reinterpret_cast<const uint64_t*>(val);  // >= +0: bits are ordered
+    int32_t* out = idx + (size_t)b * Npad_out;
+
+    uint64_t tau = 0;
+    uint32_t remaining = 0;
+    if (k > 0) {
+        // ---- 1. range
+        double lo = INFINITY, hi = -INFINITY;
+        for (int n = tid; n < L; n += 1024) {
+            lo = fmin(lo, val[n]);
+            hi = fmax(hi, val[n]);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            lo = fmin(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+            hi = fmax(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+        }
+        if (lane == 0) {
+            red[wid] = lo;
+            red[32 + wid] = hi;
+        }
+        __syncthreads();
+        if (wid == 0) {
+            lo = red[lane];
+            hi = red[32 + lane];
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                lo = fmin(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+                hi = fmax(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+            }
+            if (lane == 0) {
+                red[0] = lo;
+                red[1] = hi;
+            }
+        }
+        __syncthreads();
+        lo = red[0];
+        hi = red[1];
+        const double range = hi - lo;
+        const double bscale = range > 0.0 ? kSelBuckets / range : 0.0;
+        bool whole = !(range > 0.0 && bscale < 1e300);   // all equal: select over the whole sample
+        int bstar = 0;
+        uint32_t above = 0, members = 0;
+        if (!whole) {
+            // ---- 2. bucket histogram and the bucket holding tau
+            auto bucket = [&](double x) { return max(0, min(kSelBuckets - 1, (int)((x - lo) * bscale))); };
+            for (int i = tid; i < kSelBuckets; i += 1024) bhist[i] = 0u;
+            __syncthreads();
+            for (int n = tid; n < L; n += 1024) atomicAdd(&bhist[bucket(val[n])], 1u);
+            __syncthreads();
+            if (wid == 0) {
+                // lane l holds buckets 2047 - 64l - e (e = 0..63), highest first
+                uint32_t tot = 0;
+                for (int e = 0; e < 64; ++e) tot += bhist[kSelBuckets - 1 - (64 * lane + e)];
+                uint32_t incl = tot;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const uint32_t u = __shfl_up_sync(0xffffffffu, incl, off);
+                    if (lane >= off) incl += u;
+                }
+                const uint32_t excl = incl - tot;
+                const uint32_t ball = __ballot_sync(0xffffffffu, excl < (uint32_t)k && (uint32_t)k <= incl);
+                const int src = ball ? __ffs(ball) - 1 : 31;
+                if (lane == src) {
+                    uint32_t acc = excl;
+                    for (int e = 0; e < 64; ++e) {
+                        const int bk = kSelBuckets - 1 - (64 * lane + e);
+                        if (acc + bhist[bk] >= (uint32_t)k) {
+                            sel[0] = (uint32_t)bk;
+                            sel[1] = acc;
+                            sel[2] = bhist[bk];
+                            break;
+                        }
+                        acc += bhist[bk];
+                    }
+                }
+            }
+            __syncthreads();
+            bstar = (int)sel[0];
+            above = sel[1];
+            members = sel[2];
+            __syncthreads();
+            whole = members > (uint32_t)kSelGather;
+            if (!whole) {
+                // ---- 3. gather bucket b*'s keys (any order) and select among them
+                if (tid == 0) sel[3] = 0u;
+                __syncthreads();
+                for (int n = tid; n < L; n += 1024)
+                    if (bucket(val[n]) == bstar) gkey[atomicAdd(&sel[3], 1u)] = key[n];
+                __syncthreads();
+                tau = block_radix_select((int)members, (uint32_t)k - above, hist, sel,
+                                         [&](int i) { return gkey[i]; }, &remaining);
+            }
+        }
+        if (whole)
+            tau = block_radix_select(L, (uint32_t)k, hist, sel, [&](int i) { return key[i]; }, &remaining);
+    }
+    // ---- 4. in-order compaction: keys above tau, and the first `remaining` keys equal to it
     int pos_base = 0, eq_base = 0;
     for (int n0 = 0; n0 < L; n0 += 1024) {
         const int n = n0 + tid;
@@ -251,10 +372,10 @@ __global__ void __launch_bounds__(1024) prune_select_kernel(const double* __rest
         const bool eq = n < L && k > 0 && x == tau;
         int eq_tot;
         const int eq_rank = block_scan_1024(eq ? 1 : 0, scan_scratch, &eq_tot);
-        const bool sel = gt || (eq && (uint32_t)(eq_base + eq_rank) < remaining);
+        const bool sel_ = gt || (eq && (uint32_t)(eq_base + eq_rank) < remaining);
         int sel_tot;
-        const int pos = block_scan_1024(sel ? 1 : 0, scan_scratch, &sel_tot);
-        if (sel) out[pos_base + pos] = n;
+        const int pos = block_scan_1024(sel_ ? 1 : 0, scan_scratch, &sel_tot);
+        if (sel_) out[pos_base + pos] = n;
         pos_base += sel_tot;
         eq_base += eq_tot;
     }
@@ -267,34 +388,48 @@ __global__ void __launch_bounds__(1024) prune_select_kernel(const double* __rest
 
 // dst[bh][p][:] = src[bh][idx[b][p]][:] for p < valid_out[b], zero rows up to Npad_out.
 // src: [B*H][N][row_bytes], dst: [B*H][Npad_out][row_bytes]; UNIT-byte copies
-// (UNIT 16 or 4, dividing row_bytes).
+// (UNIT 16 or 4, dividing row_bytes).  blockIdx.y = bh, so the sample's kept count and
+// index list are fixed per CTA and the unit arithmetic stays in 32 bits; each thread has
+// four loads in flight before it stores.
 template <int UNIT>
 __global__ void __launch_bounds__(256) gather_rows_kernel(const unsigned char* __restrict__ src,
                                                           unsigned char* __restrict__ dst,
                                                           const int32_t* __restrict__ idx,
                                                           const int32_t* __restrict__ valid_out, int H, int N,
-                                                          int row_bytes, int Npad_out, long long units) {
+                                                          int row_bytes, int Npad_out) {
     using T = typename std::conditional<UNIT == 16, uint4, uint32_t>::type;
+    constexpr int kIn = 4;
     const int per_row = row_bytes / UNIT;
-    for (long long u = (long long)blockIdx.x * blockDim.x + threadIdx.x; u < units;
-         u += (long long)gridDim.x * blockDim.x) {
-        const long long orow = u / per_row;   // (bh, p)
-        const int part = (int)(u % per_row);
-        const long long bh = orow / Npad_out;
-        const int p = (int)(orow % Npad_out);
-        const int b = (int)(bh / H);
-        T v;
-        if (p < valid_out[b]) {
-            int n = idx[(size_t)b * Npad_out + p];
-            if (n < 0 || n >= N) {
-                raise_device_error(kErrBadRouting);
-                n = 0;
+    const int bh = blockIdx.y, b = bh / H;
+    const int kept = valid_out[b];
+    const int units = Npad_out * per_row;
+    const T* s = reinterpret_cast<const T*>(src + (size_t)bh * N * row_bytes);
+    T* d = reinterpret_cast<T*>(dst + (size_t)bh * Npad_out * row_bytes);
+    const int32_t* ib = idx + (size_t)b * Npad_out;
+    const int stride = gridDim.x * blockDim.x;
+    for (int u0 = blockIdx.x * blockDim.x + threadIdx.x; u0 < units; u0 += kIn * stride) {
+        T v[kIn];
+#pragma unroll
+        for (int i = 0; i < kIn; ++i) {
+            const int u = u0 + i * stride;
+            v[i] = T{};
+            if (u < units) {
+                const int p = u / per_row;
+                if (p < kept) {
+                    int n = ib[p];
+                    if (n < 0 || n >= N) {
+                        raise_device_error(kErrBadRouting);
+                        n = 0;
+                    }
+                    v[i] = s[(size_t)n * per_row + (u - p * per_row)];
+                }
             }
-            v = reinterpret_cast<const T*>(src + ((size_t)bh * N + n) * row_bytes)[part];
-        } else {
-            v = T{};
         }
-        reinterpret_cast<T*>(dst + (size_t)orow * row_bytes)[part] = v;
+#pragma unroll
+        for (int i = 0; i < kIn; ++i) {
+            const int u = u0 + i * stride;
+            if (u < units) d[u] = v[i];
+        }
     }
 }
 

@@ -619,7 +619,7 @@ extern "C" sba_status sba_token_prune_select(const void* x, int B, int N, int C,
         return SBA_ERR_CUDA;
     double* norm2 = static_cast<double*>(workspace);
     const unsigned grid = (unsigned)((rows + sba::kNormRows - 1) / sba::kNormRows);
-    sba::token_norm_kernel<<<grid, 96, sba::kNormSmem, s>>>(tx, valid_len, N, C, rows, norm2, g_wait_limit);
+    sba::token_norm_kernel<<<grid, 160, sba::kNormSmem, s>>>(tx, valid_len, N, C, rows, norm2, g_wait_limit);
     sba::prune_select_kernel<<<(unsigned)B, 1024, 0, s>>>(norm2, valid_len, N, keep_ratio, Npad_out, idx,
                                                            valid_len_out);
     return cudaGetLastError() == cudaSuccess ? SBA_OK : SBA_ERR_CUDA;
@@ -629,6 +629,9 @@ extern "C" sba_status sba_gather_tokens(const void* src, int B, int H, int N, in
                                         const int32_t* valid_len_out, int Npad_out, void* dst, void* stream) {
     if (B <= 0 || H <= 0 || N <= 0 || Npad_out <= 0 || row_bytes <= 0) return SBA_ERR_INVALID_ARG;
     if (row_bytes % 4 != 0) return SBA_ERR_UNSUPPORTED;
+    if ((long long)B * H > 65535 || (long long)Npad_out * (row_bytes / 4) > 0x7fffffffll ||
+        (long long)N * (row_bytes / 4) > 0x7fffffffll)
+        return SBA_ERR_UNSUPPORTED;
     if (!src || !dst || !idx || !valid_len_out) return SBA_ERR_INVALID_ARG;
     const int unit = row_bytes % 16 == 0 ? 16 : 4;
     const uintptr_t am = (uintptr_t)unit - 1;
@@ -636,19 +639,14 @@ extern "C" sba_status sba_gather_tokens(const void* src, int B, int H, int N, in
         (reinterpret_cast<uintptr_t>(idx) & 3u) || (reinterpret_cast<uintptr_t>(valid_len_out) & 3u))
         return SBA_ERR_ALIGNMENT;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const long long units = (long long)B * H * Npad_out * (row_bytes / unit);
-    int dev = 0, sms = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
-        return SBA_ERR_CUDA;
-    const long long want = (units + 255) / 256;
-    const unsigned grid = (unsigned)(want < 8ll * sms ? want : 8ll * sms);
+    const long long units = (long long)Npad_out * (row_bytes / unit);   // per (b, h)
+    const dim3 grid((unsigned)((units + 4 * 256 - 1) / (4 * 256)), (unsigned)(B * H));
     const auto* sp = static_cast<const unsigned char*>(src);
     auto* dp = static_cast<unsigned char*>(dst);
     if (unit == 16)
-        sba::gather_rows_kernel<16><<<grid, 256, 0, s>>>(sp, dp, idx, valid_len_out, H, N, row_bytes, Npad_out, units);
+        sba::gather_rows_kernel<16><<<grid, 256, 0, s>>>(sp, dp, idx, valid_len_out, H, N, row_bytes, Npad_out);
     else
-        sba::gather_rows_kernel<4><<<grid, 256, 0, s>>>(sp, dp, idx, valid_len_out, H, N, row_bytes, Npad_out, units);
+        sba::gather_rows_kernel<4><<<grid, 256, 0, s>>>(sp, dp, idx, valid_len_out, H, N, row_bytes, Npad_out);
     return cudaGetLastError() == cudaSuccess ? SBA_OK : SBA_ERR_CUDA;
 }
 
