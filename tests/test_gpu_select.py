@@ -117,10 +117,11 @@ def test_valid_len_one(sba, oracle_mod):
     check_routing(sba, oracle_mod, w)
 
 
-def test_fast_rows_and_handed_back_rows_in_one_call(sba, oracle_mod):
-    """The thread-per-row top-k hands rows it cannot settle within its window (all
-    scores equal, or a tie band wider than its cache) to the warp-per-row kernel; both
-    kinds of rows side by side in one call must match the oracle."""
+def test_tie_rows_beside_ordinary_rows(sba, oracle_mod):
+    """Rows whose scores are all equal (a zero query block) and rows whose selection
+    boundary falls inside a 24-way exact tie (24 identical key blocks: a tie band wider
+    than the band cache, decided by the radix fallback) beside ordinary rows in one
+    call: every row must match the oracle."""
     rng = np.random.default_rng(23)
     w = make_custom(1, 2, 128, (4, 16, 40), 0.75, seed=24)       # 40 blocks
     q = w.q.copy()
