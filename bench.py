@@ -82,8 +82,8 @@ def parse():
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one attention launch,
 # from the ncu captures summarised in profiles/attn_kernel_*.md, and the hash
 # of the kernel sources it was taken with.  Reported only while the sources match.
-ATTN_TRAFFIC = {"480p_dense": (633137152 + 190604544, "97729a2a40a5b977"),
-                "720p": (2978964000 + 805915904, "97729a2a40a5b977"),
+ATTN_TRAFFIC = {"480p_dense": (631392000 + 186171904, "46d3116201e64454"),
+                "720p": (2972415488 + 801916160, "46d3116201e64454"),
                 "long_clip": (2696579328 + 909271552, "46d3116201e64454")}
 KERNEL_SOURCES = ("video_dit_block_b200/csrc/attention.cuh", "video_dit_block_b200/csrc/ptx.cuh",
                   "video_dit_block_b200/csrc/common.cuh")

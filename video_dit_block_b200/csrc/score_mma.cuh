@@ -102,11 +102,16 @@ __global__ void __launch_bounds__(128, 1)
     // epilogue: row r of the tile = TMEM lane r
     const bool ok = warp_wait_bounded(bar_mma, 0, abort_flag, wait_limit);
     tc_fence_after();
-    const int row = m0 + warp * 32 + lane;
     const uint32_t tl = tmem + (static_cast<uint32_t>(warp * 32) << 16);
     const bool go = __all_sync(0xffffffffu, ok && !*abort_flag);
     if (go) {
-        float* dst = scores + ((size_t)bh * nB + row) * ld + n0;
+        // Each 32 x 32 chunk of the warp's rows goes through shared memory (the operand
+        // tiles are free once the MMAs are done), so that the global stores are whole
+        // 128-byte row segments: thread t writes row t of the chunk as eight 16-byte
+        // stores, then eight lanes write each row (row stride 36 words: both phases are
+        // free of bank conflicts).
+        float* stage = reinterpret_cast<float*>(sm) + warp * (32 * 36);
+        const int rbase = m0 + warp * 32;
 #pragma unroll 1
         for (int c0 = 0; c0 < 256; c0 += 32) {
             uint32_t v[32], v2[32];
@@ -114,14 +119,24 @@ __global__ void __launch_bounds__(128, 1)
             tmem_ld32(tl + 256 + c0, v2);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) + __uint_as_float(v2[i]));
-            if (row < nB && n0 + c0 < ld) {
-                float4* d4 = reinterpret_cast<float4*>(dst + c0);
+            for (int i = 0; i < 8; ++i)
+                *reinterpret_cast<float4*>(stage + lane * 36 + 4 * i) =
+                    make_float4(__uint_as_float(v[4 * i]) + __uint_as_float(v2[4 * i]),
+                                __uint_as_float(v[4 * i + 1]) + __uint_as_float(v2[4 * i + 1]),
+                                __uint_as_float(v[4 * i + 2]) + __uint_as_float(v2[4 * i + 2]),
+                                __uint_as_float(v[4 * i + 3]) + __uint_as_float(v2[4 * i + 3]));
+            __syncwarp();
+            if (n0 + c0 < ld) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    d4[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                        __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+                for (int k = 0; k < 8; ++k) {   // four rows per pass, eight lanes per row
+                    const int r = 4 * k + lane / 8;
+                    const float4 val = *reinterpret_cast<const float4*>(stage + r * 36 + 4 * (lane % 8));
+                    if (rbase + r < nB)
+                        *reinterpret_cast<float4*>(scores + ((size_t)bh * nB + rbase + r) * ld + n0 + c0 +
+                                                   4 * (lane % 8)) = val;
+                }
             }
+            __syncwarp();
         }
     }
     tc_fence_before();
