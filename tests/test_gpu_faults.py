@@ -37,6 +37,27 @@ def test_wait_limit_expiry_reports_timeout(sba, oracle_mod):
     assert mx <= MAX_ABS and mean <= MEAN_ABS
 
 
+def test_routing_wait_limit_expiry_reports_timeout(sba):
+    """A wait of the fused screen that runs out: status 5, and the next routing call on
+    the same context gives the same lists as before."""
+    w = make_workload("tiny")
+    q, k, v, vl = to_device(w, DEV)
+    idx0, cnt0 = sba.pool_select(q, k, vl, w.sparsity)
+    assert sba.device_status() == 0
+    sba.set_wait_limit(1)
+    try:
+        sba.pool_select(q, k, vl, w.sparsity)
+        assert sba.device_status() == 5
+    finally:
+        sba.set_wait_limit(0)
+    idx, cnt = sba.pool_select(q, k, vl, w.sparsity)
+    assert sba.device_status() == 0
+    assert torch.equal(cnt, cnt0)
+    for r in np.ndindex(tuple(cnt.shape)):
+        c = int(cnt[r])
+        assert torch.equal(idx[r][:c], idx0[r][:c])
+
+
 def test_bad_routing_entry_is_flagged_and_skipped(sba):
     w = make_workload("tiny")
     q, k, v, vl = to_device(w, DEV)

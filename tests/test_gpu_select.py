@@ -135,3 +135,21 @@ def test_tie_rows_beside_ordinary_rows(sba, oracle_mod):
     w.k = k
     for s in (0.5, 0.75, 0.9):
         check_routing(sba, oracle_mod, w, s)
+
+
+def test_wide_windows_fall_back_to_the_row_routine(sba, oracle_mod):
+    """Rows with more than 64 blocks inside the fused screen's window: a zero query block
+    (every score equal over 120 blocks) and, in head 0, an 81-way exact tie that the
+    selection boundary falls into for the rows that rank it high.  Such rows leave the
+    fused kernel with their screened scores and finish in the row routine; the ordinary
+    rows of the same tiles stay in the fused kernel.  Every row must match the oracle."""
+    w = make_custom(1, 2, 128, (4, 30, 64), 0.75, seed=26)       # 120 blocks
+    q = w.q.copy()
+    q[:, :, 64 * 5:64 * 6] = 0                                      # block 5: all scores 0
+    w.q = q
+    k = w.k.copy()
+    for J in range(1, 81):
+        k[:, 0, 64 * J:64 * (J + 1)] = k[:, 0, 0:64]
+    w.k = k
+    for s in (0.5, 0.75, 0.9):
+        check_routing(sba, oracle_mod, w, s)

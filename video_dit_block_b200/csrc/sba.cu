@@ -15,6 +15,7 @@
 #include "common.cuh"
 #include "select.cuh"
 #include "score_mma.cuh"
+#include "select_fused.cuh"
 #include "score_lse.cuh"
 #include "pair.cuh"
 #include "producer.cuh"
@@ -85,6 +86,21 @@ bool make_map_2d(CUtensorMap* map, const void* base, long long rows, int cols, i
     cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// The key means of one head sampled every `stride` blocks: [BH][nB][D] bf16 viewed as
+// 3-D (D, floor(nB / stride), BH) with row pitch stride * D * 2 bytes; box 64 x 128 rows.
+bool make_map_sample(CUtensorMap* map, const void* base, int BH, int nB, int D, int stride) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)(nB / stride), (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)stride * D * 2, (cuuint64_t)nB * D * 2};
+    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
@@ -220,11 +236,13 @@ sba_status run_select(const void* q, const void* k, int B, int H, int Npad, cons
     const auto* qb = static_cast<const __nv_bfloat16*>(q);
     const auto* kb = static_cast<const __nv_bfloat16*>(k);
     const bool need_scores = sparsity > 0.0;
-    CUtensorMap tqh, tql, tkh, tkl;
-    const int brows = NSUB == 1 ? 256 : 128;  // key-side box rows of the screen
-    if (need_scores && (!make_map(&tqh, ws.qhi, (int)BH, nP, D, 128) || !make_map(&tql, ws.qlo, (int)BH, nP, D, 128) ||
-                        !make_map(&tkh, ws.khi, (int)BH, nP, D, brows) ||
-                        !make_map(&tkl, ws.klo, (int)BH, nP, D, brows)))
+    CUtensorMap tqh, tql, tkh, tkl, tks;
+    const int sample_stride = nB / 128 > 1 ? nB / 128 : 1;  // the fused screen's range sample
+    if (NSUB == 1 && BH > 65535) return SBA_ERR_UNSUPPORTED;  // grid.y of the fused screen
+    if ((need_scores || NSUB == 1) &&
+        (!make_map(&tqh, ws.qhi, (int)BH, nP, D, 128) || !make_map(&tql, ws.qlo, (int)BH, nP, D, 128) ||
+         !make_map(&tkh, ws.khi, (int)BH, nP, D, 128) || !make_map(&tkl, ws.klo, (int)BH, nP, D, 128) ||
+         (NSUB == 1 && !make_map_sample(&tks, ws.khi, (int)BH, nB, D, sample_stride))))
         return SBA_ERR_CUDA;
     if (qmean && kmean) {
         ws.qmean64 = const_cast<double*>(qmean);
@@ -238,14 +256,32 @@ sba_status run_select(const void* q, const void* k, int B, int H, int Npad, cons
                                                            ws.knorm, pgroups);
     }
     sba::kmax_kernel<<<(unsigned)((BH + 7) / 8), 256, 0, s>>>(ws, valid_len, H, Npad, (int)BH, BLK);
-    if (need_scores && NSUB == 1) {
-        using SM = sba::ScoreSmem<D>;
-        if (cudaFuncSetAttribute(sba::score_mma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 SM::kAlloc) != cudaSuccess)
+    if (NSUB == 1) {
+        // screen and top-k in one kernel; the rows it hands back finish in topk_rest_kernel
+        using SM = sba::FusedSmem<D>;
+        if (cudaFuncSetAttribute(sba::select_fused_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 SM::kAlloc) != cudaSuccess ||
+            cudaFuncSetAttribute(sba::topk_rest_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)tsmem) != cudaSuccess)
             return SBA_ERR_CUDA;
-        const dim3 sgrid((nP + 127) / 128, (nP + 255) / 256, (unsigned)BH);
-        sba::score_mma_kernel<D><<<sgrid, 128, SM::kAlloc, s>>>(tqh, tql, tkh, tkl, ws.scores, nB, ws.ld,
-                                                                g_wait_limit);
+        int dev = 0, sms = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+            return SBA_ERR_CUDA;
+        const dim3 fgrid((unsigned)((nB + 127) / 128), (unsigned)BH);
+        sba::select_fused_kernel<D><<<fgrid, sba::kFusedThreads, SM::kAlloc, s>>>(
+            tqh, tql, tkh, tkl, tks, ws, valid_len, H, Npad, sample_stride, sparsity, budget, kmax, kv_idx, kv_cnt,
+            g_wait_limit);
+        using FS = sba::FinishSmem<D>;
+        if (cudaFuncSetAttribute(sba::select_finish_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 FS::kTotal) != cudaSuccess)
+            return SBA_ERR_CUDA;
+        sba::select_finish_kernel<D><<<(unsigned)((rows + sba::kFinishWarps - 1) / sba::kFinishWarps),
+                                       32 * sba::kFinishWarps, FS::kTotal, s>>>(ws, valid_len, H, Npad, sparsity,
+                                                                               budget, kmax, kv_idx, kv_cnt, rows);
+        sba::topk_rest_kernel<D><<<(unsigned)(2 * sms), 32 * wpb, tsmem, s>>>(ws, valid_len, H, Npad, sparsity,
+                                                                              budget, kmax, kv_idx, kv_cnt);
+        return cudaGetLastError() == cudaSuccess ? SBA_OK : SBA_ERR_CUDA;
     } else if (need_scores) {
         // persistent: one CTA per SM over the (b, h, query tile) items
         using SM = sba::LseSmem<D>;

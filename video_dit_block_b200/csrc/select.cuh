@@ -35,6 +35,8 @@ constexpr int kBlock = 64;
 //   qnorm, knorm     : double [BH][nP]      Euclidean norm of each mean
 //   kmaxn            : double [BH]          largest key-mean norm of the sample
 //   scores           : float [BH][nB][ld]   screened block scores, ld = 64 * ceil(nB / 64)
+//   ovf_count, ovf_rows : int32 [1], [BH * nB]  rows left by the fused screen
+//   finish           : [BH * nB] records of fused_row_bytes(nB) bytes (fused screen)
 struct SelectWorkspace {
     double* qmean64;
     double* kmean64;
@@ -46,12 +48,22 @@ struct SelectWorkspace {
     double* knorm;
     double* kmaxn;
     float* scores;
+    int32_t* ovf_count;     // rows the fused screen hands to topk_rest_kernel
+    int32_t* ovf_rows;      // [BH * nB]
+    unsigned char* finish;  // [BH * nB] records of fused_row_bytes(nB): the fused screen's
+                            // per-row result for select_finish_kernel
     int ld;
+    int fstride;
 };
 
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 __host__ __device__ inline size_t select_score_ld(size_t nB) { return (nB + 63) / 64 * 64; }
+
+// The fused screen's per-row record: a 32-byte header, kFusedList window entries
+// (value, block) of 8 bytes, and the keep mask, four words per 128 key blocks.
+constexpr int kFusedList = 64;
+__host__ __device__ inline size_t fused_row_bytes(size_t nB) { return 32 + 8 * kFusedList + 16 * ((nB + 127) / 128); }
 
 __host__ __device__ inline size_t select_workspace_bytes(size_t BH, size_t nB, size_t D, size_t nsub = 1) {
     const size_t nP = nB * nsub;
@@ -60,7 +72,9 @@ __host__ __device__ inline size_t select_workspace_bytes(size_t BH, size_t nB, s
     const size_t nrm = align256(BH * nP * sizeof(double));
     const size_t kmx = align256(BH * sizeof(double));
     const size_t sco = align256(BH * nB * select_score_ld(nB) * sizeof(float));
-    return 2 * m64 + 4 * m16 + 2 * nrm + kmx + sco;
+    const size_t ovf = 256 + align256(BH * nB * sizeof(int32_t));
+    const size_t fin = align256(BH * nB * fused_row_bytes(nB));
+    return 2 * m64 + 4 * m16 + 2 * nrm + kmx + sco + ovf + fin;
 }
 
 __host__ __device__ inline SelectWorkspace carve_select_workspace(void* base, size_t BH, size_t nB,
@@ -83,6 +97,12 @@ __host__ __device__ inline SelectWorkspace carve_select_workspace(void* base, si
     w.kmaxn = reinterpret_cast<double*>(p); p += kmx;
     w.scores = reinterpret_cast<float*>(p);
     w.ld = (int)select_score_ld(nB);
+    p += align256(BH * nB * (size_t)w.ld * sizeof(float));
+    w.ovf_count = reinterpret_cast<int32_t*>(p);
+    w.ovf_rows = reinterpret_cast<int32_t*>(p + 256);
+    p += 256 + align256(BH * nB * sizeof(int32_t));
+    w.finish = reinterpret_cast<unsigned char*>(p);
+    w.fstride = (int)fused_row_bytes(nB);
     return w;
 }
 
@@ -475,6 +495,7 @@ __global__ void kmax_kernel(SelectWorkspace ws, const int32_t* __restrict__ vali
                             int BH, int blk) {
     const int bh = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
     const int lane = threadIdx.x & 31;
+    if (blockIdx.x == 0 && threadIdx.x == 0) *ws.ovf_count = 0;  // the fused screen counts from here
     if (bh >= BH) return;
     const int nBmax = Npad / blk;
     const int nB = (sample_len(valid_len, bh / H, Npad) + blk - 1) / blk;
@@ -530,16 +551,12 @@ __host__ __device__ inline size_t topk_smem(int warps, int ld) { return (size_t)
 // count-weighted sum of at most 16 terms (at least 1, the term of the max) to
 // 2^-19; log2 of a value below 4097 to two ulps; the last add and the product by
 // ln 2 to 2^-23 (R + 12).  The total is multiplied by 1.25 for margin.
-template <int D, int NSUB = 1>
-__global__ void __launch_bounds__(256, NSUB == 1 ? 4 : 3) topk_kernel(SelectWorkspace ws, const int32_t* __restrict__ valid_len,
-                                                   int H, int Npad, double sparsity, int budget, int kmax,
-                                                   int32_t* __restrict__ kv_idx, int32_t* __restrict__ kv_cnt,
-                                                   long long rows) {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int wpb = blockDim.x >> 5;
-    const long long rid = (long long)blockIdx.x * wpb + warp;
-    if (rid >= rows) return;
+// One routing row `rid` = (bh, I) by one warp; `wsm` is the warp's topk_warp_smem bytes.
+template <int D, int NSUB>
+__device__ void topk_row(const SelectWorkspace& ws, const int32_t* __restrict__ valid_len, int H, int Npad,
+                         double sparsity, int budget, int kmax, int32_t* __restrict__ kv_idx,
+                         int32_t* __restrict__ kv_cnt, long long rid, unsigned char* wsm) {
+    const int lane = threadIdx.x & 31;
     const int nBmax = Npad / kBlock;
     const int ld = ws.ld;
     const long long bh = rid / nBmax;
@@ -557,7 +574,7 @@ __global__ void __launch_bounds__(256, NSUB == 1 ? 4 : 3) topk_kernel(SelectWork
         if (lane == 0) kv_cnt[rid] = nB;
         return;
     }
-    float* row = reinterpret_cast<float*>(smem_raw + (size_t)warp * topk_warp_smem(ld));
+    float* row = reinterpret_cast<float*>(wsm);
     uint32_t* whist = reinterpret_cast<uint32_t*>(row + ld);
     int32_t* wslots = reinterpret_cast<int32_t*>(whist + 256);
     double* bx = reinterpret_cast<double*>(wslots + kBandCache);  // 8-byte aligned: ld % 64 == 0
@@ -800,6 +817,35 @@ __global__ void __launch_bounds__(256, NSUB == 1 ? 4 : 3) topk_kernel(SelectWork
         kv_cnt[rid] = pos;
         if (pos != k) raise_device_error(kErrBadRouting);
     }
+}
+
+template <int D, int NSUB = 1>
+__global__ void __launch_bounds__(256, NSUB == 1 ? 4 : 3) topk_kernel(SelectWorkspace ws, const int32_t* __restrict__ valid_len,
+                                                   int H, int Npad, double sparsity, int budget, int kmax,
+                                                   int32_t* __restrict__ kv_idx, int32_t* __restrict__ kv_cnt,
+                                                   long long rows) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int warp = threadIdx.x >> 5;
+    const long long rid = (long long)blockIdx.x * (blockDim.x >> 5) + warp;
+    if (rid >= rows) return;
+    topk_row<D, NSUB>(ws, valid_len, H, Npad, sparsity, budget, kmax, kv_idx, kv_cnt, rid,
+                      smem_raw + (size_t)warp * topk_warp_smem(ws.ld));
+}
+
+// The rows that the fused screen left to the row routine above: ws.ovf_rows[0 ..
+// *ws.ovf_count), their screened scores already in ws.scores.  Grid-stride over warps,
+// so the grid need not know the count.
+template <int D>
+__global__ void __launch_bounds__(256, 4) topk_rest_kernel(SelectWorkspace ws, const int32_t* __restrict__ valid_len,
+                                                           int H, int Npad, double sparsity, int budget, int kmax,
+                                                           int32_t* __restrict__ kv_idx,
+                                                           int32_t* __restrict__ kv_cnt) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int warp = threadIdx.x >> 5, wpb = blockDim.x >> 5;
+    const int n = *ws.ovf_count;
+    for (int i = blockIdx.x * wpb + warp; i < n; i += gridDim.x * wpb)
+        topk_row<D, 1>(ws, valid_len, H, Npad, sparsity, budget, kmax, kv_idx, kv_cnt, ws.ovf_rows[i],
+                       smem_raw + (size_t)warp * topk_warp_smem(ws.ld));
 }
 
 }  // namespace sba

@@ -1,0 +1,738 @@
+// select_fused.cuh -- the one-sub-block router's screen and top-k without a score matrix.
+//
+// Same selection as the block-mean routing of the page "MiniMax-H3 on 8xH200
+// benchmark", section "How SubBlock sparse attention works" (keep the best-scoring
+// keep(n, s) key blocks per query block, ties to the lower index), reached the same
+// exact way as topk_kernel (fp32 screen with a proven error bound delta, fp64
+// re-scoring of the band around the k-th value), but the screened scores live only in
+// TMEM and registers.
+//
+// select_fused_kernel.  A CTA owns 128 query blocks I = m0 + t of one (b, h): thread t
+// of warps 0-3 owns row t = TMEM lane t.  The tensor cores score the row against 128
+// key blocks at a time (a "chunk": M128 N128, S = qhi.khi + qlo.khi + qhi.klo in one
+// fp32 TMEM buffer of 128 columns, two buffers), in this order:
+//   sample   one hi.hi product against 128 key blocks spread evenly over the head
+//            gives the row a value range [vlo, vhi];
+//   pass A   every chunk: a 256-bucket histogram of the screened scores over that
+//            range (the edge buckets open), which locates the bucket [A, Bv) holding
+//            the k-th largest screened value, and its rank kk inside;
+//   pass B   every chunk again (the tensor cores give the same bits): scores at or
+//            above hiT = Bv + 2 delta are kept outright (a bitmask), scores in
+//            [A - 2 delta, hiT) -- the window -- go to a list of at most kFusedList
+//            (value, J) entries.
+// Each row then writes a record (header, window, mask) for select_finish_kernel.  A row
+// whose window overflows, or whose bound is not finite, gets a pass C instead: its screened scores go to ws.scores and
+// its index to ws.ovf_rows, and topk_rest_kernel finishes it with topk_kernel's routine.
+//
+// Warp roles (192 threads, one CTA per SM: 224 KB of shared memory for D = 128):
+//   warps 0-3  rows
+//   warp 4     TMA: Q hi/lo once, then K hi / K lo tiles through a 3-slot ring
+//   warp 5     TMEM allocation (256 columns) and the MMAs (one lane)
+// Every wait is bounded (SBA_ERR_TIMEOUT; the CTA then drains its own copies and
+// MMAs before freeing TMEM).
+//
+// select_finish_kernel, one warp per row: tau = the k-th largest screened value,
+// found among the window's entries of [A, Bv); entries above tau + 2 delta kept, below
+// tau - 2 delta dropped, the rest (the band) ordered by an fp64 dot product in any
+// order, and only the members that its error cannot separate at the cut decided on
+// exact_score (fixed sequential order), ties to the lower J; the kept blocks written in
+// ascending order from the mask.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "select.cuh"
+
+namespace sba {
+
+constexpr int kFusedThreads = 192;
+
+template <int D>
+struct FusedSmem {
+    static constexpr int kTile = 128 * D * 2;          // 128 rows of bf16 means
+    static constexpr int kSlots = 3;
+    static constexpr int kQh = 0;
+    static constexpr int kQl = kQh + kTile;
+    static constexpr int kK = kQl + kTile;
+    static constexpr int kList = kK + kSlots * kTile;  // histograms [128 words][128], then the window lists [kFusedList][128]
+    static constexpr int kListBytes = kFusedList * 128 * 8;
+    static constexpr int kBars = kList + kListBytes;   // q_full, k_full[3], k_free[3], acc_full[2], acc_empty[2], drain
+    static constexpr int kCtl = kBars + 12 * 8;        // tmem base, abort flag
+    static constexpr int kTotal = kCtl + 16;
+    static constexpr int kAlloc = kTotal + 1024;
+};
+
+// Header of a row's record in ws.finish (32 bytes); the window entries follow, then
+// the keep mask.
+struct FusedRowHead {
+    float A, Bv;   // bucket of the k-th largest screened value: [A, Bv)
+    double delta;  // screen error bound of the row
+    int32_t cnt;   // window entries; -1: the row was handed to topk_rest_kernel
+    int32_t n_sure;
+    int32_t kk;    // rank of the k-th value inside its bucket (1-based)
+    int32_t pad;
+};
+
+// Bucket of a screened value: floor((f - vlo) * bscale) clamped to [0, 255], each
+// operation rounded to nearest, so the map is non-decreasing in f.
+__device__ __forceinline__ int fused_bucket(float f, float vlo, float bscale) {
+    const int b = __float2int_rd(__fmul_rn(__fsub_rn(f, vlo), bscale));
+    return min(255, max(0, b));
+}
+
+// Smallest float x (over all non-NaN floats, in order) with fused_bucket(x) >= b, for
+// 1 <= b <= 255 and a finite bscale > 0 (then bucket(-inf) = 0 and bucket(+inf) = 255).
+__device__ float fused_bucket_edge(int b, float vlo, float bscale) {
+    uint32_t lo = f32_key(-INFINITY), hi = f32_key(INFINITY);
+    while (hi - lo > 1u) {
+        const uint32_t mid = lo + (hi - lo) / 2u;
+        if (fused_bucket(key_to_f32(mid), vlo, bscale) >= b)
+            hi = mid;
+        else
+            lo = mid;
+    }
+    return key_to_f32(hi);
+}
+
+// maps: bf16 [BH][nB][D] as 3-D (D, nB, BH), box 64 x 128 rows; tmKs views khi with
+// row stride `stride` blocks (the sample).  Grid (ceil(nB / 128), BH).
+template <int D>
+__global__ void __launch_bounds__(kFusedThreads, 1)
+    select_fused_kernel(const __grid_constant__ CUtensorMap tmQh, const __grid_constant__ CUtensorMap tmQl,
+                        const __grid_constant__ CUtensorMap tmKh, const __grid_constant__ CUtensorMap tmKl,
+                        const __grid_constant__ CUtensorMap tmKs, SelectWorkspace ws,
+                        const int32_t* __restrict__ valid_len, int H, int Npad, int stride, double sparsity,
+                        int budget, int kmax, int32_t* __restrict__ kv_idx, int32_t* __restrict__ kv_cnt,
+                        unsigned long long wait_limit) {
+    using SM = FusedSmem<D>;
+    constexpr int NCH = D / 64;
+    constexpr uint32_t kIdesc = idesc_bf16_f32(128, 128, 0, 0);
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* sm = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int nBmax = Npad / kBlock;
+    const int m0 = blockIdx.x * 128, bh = blockIdx.y;
+    const int L = sample_len(valid_len, bh / H, Npad);
+    const int nBb = (L + kBlock - 1) / kBlock;
+    const int k = keep_count_budget(nBb, sparsity, budget);
+
+    // ---- nothing dropped: every block, ascending; no tensor work.  (Rows I >= nBb
+    // of other tiles are left to select_finish_kernel.)
+    if (k >= nBb || m0 >= nBb) {
+        if (k >= nBb) {
+            for (int r = warp; r < 128 && m0 + r < nBmax; r += kFusedThreads / 32) {
+                const size_t rid = (size_t)bh * nBmax + m0 + r;
+                const int n = m0 + r < nBb ? nBb : 0;
+                for (int j = lane; j < n; j += 32) kv_idx[rid * kmax + j] = j;
+                if (lane == 0) kv_cnt[rid] = n;
+            }
+        }
+        return;
+    }
+
+    const uint32_t sQh = smem_u32(sm + SM::kQh), sQl = smem_u32(sm + SM::kQl), sK = smem_u32(sm + SM::kK);
+    const uint32_t bars = smem_u32(sm + SM::kBars);
+    const uint32_t q_full = bars, k_full = bars + 8, k_free = bars + 32, acc_full = bars + 56,
+                   acc_empty = bars + 72, drain_bar = bars + 88;
+    uint32_t* ctl = reinterpret_cast<uint32_t*>(sm + SM::kCtl);
+    volatile uint32_t* abort_flag = ctl + 1;
+    const int nC = (nBb + 127) / 128;  // chunks of this sample's key blocks
+
+    if (tid == 0) {
+        mbar_init(q_full, 1);
+        for (int i = 0; i < 3; ++i) {
+            mbar_init(k_full + 8 * i, 1);
+            mbar_init(k_free + 8 * i, 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(acc_full + 8 * i, 1);
+            mbar_init(acc_empty + 8 * i, 4);
+        }
+        mbar_init(drain_bar, 1);
+        *abort_flag = 0u;
+        fence_barrier_init();
+    }
+    if (warp == 5) tmem_alloc(smem_u32(ctl), 256);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ctl[0];
+
+    bool any_fallback = false;
+    if (warp == 4) {
+        // ------------------------------------------------------------ TMA producer
+        int g = 0;  // K tiles issued
+        auto load_k = [&](const CUtensorMap* map, int row) -> bool {
+            const int slot = g % 3;
+            if (g >= 3 && !wait_bounded(k_free + 8 * slot, ((g / 3) - 1) & 1, abort_flag, wait_limit)) return false;
+            mbar_arrive_expect_tx(k_full + 8 * slot, SM::kTile);
+            for (int c = 0; c < NCH; ++c)
+                tma_load_3d(sK + slot * SM::kTile + c * (128 * 128), map, k_full + 8 * slot, c * 64, row, bh);
+            ++g;
+            return true;
+        };
+        auto load_passes = [&](int npass) {
+            for (int p = 0; p < npass; ++p)
+                for (int ch = 0; ch < nC; ++ch)
+                    if (!load_k(&tmKh, ch * 128) || !load_k(&tmKl, ch * 128)) return;
+        };
+        if (lane == 0) {
+            mbar_arrive_expect_tx(q_full, 2 * SM::kTile);
+            for (int c = 0; c < NCH; ++c) {
+                tma_load_3d(sQh + c * (128 * 128), &tmQh, q_full, c * 64, m0, bh);
+                tma_load_3d(sQl + c * (128 * 128), &tmQl, q_full, c * 64, m0, bh);
+            }
+            if (load_k(&tmKs, 0)) load_passes(2);
+        }
+        __syncwarp();
+        any_fallback = __syncthreads_or(0);
+        if (any_fallback && lane == 0 && !*abort_flag) load_passes(1);
+        __syncwarp();
+        if (*abort_flag && lane == 0) {
+            // let the copies this CTA issued land before the CTA exits
+            const long long t0 = clock64();
+            while (!mbar_try_wait(q_full, 0) && (uint64_t)(clock64() - t0) < (1ull << 32)) {}
+            for (int i = g - 3 < 0 ? 0 : g - 3; i < g; ++i) {
+                const long long t1 = clock64();
+                while (!mbar_try_wait(k_full + 8 * (i % 3), (i / 3) & 1) && (uint64_t)(clock64() - t1) < (1ull << 32)) {}
+            }
+        }
+    } else if (warp == 5) {
+        // ------------------------------------------------------------ MMA issuer
+        int g = 0, a = 0;  // K tiles consumed, accumulator uses
+        auto acquire = [&](uint32_t& d) -> bool {
+            const int buf = a & 1;
+            if (a >= 2 && !poll_bounded(acc_empty + 8 * buf, ((a >> 1) - 1) & 1, abort_flag, wait_limit)) return false;
+            d = tmem + 128u * buf;
+            return true;
+        };
+        auto product = [&](uint32_t d, uint32_t A, uint32_t B, bool first) {
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint64_t ad = smem_desc_sw128(A + (kk / 4) * (128 * 128) + (kk % 4) * 32, 16, 1024);
+                const uint64_t bd = smem_desc_sw128(B + (kk / 4) * (128 * 128) + (kk % 4) * 32, 16, 1024);
+                mma_bf16_ss(d, ad, bd, kIdesc, (first && kk == 0) ? 0u : 1u);
+            }
+        };
+        auto chunk = [&]() -> bool {
+            uint32_t d;
+            if (!acquire(d)) return false;
+            const int hs = g % 3, ls = (g + 1) % 3;
+            if (!poll_bounded(k_full + 8 * hs, (g / 3) & 1, abort_flag, wait_limit)) return false;
+            tc_fence_after();
+            product(d, sQh, sK + hs * SM::kTile, true);   // hi.hi
+            product(d, sQl, sK + hs * SM::kTile, false);  // lo.hi
+            mma_commit(k_free + 8 * hs);
+            if (!poll_bounded(k_full + 8 * ls, ((g + 1) / 3) & 1, abort_flag, wait_limit)) return false;
+            tc_fence_after();
+            product(d, sQh, sK + ls * SM::kTile, false);  // hi.lo
+            mma_commit(k_free + 8 * ls);
+            mma_commit(acc_full + 8 * (a & 1));
+            g += 2;
+            ++a;
+            return true;
+        };
+        auto passes = [&](int npass) {
+            for (int p = 0; p < npass; ++p)
+                for (int ch = 0; ch < nC; ++ch)
+                    if (!chunk()) return;
+        };
+        if (lane == 0 && wait_bounded(q_full, 0, abort_flag, wait_limit)) {
+            uint32_t d;
+            if (acquire(d) && poll_bounded(k_full, 0, abort_flag, wait_limit)) {
+                tc_fence_after();
+                product(d, sQh, sK, true);  // the sample: hi.hi only
+                mma_commit(k_free);
+                mma_commit(acc_full);
+                g = 1;
+                a = 1;
+                passes(2);
+            }
+        }
+        __syncwarp();
+        any_fallback = __syncthreads_or(0);
+        if (any_fallback && lane == 0 && !*abort_flag) passes(1);
+        __syncwarp();
+        if (*abort_flag && lane == 0) {
+            mma_commit(drain_bar);  // arrives once every MMA issued above is done
+            const long long t0 = clock64();
+            while (!mbar_try_wait(drain_bar, 0) && (uint64_t)(clock64() - t0) < (1ull << 32)) {}
+        }
+    } else {
+        // ------------------------------------------------------------ rows
+        const int t = tid;  // 0..127
+        const int I = m0 + t;
+        const bool active = I < nBb;
+        const long long rid = (long long)bh * nBmax + I;
+        const uint32_t tl = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+        float2* list = reinterpret_cast<float2*>(sm + SM::kList);  // [kFusedList][128] (value, J as int bits)
+        const uint32_t list_s = smem_u32(list) + 8u * t;
+        unsigned char* rec = ws.finish + (size_t)rid * ws.fstride;
+        int a = 0;
+        bool ok = true;
+        // The next accumulator use is read 32 columns (a "part") at a time: wait_acc waits
+        // for it, load_part(s, v) loads columns [32 s, 32 s + 32) and, after the last
+        // part, hands the buffer back to the MMA warp.  (Loops over parts keep the code
+        // small; a fully unrolled chunk does not fit the instruction cache.)
+        int buf = 0;
+        auto wait_acc = [&]() -> bool {
+            buf = a & 1;
+            const bool got = warp_wait_bounded(acc_full + 8 * buf, (a >> 1) & 1, abort_flag, wait_limit);
+            ++a;
+            if (got) tc_fence_after();
+            return got;
+        };
+        auto load_part = [&](int part, uint32_t (&v)[32]) {
+            tmem_ld32(tl + 128u * buf + 32u * part, v);
+            tmem_wait_ld();
+            if (part == 3) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(acc_empty + 8 * buf);
+            }
+        };
+        uint32_t* hist = reinterpret_cast<uint32_t*>(sm + SM::kList);  // histograms, then the lists
+        const uint32_t hist_s = smem_u32(hist) + 4u * t;
+
+        // ---- sample: the row's value range [vlo, vlo + 256 / bscale]
+        float vlo = 0.f, bscale = 0.f;
+        ok = wait_acc();
+        if (ok) {
+            float lo = INFINITY, hi = -INFINITY;
+#pragma unroll 1
+            for (int part = 0; part < 4; ++part) {
+                uint32_t v[32];
+                load_part(part, v);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const bool in = (long long)stride * (32 * part + i) < nBb;
+                    lo = in ? fminf(lo, __uint_as_float(v[i])) : lo;
+                    hi = in ? fmaxf(hi, __uint_as_float(v[i])) : hi;
+                }
+            }
+            const float range = hi - lo;
+            if (range > 0.f && range <= 3.0e38f) {
+                const float sc = 256.0f / range;
+                if (sc <= 3.0e38f) {
+                    vlo = lo;
+                    bscale = sc;
+                }
+            }
+        }
+        for (int w = 0; w < 128; ++w) hist[w * 128 + t] = 0u;
+
+        // ---- pass A: 256-bucket histogram of the row's screened scores
+        for (int ch = 0; ch < nC && ok; ++ch) {
+            if (!(ok = wait_acc())) break;
+            const int lim = active ? nBb - ch * 128 : 0;  // columns < lim are blocks of the sample
+#pragma unroll 1
+            for (int part = 0; part < 4; ++part) {
+                uint32_t v[32];
+                load_part(part, v);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int b = fused_bucket(__uint_as_float(v[i]), vlo, bscale);
+                    red_add_shared_if(32 * part + i < lim, hist_s + (uint32_t)(b >> 1) * 512u, 1u << ((b & 1) << 4));
+                }
+            }
+        }
+
+        // ---- the bucket [A, Bv) of the k-th largest value, its rank kk inside, and the
+        // window around it
+        double delta = INFINITY;
+        int kk = 0;
+        float A = -INFINITY, Bv = INFINITY, hiT = INFINITY, loT = -INFINITY;
+        bool fallback = false;
+        if (active && ok) {
+            int cum = 0, bstar = -1;
+            // buckets from the top, 16 words (32 buckets) loaded at a time
+            for (int w0 = 112; w0 >= 0 && bstar < 0; w0 -= 16) {
+                uint32_t words[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) words[i] = hist[(w0 + i) * 128 + t];
+#pragma unroll
+                for (int i = 15; i >= 0; --i) {
+                    const int c1 = (int)(words[i] >> 16), c0 = (int)(words[i] & 0xFFFFu);
+                    if (bstar < 0) {
+                        if (cum + c1 >= k) {
+                            bstar = 2 * (w0 + i) + 1;
+                        } else {
+                            cum += c1;
+                            if (cum + c0 >= k)
+                                bstar = 2 * (w0 + i);
+                            else
+                                cum += c0;
+                        }
+                    }
+                }
+            }
+            kk = k - cum;  // 1 <= kk <= the bucket's count
+            const double qn = ws.qnorm[(size_t)rid];
+            const double kmx = ws.kmaxn[bh];
+            delta = 2.0 * (4.0 * 0x1p-16 + 3.0 * D * 0x1p-22) * qn * kmx + 3.0 * D * 0x1p-120 * (1.0 + qn + kmx);
+            // a bound that is not meaningful in fp32 goes to the row routine
+            fallback = bstar < 0 || !(qn * kmx < 1.0e30) || !(delta < 1.0e30);
+            if (!fallback) {
+                if (bscale > 0.f) {
+                    if (bstar > 0) A = fused_bucket_edge(bstar, vlo, bscale);
+                    if (bstar < 255) Bv = fused_bucket_edge(bstar + 1, vlo, bscale);
+                }
+                if (Bv < INFINITY) hiT = __double2float_ru((double)Bv + 2.0 * delta);
+                if (A > -INFINITY) loT = __double2float_rd((double)A - 2.0 * delta);
+            }
+        }
+        named_bar_sync(1, 128);  // histograms read: the lists may overwrite them
+
+        // ---- pass B: sure keeps into the row's mask, the window into the list
+        int cnt = 0, n_sure = 0;
+        const bool collect = active && !fallback;
+        for (int ch = 0; ch < nC && ok; ++ch) {
+            if (!(ok = wait_acc())) break;
+            const int j0 = ch * 128;
+            const int lim = collect ? nBb - j0 : 0;
+#pragma unroll 1
+            for (int part = 0; part < 4; ++part) {
+                uint32_t v[32];
+                load_part(part, v);
+                uint32_t word = 0u;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float f = __uint_as_float(v[i]);
+                    const bool in = 32 * part + i < lim;
+                    word |= (in && f >= hiT) ? 1u << i : 0u;
+                    const bool win = in && f >= loT && f < hiT;
+                    if (__any_sync(0xffffffffu, win))  // rare: no shared-memory traffic otherwise
+                        st_shared_v2_if(win, list_s + (uint32_t)min(cnt, kFusedList - 1) * 1024u, v[i],
+                                        (uint32_t)(j0 + 32 * part + i));
+                    cnt += win ? 1 : 0;
+                }
+                if (collect) {
+                    n_sure += __popc(word);
+                    *reinterpret_cast<uint32_t*>(rec + 32 + 8 * kFusedList + 16 * ch + 4 * part) = word;
+                }
+            }
+        }
+        if (collect && cnt > kFusedList) fallback = true;
+        any_fallback = __syncthreads_or(active && fallback && ok);
+
+        // ---- pass C (only when some row of the tile fell back): its screened scores
+        if (any_fallback && ok) {
+            for (int ch = 0; ch < nC && ok; ++ch) {
+                if (!(ok = wait_acc())) break;
+#pragma unroll 1
+                for (int part = 0; part < 4; ++part) {
+                    uint32_t v[32];
+                    load_part(part, v);
+                    if (active && fallback) {
+                        float* dst = ws.scores + (size_t)rid * ws.ld + ch * 128 + 32 * part;
+#pragma unroll
+                        for (int i = 0; i < 32; i += 4)
+                            if (ch * 128 + 32 * part + i + 4 <= ws.ld)
+                                *reinterpret_cast<float4*>(dst + i) =
+                                    make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]),
+                                                __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
+                    }
+                }
+            }
+            if (ok && active && fallback) ws.ovf_rows[atomicAdd(ws.ovf_count, 1)] = (int32_t)rid;
+        }
+        if (!__all_sync(0xffffffffu, ok)) ok = false;
+
+        // ---- the record: header, then (warp by warp, coalesced) the window entries
+        if (ok && active) {
+            FusedRowHead h;
+            h.A = A;
+            h.Bv = Bv;
+            h.delta = delta;
+            h.cnt = fallback ? -1 : cnt;
+            h.n_sure = n_sure;
+            h.kk = kk;
+            h.pad = 0;
+            *reinterpret_cast<FusedRowHead*>(rec) = h;
+        }
+        const int n_copy = (ok && active && !fallback) ? cnt : 0;
+        for (int r = 0; r < 32; ++r) {
+            const int row = warp * 32 + r;
+            const int n = __shfl_sync(0xffffffffu, n_copy, r);
+            float2* dst = reinterpret_cast<float2*>(ws.finish + ((size_t)bh * nBmax + m0 + row) * ws.fstride + 32);
+            for (int e = lane; e < n; e += 32) dst[e] = list[e * 128 + row];
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+// ------------------------------------------------------------------ finish
+constexpr int kFinishWarps = 8;
+
+// Shared-memory bytes per warp: the band's refined and exact scores and blocks, the
+// blocks kept beyond the mask, and the row's mask words.
+template <int D>
+struct FinishSmem {
+    static constexpr int kR = 0;                       // double [64] refined band scores
+    static constexpr int kX = kR + kFusedList * 8;     // double [64] exact scores (or blocks)
+    static constexpr int kJ = kX + kFusedList * 8;     // int [64] band blocks
+    static constexpr int kE = kJ + kFusedList * 4;     // int [64] extra kept blocks
+    static constexpr int kW = kE + kFusedList * 4;     // uint32 [128] mask words
+    static constexpr int kWarp = kW + 128 * 4;
+    static constexpr int kTotal = kFinishWarps * kWarp;
+};
+
+// One routing row per warp from its record (see the file comment).  Rows of samples
+// that keep every block were written by select_fused_kernel; rows past the sample's
+// blocks get kv_cnt = 0 here; rows handed to topk_rest_kernel are skipped.
+template <int D>
+__global__ void __launch_bounds__(32 * kFinishWarps) select_finish_kernel(SelectWorkspace ws,
+                                                                          const int32_t* __restrict__ valid_len,
+                                                                          int H, int Npad, double sparsity, int budget,
+                                                                          int kmax, int32_t* __restrict__ kv_idx,
+                                                                          int32_t* __restrict__ kv_cnt, long long rows) {
+    using FS = FinishSmem<D>;
+    extern __shared__ __align__(16) unsigned char fsm_raw[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long rid = (long long)blockIdx.x * kFinishWarps + warp;
+    if (rid >= rows) return;
+    unsigned char* wsm = fsm_raw + warp * FS::kWarp;
+    const int nBmax = Npad / kBlock;
+    const long long bh = rid / nBmax;
+    const int I = (int)(rid % nBmax);
+    const int L = sample_len(valid_len, (int)(bh / H), Npad);
+    const int nBb = (L + kBlock - 1) / kBlock;
+    const int k = keep_count_budget(nBb, sparsity, budget);
+    if (I >= nBb) {
+        if (lane == 0) kv_cnt[rid] = 0;
+        return;
+    }
+    if (k >= nBb) return;
+    const unsigned char* rec = ws.finish + (size_t)rid * ws.fstride;
+    const FusedRowHead h = *reinterpret_cast<const FusedRowHead*>(rec);
+    if (h.cnt < 0) return;
+    const int cnt = min(h.cnt, kFusedList);
+    const float2* ent = reinterpret_cast<const float2*>(rec + 32);
+
+    // ---- the window: lane holds entries lane and lane + 32
+    float f[2];
+    int jb[2];
+    bool has[2], mem[2];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+        const int e = lane + 32 * q;
+        has[q] = e < cnt;
+        const float2 x = has[q] ? ent[e] : make_float2(0.f, 0.f);
+        f[q] = x.x;
+        jb[q] = __float_as_int(x.y);
+        mem[q] = has[q] && f[q] >= h.A && f[q] < h.Bv;
+    }
+    // a record not written by this call (its screen aborted) must not send us out of bounds
+    if (__any_sync(0xffffffffu, (has[0] && (jb[0] < 0 || jb[0] >= nBb)) || (has[1] && (jb[1] < 0 || jb[1] >= nBb)))) {
+        if (lane == 0) raise_device_error(kErrBadRouting);
+        return;
+    }
+    // tau: the kk-th largest member of the bucket
+    int gt[2] = {0, 0}, ge[2] = {0, 0};
+    for (int u = 0; u < cnt; ++u) {
+        const float fu = __shfl_sync(0xffffffffu, u < 32 ? f[0] : f[1], u & 31);
+        const bool mu = __shfl_sync(0xffffffffu, u < 32 ? mem[0] : mem[1], u & 31);
+        if (mu) {
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                gt[q] += fu > f[q] ? 1 : 0;
+                ge[q] += fu >= f[q] ? 1 : 0;
+            }
+        }
+    }
+    const bool hit0 = mem[0] && gt[0] < h.kk && h.kk <= ge[0];
+    const bool hit1 = mem[1] && gt[1] < h.kk && h.kk <= ge[1];
+    const uint32_t hb0 = __ballot_sync(0xffffffffu, hit0), hb1 = __ballot_sync(0xffffffffu, hit1);
+    if (!hb0 && !hb1) {  // cannot happen when both passes saw the same scores
+        if (lane == 0) raise_device_error(kErrBadRouting);
+        return;
+    }
+    const float tau =
+        hb0 ? __shfl_sync(0xffffffffu, f[0], __ffs(hb0) - 1) : __shfl_sync(0xffffffffu, f[1], __ffs(hb1) - 1);
+    const float hi2 = __double2float_ru((double)tau + 2.0 * h.delta);
+    const float lo2 = __double2float_rd((double)tau - 2.0 * h.delta);
+    bool keep[2], band[2];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+        keep[q] = has[q] && f[q] > hi2;
+        band[q] = has[q] && !keep[q] && f[q] >= lo2;
+    }
+    const uint32_t kb0 = __ballot_sync(0xffffffffu, keep[0]), kb1 = __ballot_sync(0xffffffffu, keep[1]);
+    const uint32_t bb0 = __ballot_sync(0xffffffffu, band[0]), bb1 = __ballot_sync(0xffffffffu, band[1]);
+    const int n_in = h.n_sure + __popc(kb0) + __popc(kb1);
+    const int n_band = __popc(bb0) + __popc(bb1);
+    const int need = k - n_in;  // 1 <= need <= n_band
+
+    int* xj = reinterpret_cast<int*>(wsm + FS::kE);  // blocks kept beyond the mask
+    int n_extra = 0;
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {  // window entries above the band
+        const uint32_t kb = q ? kb1 : kb0;
+        if (keep[q]) xj[n_extra + __popc(kb & lanemask_lt())] = jb[q];
+        n_extra += __popc(kb);
+    }
+    if (need >= n_band) {
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const uint32_t bb = q ? bb1 : bb0;
+            if (band[q]) xj[n_extra + __popc(bb & lanemask_lt())] = jb[q];
+            n_extra += __popc(bb);
+        }
+    } else {
+        // The band in fp64.  First every member's dot product q.k_J in any order (lanes
+        // over channels, fused multiply-adds, a butterfly): r_m.  It and exact_score
+        // (the fixed sequential order) are each within (D + 2) 2^-53 sum_d |q_d k_d|
+        // <= (D + 2) 2^-53 |q| max|k| of the true product, so members whose r differ by
+        // more than 2 eps are ordered by r; only those within 2 eps of the cut are
+        // decided on exact_score, ties to the lower J.
+        double* rx = reinterpret_cast<double*>(wsm + FS::kR);
+        double* ex = reinterpret_cast<double*>(wsm + FS::kX);
+        int* bj = reinterpret_cast<int*>(wsm + FS::kJ);
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const uint32_t bb = q ? bb1 : bb0;
+            const int base = q ? __popc(bb0) : 0;
+            if (band[q]) bj[base + __popc(bb & lanemask_lt())] = jb[q];
+        }
+        __syncwarp();
+        const double* qrow = ws.qmean64 + (size_t)rid * D;
+        const double* kbase = ws.kmean64 + (size_t)bh * nBmax * D;
+        const double inv = __ddiv_rn(1.0, __dsqrt_rn((double)D));
+        double qd[D / 32];
+#pragma unroll
+        for (int i = 0; i < D / 32; ++i) qd[i] = qrow[lane + 32 * i];
+        for (int m = 0; m < n_band; m += 2) {  // two members per step: more loads in flight
+            const double* k0 = kbase + (size_t)bj[m] * D;
+            const double* k1 = kbase + (size_t)bj[m + 1 < n_band ? m + 1 : m] * D;
+            double p0 = 0.0, p1 = 0.0;
+#pragma unroll
+            for (int i = 0; i < D / 32; ++i) {
+                p0 = fma(qd[i], k0[lane + 32 * i], p0);
+                p1 = fma(qd[i], k1[lane + 32 * i], p1);
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                p0 += __shfl_xor_sync(0xffffffffu, p0, off);
+                p1 += __shfl_xor_sync(0xffffffffu, p1, off);
+            }
+            if (lane == 0) {
+                rx[m] = p0 * inv;
+                if (m + 1 < n_band) rx[m + 1] = p1 * inv;
+            }
+        }
+        __syncwarp();
+        const double qn = ws.qnorm[(size_t)rid], kmx = ws.kmaxn[bh];
+        const double eps = 2.0 * (D + 4.0) * 0x1p-53 * qn * kmx * inv + 0x1p-1000;
+        // r_cut: the need-th largest r
+        double r_cut = 0.0;
+        bool got = false;
+        for (int r0 = 0; r0 < n_band; r0 += 32) {
+            const int m = r0 + lane;
+            bool hit = false;
+            double rm = 0.0;
+            if (m < n_band) {
+                rm = rx[m];
+                int gt = 0, ge = 0;
+                for (int u = 0; u < n_band; ++u) {
+                    gt += rx[u] > rm ? 1 : 0;
+                    ge += rx[u] >= rm ? 1 : 0;
+                }
+                hit = gt < need && need <= ge;
+            }
+            const uint32_t hb = __ballot_sync(0xffffffffu, hit);
+            if (hb && !got) {
+                r_cut = __shfl_sync(0xffffffffu, rm, __ffs(hb) - 1);
+                got = true;
+            }
+        }
+        const double hiC = r_cut + 2.0 * eps, loC = r_cut - 2.0 * eps;
+        // above the cut: kept; at the cut: to decide exactly
+        int n_top = 0, n_tie = 0;
+        for (int r0 = 0; r0 < n_band; r0 += 32) {
+            const int m = r0 + lane;
+            const double rm = m < n_band ? rx[m] : -INFINITY;
+            const bool top = m < n_band && rm > hiC;
+            const bool tie = m < n_band && !top && rm >= loC;
+            const uint32_t tb = __ballot_sync(0xffffffffu, top);
+            if (top) xj[n_extra + __popc(tb & lanemask_lt())] = bj[m];
+            n_extra += __popc(tb);
+            n_top += __popc(tb);
+            const uint32_t eb = __ballot_sync(0xffffffffu, tie);
+            if (tie) ex[n_tie + __popc(eb & lanemask_lt())] = __longlong_as_double((long long)bj[m]);
+            n_tie += __popc(eb);
+        }
+        __syncwarp();
+        const int slots = need - n_top;  // 1 <= slots <= n_tie
+        if (slots >= n_tie) {
+            for (int e = lane; e < n_tie; e += 32) xj[n_extra + e] = (int)__double_as_longlong(ex[e]);
+            n_extra += n_tie;
+        } else {
+            // exact_score for the members at the cut (rare: near-equal scores)
+            int* tj = bj;  // reuse: the band's blocks are no longer needed
+            for (int e = lane; e < n_tie; e += 32) tj[e] = (int)__double_as_longlong(ex[e]);
+            __syncwarp();
+            for (int e = lane; e < n_tie; e += 32) ex[e] = exact_score(qrow, kbase + (size_t)tj[e] * D, D, inv);
+            __syncwarp();
+            for (int r0 = 0; r0 < n_tie; r0 += 32) {
+                const int m = r0 + lane;
+                bool kept = false;
+                if (m < n_tie) {
+                    const double xm = ex[m];
+                    const int jm = tj[m];
+                    int rank = 0;
+                    for (int u = 0; u < n_tie; ++u)
+                        rank += (ex[u] > xm || (ex[u] == xm && tj[u] < jm)) ? 1 : 0;
+                    kept = rank < slots;
+                }
+                const uint32_t kbm = __ballot_sync(0xffffffffu, kept);
+                if (kept) xj[n_extra + __popc(kbm & lanemask_lt())] = tj[m];
+                n_extra += __popc(kbm);
+            }
+        }
+    }
+    __syncwarp();
+
+    // ---- the mask plus the extra blocks, written in ascending order
+    uint32_t* words = reinterpret_cast<uint32_t*>(wsm + FS::kW);
+    const int W = (nBb + 31) / 32;
+    const uint32_t* mw = reinterpret_cast<const uint32_t*>(rec + 32 + 8 * kFusedList);
+    for (int w = lane; w < W; w += 32) words[w] = mw[w];
+    __syncwarp();
+    for (int e = lane; e < n_extra; e += 32) atomicOr(&words[xj[e] >> 5], 1u << (xj[e] & 31));
+    __syncwarp();
+    int32_t* out = kv_idx + (size_t)rid * kmax;
+    int pos = 0;
+    for (int w0 = 0; w0 < W; w0 += 32) {
+        uint32_t word = w0 + lane < W ? words[w0 + lane] : 0u;
+        const int c = __popc(word);
+        int incl = c;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += y;
+        }
+        int p = pos + incl - c;
+        while (word) {
+            const int bit = __ffs(word) - 1;
+            word &= word - 1;
+            if (p < kmax) out[p] = 32 * (w0 + lane) + bit;
+            ++p;
+        }
+        pos += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) {
+        kv_cnt[rid] = pos;
+        if (pos != k) raise_device_error(kErrBadRouting);
+    }
+}
+
+}  // namespace sba
