@@ -62,7 +62,7 @@ __host__ __device__ inline size_t select_score_ld(size_t nB) { return (nB + 63) 
 
 // The fused screen's per-row record: a 32-byte header, kFusedList window entries
 // (value, block) of 8 bytes, and the keep mask, four words per 128 key blocks.
-constexpr int kFusedList = 64;
+constexpr int kFusedList = 56;
 __host__ __device__ inline size_t fused_row_bytes(size_t nB) { return 32 + 8 * kFusedList + 16 * ((nB + 127) / 128); }
 
 __host__ __device__ inline size_t select_workspace_bytes(size_t BH, size_t nB, size_t D, size_t nsub = 1) {

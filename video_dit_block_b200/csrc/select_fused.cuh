@@ -24,10 +24,12 @@
 // whose window overflows, or whose bound is not finite, gets a pass C instead: its screened scores go to ws.scores and
 // its index to ws.ovf_rows, and topk_rest_kernel finishes it with topk_kernel's routine.
 //
-// Warp roles (192 threads, one CTA per SM: 224 KB of shared memory for D = 128):
-//   warps 0-3  rows
-//   warp 4     TMA: Q hi/lo once, then K hi / K lo tiles through a 3-slot ring
-//   warp 5     TMEM allocation (256 columns) and the MMAs (one lane)
+// Warp roles (576 threads, one CTA per SM: 224 KB of shared memory for D = 128):
+//   warps 0-15 rows: warp w reads TMEM lanes 32 (w mod 4) .. + 31 and columns 32 (w / 4)
+//              .. + 31 of each chunk, so four threads share a row (its histogram by
+//              shared-memory atomics, its window by an atomic slot counter)
+//   warp 16    TMA: Q hi/lo once, then K hi / K lo tiles through a 3-slot ring
+//   warp 17    TMEM allocation (256 columns) and the MMAs (one lane)
 // Every wait is bounded (SBA_ERR_TIMEOUT; the CTA then drains its own copies and
 // MMAs before freeing TMEM).
 //
@@ -47,7 +49,9 @@
 
 namespace sba {
 
-constexpr int kFusedThreads = 192;
+constexpr int kFusedRowWarps = 16;  // four per 32-lane group of TMEM, 32 columns each
+constexpr int kFusedThreads = 32 * kFusedRowWarps + 64;
+constexpr int kProducerWarp = kFusedRowWarps, kMmaWarp = kFusedRowWarps + 1;
 
 template <int D>
 struct FusedSmem {
@@ -56,12 +60,16 @@ struct FusedSmem {
     static constexpr int kQh = 0;
     static constexpr int kQl = kQh + kTile;
     static constexpr int kK = kQl + kTile;
-    static constexpr int kList = kK + kSlots * kTile;  // histograms [128 words][128], then the window lists [kFusedList][128]
+    // histograms [128 words][128 rows] during pass A; then the window lists
+    // [kFusedList][128], the rows' FusedRowInfo and their list counters
+    static constexpr int kList = kK + kSlots * kTile;
     static constexpr int kListBytes = kFusedList * 128 * 8;
-    static constexpr int kBars = kList + kListBytes;   // q_full, k_full[3], k_free[3], acc_full[2], acc_empty[2], drain
+    static constexpr int kRegionBytes = 128 * 128 * 4;
+    static constexpr int kBars = kList + kRegionBytes;   // q_full, k_full[3], k_free[3], acc_full[2], acc_empty[2], drain
     static constexpr int kCtl = kBars + 12 * 8;        // tmem base, abort flag
     static constexpr int kTotal = kCtl + 16;
     static constexpr int kAlloc = kTotal + 1024;
+    static_assert(kListBytes + 128 * 32 + 128 * 4 <= kRegionBytes, "lists, row info and counters share the region");
 };
 
 // Header of a row's record in ws.finish (32 bytes); the window entries follow, then
@@ -70,9 +78,16 @@ struct FusedRowHead {
     float A, Bv;   // bucket of the k-th largest screened value: [A, Bv)
     double delta;  // screen error bound of the row
     int32_t cnt;   // window entries; -1: the row was handed to topk_rest_kernel
-    int32_t n_sure;
     int32_t kk;    // rank of the k-th value inside its bucket (1-based)
-    int32_t pad;
+    int32_t pad[2];
+};
+
+// What the row's thread of part 0 publishes for the row's other three threads.
+struct FusedRowInfo {
+    float A, Bv, hiT, loT;
+    double delta;
+    int32_t kk;
+    int32_t flags;  // 1: collect the window; 2: hand the row to topk_rest_kernel
 };
 
 // Bucket of a screened value: floor((f - vlo) * bscale) clamped to [0, 255], each
@@ -149,20 +164,20 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(acc_full + 8 * i, 1);
-            mbar_init(acc_empty + 8 * i, 4);
+            mbar_init(acc_empty + 8 * i, kFusedRowWarps);
         }
         mbar_init(drain_bar, 1);
         *abort_flag = 0u;
         fence_barrier_init();
     }
-    if (warp == 5) tmem_alloc(smem_u32(ctl), 256);
+    if (warp == kMmaWarp) tmem_alloc(smem_u32(ctl), 256);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ctl[0];
 
     bool any_fallback = false;
-    if (warp == 4) {
+    if (warp == kProducerWarp) {
         // ------------------------------------------------------------ TMA producer
         int g = 0;  // K tiles issued
         auto load_k = [&](const CUtensorMap* map, int row) -> bool {
@@ -200,7 +215,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 while (!mbar_try_wait(k_full + 8 * (i % 3), (i / 3) & 1) && (uint64_t)(clock64() - t1) < (1ull << 32)) {}
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         int g = 0, a = 0;  // K tiles consumed, accumulator uses
         auto acquire = [&](uint32_t& d) -> bool {
@@ -263,55 +278,64 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         }
     } else {
         // ------------------------------------------------------------ rows
-        const int t = tid;  // 0..127
+        // Warp w serves rows 32 (w mod 4) .. + 31 (its TMEM lanes) and columns
+        // 32 part .. + 31 of every chunk, part = w / 4: four threads per row.
+        const int part = warp >> 2;
+        const int t = 32 * (warp & 3) + lane;  // row of the tile = TMEM lane
         const int I = m0 + t;
         const bool active = I < nBb;
         const long long rid = (long long)bh * nBmax + I;
-        const uint32_t tl = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-        float2* list = reinterpret_cast<float2*>(sm + SM::kList);  // [kFusedList][128] (value, J as int bits)
-        const uint32_t list_s = smem_u32(list) + 8u * t;
+        const uint32_t tl = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
+        unsigned char* region = sm + SM::kList;
+        uint32_t* hist = reinterpret_cast<uint32_t*>(region);  // [128 words][128 rows], pass A
+        float2* list = reinterpret_cast<float2*>(region);      // [kFusedList][128] (value, J bits), pass B
+        FusedRowInfo* info = reinterpret_cast<FusedRowInfo*>(region + SM::kListBytes);
+        int* rowcnt = reinterpret_cast<int*>(region + SM::kListBytes + 128 * sizeof(FusedRowInfo));
+        float* part_lo = reinterpret_cast<float*>(region);  // [4][128] sample ranges, before pass A
+        float* part_hi = part_lo + 4 * 128;
         unsigned char* rec = ws.finish + (size_t)rid * ws.fstride;
-        int a = 0;
+        auto rows_sync = [&]() { named_bar_sync(1, 32 * kFusedRowWarps); };
+        int a = 0, buf = 0;
         bool ok = true;
-        // The next accumulator use is read 32 columns (a "part") at a time: wait_acc waits
-        // for it, load_part(s, v) loads columns [32 s, 32 s + 32) and, after the last
-        // part, hands the buffer back to the MMA warp.  (Loops over parts keep the code
-        // small; a fully unrolled chunk does not fit the instruction cache.)
-        int buf = 0;
-        auto wait_acc = [&]() -> bool {
+        // this warp's 32 columns of the next accumulator use; then the buffer is released
+        auto fetch = [&](uint32_t (&v)[32]) -> bool {
             buf = a & 1;
             const bool got = warp_wait_bounded(acc_full + 8 * buf, (a >> 1) & 1, abort_flag, wait_limit);
             ++a;
-            if (got) tc_fence_after();
-            return got;
-        };
-        auto load_part = [&](int part, uint32_t (&v)[32]) {
+            if (!got) return false;
+            tc_fence_after();
             tmem_ld32(tl + 128u * buf + 32u * part, v);
             tmem_wait_ld();
-            if (part == 3) {
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(acc_empty + 8 * buf);
-            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty + 8 * buf);
+            return true;
         };
-        uint32_t* hist = reinterpret_cast<uint32_t*>(sm + SM::kList);  // histograms, then the lists
-        const uint32_t hist_s = smem_u32(hist) + 4u * t;
 
         // ---- sample: the row's value range [vlo, vlo + 256 / bscale]
-        float vlo = 0.f, bscale = 0.f;
-        ok = wait_acc();
-        if (ok) {
+        {
             float lo = INFINITY, hi = -INFINITY;
-#pragma unroll 1
-            for (int part = 0; part < 4; ++part) {
-                uint32_t v[32];
-                load_part(part, v);
+            uint32_t v[32];
+            ok = fetch(v);
+            if (ok) {
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const bool in = (long long)stride * (32 * part + i) < nBb;
                     lo = in ? fminf(lo, __uint_as_float(v[i])) : lo;
                     hi = in ? fmaxf(hi, __uint_as_float(v[i])) : hi;
                 }
+            }
+            part_lo[part * 128 + t] = lo;
+            part_hi[part * 128 + t] = hi;
+        }
+        rows_sync();
+        float vlo = 0.f, bscale = 0.f;
+        {
+            float lo = part_lo[t], hi = part_hi[t];
+#pragma unroll
+            for (int q = 1; q < 4; ++q) {
+                lo = fminf(lo, part_lo[q * 128 + t]);
+                hi = fmaxf(hi, part_hi[q * 128 + t]);
             }
             const float range = hi - lo;
             if (range > 0.f && range <= 3.0e38f) {
@@ -322,31 +346,35 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 }
             }
         }
-        for (int w = 0; w < 128; ++w) hist[w * 128 + t] = 0u;
+        rows_sync();  // the ranges are read: clear this thread's quarter of the row's histogram
+#pragma unroll 8
+        for (int w = 32 * part; w < 32 * part + 32; ++w) hist[w * 128 + t] = 0u;
+        rows_sync();
 
         // ---- pass A: 256-bucket histogram of the row's screened scores
         for (int ch = 0; ch < nC && ok; ++ch) {
-            if (!(ok = wait_acc())) break;
-            const int lim = active ? nBb - ch * 128 : 0;  // columns < lim are blocks of the sample
-#pragma unroll 1
-            for (int part = 0; part < 4; ++part) {
-                uint32_t v[32];
-                load_part(part, v);
+            uint32_t v[32];
+            if (!(ok = fetch(v))) break;
+            const int lim = active ? nBb - ch * 128 - 32 * part : 0;  // columns i < lim are blocks
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int b = fused_bucket(__uint_as_float(v[i]), vlo, bscale);
-                    red_add_shared_if(32 * part + i < lim, hist_s + (uint32_t)(b >> 1) * 512u, 1u << ((b & 1) << 4));
-                }
+            for (int i = 0; i < 32; ++i) {
+                const int b = fused_bucket(__uint_as_float(v[i]), vlo, bscale);
+                atomicAdd(&hist[(b >> 1) * 128 + t], i < lim ? 1u << ((b & 1) << 4) : 0u);
             }
         }
+        rows_sync();
 
-        // ---- the bucket [A, Bv) of the k-th largest value, its rank kk inside, and the
-        // window around it
-        double delta = INFINITY;
-        int kk = 0;
-        float A = -INFINITY, Bv = INFINITY, hiT = INFINITY, loT = -INFINITY;
-        bool fallback = false;
-        if (active && ok) {
+        // ---- (part 0) the bucket [A, Bv) of the k-th largest value, its rank kk inside,
+        // and the window around it
+        FusedRowInfo ri;
+        ri.A = -INFINITY;
+        ri.Bv = INFINITY;
+        ri.hiT = INFINITY;
+        ri.loT = -INFINITY;
+        ri.delta = INFINITY;
+        ri.kk = 0;
+        ri.flags = 0;
+        if (part == 0 && active && ok) {
             int cum = 0, bstar = -1;
             // buckets from the top, 16 words (32 buckets) loaded at a time
             for (int w0 = 112; w0 >= 0 && bstar < 0; w0 -= 16) {
@@ -369,102 +397,106 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                     }
                 }
             }
-            kk = k - cum;  // 1 <= kk <= the bucket's count
+            ri.kk = k - cum;  // 1 <= kk <= the bucket's count
             const double qn = ws.qnorm[(size_t)rid];
             const double kmx = ws.kmaxn[bh];
-            delta = 2.0 * (4.0 * 0x1p-16 + 3.0 * D * 0x1p-22) * qn * kmx + 3.0 * D * 0x1p-120 * (1.0 + qn + kmx);
+            ri.delta = 2.0 * (4.0 * 0x1p-16 + 3.0 * D * 0x1p-22) * qn * kmx + 3.0 * D * 0x1p-120 * (1.0 + qn + kmx);
             // a bound that is not meaningful in fp32 goes to the row routine
-            fallback = bstar < 0 || !(qn * kmx < 1.0e30) || !(delta < 1.0e30);
-            if (!fallback) {
+            if (bstar < 0 || !(qn * kmx < 1.0e30) || !(ri.delta < 1.0e30)) {
+                ri.flags = 2;
+            } else {
+                ri.flags = 1;
                 if (bscale > 0.f) {
-                    if (bstar > 0) A = fused_bucket_edge(bstar, vlo, bscale);
-                    if (bstar < 255) Bv = fused_bucket_edge(bstar + 1, vlo, bscale);
+                    if (bstar > 0) ri.A = fused_bucket_edge(bstar, vlo, bscale);
+                    if (bstar < 255) ri.Bv = fused_bucket_edge(bstar + 1, vlo, bscale);
                 }
-                if (Bv < INFINITY) hiT = __double2float_ru((double)Bv + 2.0 * delta);
-                if (A > -INFINITY) loT = __double2float_rd((double)A - 2.0 * delta);
+                if (ri.Bv < INFINITY) ri.hiT = __double2float_ru((double)ri.Bv + 2.0 * ri.delta);
+                if (ri.A > -INFINITY) ri.loT = __double2float_rd((double)ri.A - 2.0 * ri.delta);
             }
         }
-        named_bar_sync(1, 128);  // histograms read: the lists may overwrite them
+        rows_sync();  // histograms read: the lists and row info may overwrite them
+        if (part == 0) {
+            info[t] = ri;
+            rowcnt[t] = 0;
+        }
+        rows_sync();
+        ri = info[t];
+        const bool collect = (ri.flags & 1) != 0;
 
         // ---- pass B: sure keeps into the row's mask, the window into the list
-        int cnt = 0, n_sure = 0;
-        const bool collect = active && !fallback;
         for (int ch = 0; ch < nC && ok; ++ch) {
-            if (!(ok = wait_acc())) break;
-            const int j0 = ch * 128;
+            uint32_t v[32];
+            if (!(ok = fetch(v))) break;
+            const int j0 = ch * 128 + 32 * part;
             const int lim = collect ? nBb - j0 : 0;
-#pragma unroll 1
-            for (int part = 0; part < 4; ++part) {
-                uint32_t v[32];
-                load_part(part, v);
-                uint32_t word = 0u;
+            uint32_t word = 0u;
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float f = __uint_as_float(v[i]);
-                    const bool in = 32 * part + i < lim;
-                    word |= (in && f >= hiT) ? 1u << i : 0u;
-                    const bool win = in && f >= loT && f < hiT;
-                    if (__any_sync(0xffffffffu, win))  // rare: no shared-memory traffic otherwise
-                        st_shared_v2_if(win, list_s + (uint32_t)min(cnt, kFusedList - 1) * 1024u, v[i],
-                                        (uint32_t)(j0 + 32 * part + i));
-                    cnt += win ? 1 : 0;
-                }
-                if (collect) {
-                    n_sure += __popc(word);
-                    *reinterpret_cast<uint32_t*>(rec + 32 + 8 * kFusedList + 16 * ch + 4 * part) = word;
+            for (int i = 0; i < 32; ++i) {
+                const float f = __uint_as_float(v[i]);
+                const bool in = i < lim;
+                word |= (in && f >= ri.hiT) ? 1u << i : 0u;
+                const bool win = in && f >= ri.loT && f < ri.hiT;
+                if (__any_sync(0xffffffffu, win)) {  // rare: no shared-memory traffic otherwise
+                    if (win) {
+                        const int slot = atomicAdd(&rowcnt[t], 1);
+                        if (slot < kFusedList) list[slot * 128 + t] = make_float2(f, __int_as_float(j0 + i));
+                    }
                 }
             }
+            if (collect) *reinterpret_cast<uint32_t*>(rec + 32 + 8 * kFusedList + 16 * ch + 4 * part) = word;
         }
-        if (collect && cnt > kFusedList) fallback = true;
-        any_fallback = __syncthreads_or(active && fallback && ok);
+        rows_sync();
+        const int cnt = rowcnt[t];
+        const bool fallback = (ri.flags & 2) != 0 || (collect && cnt > kFusedList);
+        any_fallback = __syncthreads_or(part == 0 && active && fallback && ok);
 
         // ---- pass C (only when some row of the tile fell back): its screened scores
         if (any_fallback && ok) {
             for (int ch = 0; ch < nC && ok; ++ch) {
-                if (!(ok = wait_acc())) break;
-#pragma unroll 1
-                for (int part = 0; part < 4; ++part) {
-                    uint32_t v[32];
-                    load_part(part, v);
-                    if (active && fallback) {
-                        float* dst = ws.scores + (size_t)rid * ws.ld + ch * 128 + 32 * part;
+                uint32_t v[32];
+                if (!(ok = fetch(v))) break;
+                if (active && fallback) {
+                    const int c0 = ch * 128 + 32 * part;
+                    float* dst = ws.scores + (size_t)rid * ws.ld + c0;
 #pragma unroll
-                        for (int i = 0; i < 32; i += 4)
-                            if (ch * 128 + 32 * part + i + 4 <= ws.ld)
-                                *reinterpret_cast<float4*>(dst + i) =
-                                    make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]),
-                                                __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
-                    }
+                    for (int i = 0; i < 32; i += 4)
+                        if (c0 + i + 4 <= ws.ld)
+                            *reinterpret_cast<float4*>(dst + i) =
+                                make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]),
+                                            __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
                 }
             }
-            if (ok && active && fallback) ws.ovf_rows[atomicAdd(ws.ovf_count, 1)] = (int32_t)rid;
+            if (part == 0 && ok && active && fallback) ws.ovf_rows[atomicAdd(ws.ovf_count, 1)] = (int32_t)rid;
         }
         if (!__all_sync(0xffffffffu, ok)) ok = false;
 
         // ---- the record: header, then (warp by warp, coalesced) the window entries
-        if (ok && active) {
+        if (part == 0 && ok && active) {
             FusedRowHead h;
-            h.A = A;
-            h.Bv = Bv;
-            h.delta = delta;
+            h.A = ri.A;
+            h.Bv = ri.Bv;
+            h.delta = ri.delta;
             h.cnt = fallback ? -1 : cnt;
-            h.n_sure = n_sure;
-            h.kk = kk;
-            h.pad = 0;
+            h.kk = ri.kk;
+            h.pad[0] = 0;
+            h.pad[1] = 0;
             *reinterpret_cast<FusedRowHead*>(rec) = h;
         }
-        const int n_copy = (ok && active && !fallback) ? cnt : 0;
-        for (int r = 0; r < 32; ++r) {
-            const int row = warp * 32 + r;
-            const int n = __shfl_sync(0xffffffffu, n_copy, r);
-            float2* dst = reinterpret_cast<float2*>(ws.finish + ((size_t)bh * nBmax + m0 + row) * ws.fstride + 32);
-            for (int e = lane; e < n; e += 32) dst[e] = list[e * 128 + row];
+        if (part == 0) {
+            const int n_copy = (ok && active && !fallback) ? cnt : 0;
+            for (int r = 0; r < 32; ++r) {
+                const int row = 32 * (warp & 3) + r;
+                const int n = __shfl_sync(0xffffffffu, n_copy, r);
+                float2* dst =
+                    reinterpret_cast<float2*>(ws.finish + ((size_t)bh * nBmax + m0 + row) * ws.fstride + 32);
+                for (int e = lane; e < n; e += 32) dst[e] = list[e * 128 + row];
+            }
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, 256);
     }
@@ -568,7 +600,19 @@ __global__ void __launch_bounds__(32 * kFinishWarps) select_finish_kernel(Select
     }
     const uint32_t kb0 = __ballot_sync(0xffffffffu, keep[0]), kb1 = __ballot_sync(0xffffffffu, keep[1]);
     const uint32_t bb0 = __ballot_sync(0xffffffffu, band[0]), bb1 = __ballot_sync(0xffffffffu, band[1]);
-    const int n_in = h.n_sure + __popc(kb0) + __popc(kb1);
+    // the row's mask (the blocks kept outright) into shared memory, and its count
+    uint32_t* words = reinterpret_cast<uint32_t*>(wsm + FS::kW);
+    const int W = (nBb + 31) / 32;
+    const uint32_t* mw = reinterpret_cast<const uint32_t*>(rec + 32 + 8 * kFusedList);
+    int n_sure = 0;
+    for (int w = lane; w < W; w += 32) {
+        const uint32_t x = mw[w];
+        words[w] = x;
+        n_sure += __popc(x);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) n_sure += __shfl_xor_sync(0xffffffffu, n_sure, off);
+    const int n_in = n_sure + __popc(kb0) + __popc(kb1);
     const int n_band = __popc(bb0) + __popc(bb1);
     const int need = k - n_in;  // 1 <= need <= n_band
 
@@ -702,11 +746,6 @@ __global__ void __launch_bounds__(32 * kFinishWarps) select_finish_kernel(Select
     __syncwarp();
 
     // ---- the mask plus the extra blocks, written in ascending order
-    uint32_t* words = reinterpret_cast<uint32_t*>(wsm + FS::kW);
-    const int W = (nBb + 31) / 32;
-    const uint32_t* mw = reinterpret_cast<const uint32_t*>(rec + 32 + 8 * kFusedList);
-    for (int w = lane; w < W; w += 32) words[w] = mw[w];
-    __syncwarp();
     for (int e = lane; e < n_extra; e += 32) atomicOr(&words[xj[e] >> 5], 1u << (xj[e] & 31));
     __syncwarp();
     int32_t* out = kv_idx + (size_t)rid * kmax;
