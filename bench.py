@@ -476,9 +476,10 @@ def run_ours(args):
         q_m = torch.empty((B, H, Npad // 64, D), dtype=torch.float64, device=dev)
         k_m = torch.empty_like(q_m)
 
-    def route(qq=q, kk=k, vll=vl):
+    def route(qq=q, kk=k, vll=vl, mid=None):
         """Routing (and, with --producer, the norm + RoPE before it); returns the Q, K
-        the attention reads."""
+        the attention reads.  `mid`, an event, is recorded between the routing call
+        and the query-block pairing."""
         if args.producer:
             sba.qk_norm_rope_pool(qq, wq, pos, vll, rope_dim=3 * D // 4, out=q_n, means=q_m, stream=stream)
             sba.qk_norm_rope_pool(kk, wk, pos, vll, rope_dim=3 * D // 4, out=k_n, means=k_m, stream=stream)
@@ -491,6 +492,8 @@ def run_ours(args):
         else:
             sba.pool_select(qq, kk, vll, w.sparsity, kmax, kv_idx=kv_idx, kv_cnt=kv_cnt, workspace=ws,
                             stream=stream)
+        if mid is not None:
+            mid.record(stream)
         if not pair_kernel:  # the CTA-pair kernel tiles four adjacent query blocks itself
             sba.pair_query_blocks(kv_idx, kv_cnt, vll, pair_order=pair_order, workspace=pws, stream=stream)
         return qq, kk
@@ -529,7 +532,7 @@ def run_ours(args):
 
     # ---- timed region: K steps, events on the launching stream
     K = args.steps
-    ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(4)) for _ in range(K)]
+    ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(5)) for _ in range(K)]
     barrier()
     torch.cuda.synchronize(dev)
     t_begin = time.monotonic()
@@ -537,7 +540,7 @@ def run_ours(args):
         ev[i][0].record(stream)
         qq, kk, vv, vll = prep()
         ev[i][3].record(stream)
-        qa, ka = route(qq, kk, vll)
+        qa, ka = route(qq, kk, vll, mid=ev[i][4])
         ev[i][1].record(stream)
         attend(qa, ka, vv, vll)
         ev[i][2].record(stream)
@@ -552,10 +555,12 @@ def run_ours(args):
     med_sel = statistics.median(e[0].elapsed_time(e[1]) for e in ev)
     med_attn = statistics.median(e[1].elapsed_time(e[2]) for e in ev)
     prune_ms = statistics.mean(e[0].elapsed_time(e[3]) for e in ev)
+    med_call = statistics.median(e[3].elapsed_time(e[4]) for e in ev)  # the routing call alone
+    med_pair = statistics.median(e[4].elapsed_time(e[1]) for e in ev)
     if sba.device_status(stream) != 0:
         raise RuntimeError("device status error in the timed region")
-    total_ms, attn_ms, sel_ms, med_step, med_sel, med_attn, prune_ms = max_over_ranks(
-        [total_ms, attn_ms, sel_ms, med_step, med_sel, med_attn, prune_ms], dist, dev)
+    total_ms, attn_ms, sel_ms, med_step, med_sel, med_attn, prune_ms, med_call, med_pair = max_over_ranks(
+        [total_ms, attn_ms, sel_ms, med_step, med_sel, med_attn, prune_ms, med_call, med_pair], dist, dev)
     ms_step = total_ms / K
     value = whole_job_value(f_step, ms_step, world)
 
@@ -660,17 +665,25 @@ def run_ours(args):
                                     f"{attn_ms:.1f} ms, well short of the seconds-long loop of the sustained figure",
                      "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
                      "traffic": traffic},
-        # per step: routing = 2 pooling + key-norm maximum + screen (only when blocks are
-        # dropped) + top-k; pairing = bitmaps + 4 x (propose, resolve) + emit (not with the
-        # CTA-pair kernel); 1 attention
+        # per step: routing = 2 pooling + key-norm maximum + fused screen + finish + rest
+        # rows (the log-sum-exp router: 2 pooling + key-norm maximum + screen, only when
+        # blocks are dropped, + top-k); pairing = bitmaps + 4 x (propose, resolve) + emit
+        # (not with the CTA-pair kernel); 1 attention
         # (--producer: 2 producer launches and 2 splits of the given means replace pooling)
         # (--compensate mean: 2 block-mean launches before the attention)
         # (--prune: norm + select + 3 gathers, and the positions' gather with --producer)
-        "gpu_launches": (4 + (1 if w.sparsity > 0 else 0) + (2 if args.producer else 0)
+        "gpu_launches": ((4 + (1 if w.sparsity > 0 else 0) if lse_router else 6) + (2 if args.producer else 0)
                          + (0 if pair_kernel else 10) + 1 + (2 if args.compensate == "mean" else 0)
                          + (5 + (1 if args.producer else 0) if args.prune is not None else 0)) * K,
         "clocks": clk,
     }
+    if not lse_router and not args.producer:
+        # the routing call alone: it reads Q and K once (the block means it writes are
+        # small beside them)
+        qk_bytes = 2 * q.numel() * 2
+        line["routing"] = {"pool_select_ms": med_call, "pair_ms": med_pair, "qk_bytes": qk_bytes,
+                           "hbm_gbs": qk_bytes / (med_call * 1e-3) / 1e9,
+                           "frac_of_hbm": qk_bytes / (med_call * 1e-3) / 1e9 / float(peaks["hbm_gbs"])}
     if e2e is not None:
         line["e2e"] = e2e
     if args.prune is not None:

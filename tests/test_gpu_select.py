@@ -73,6 +73,26 @@ def test_block_means_bit_exact(sba, oracle_mod):
         np.testing.assert_array_equal(m, ref)
 
 
+def test_block_means_extreme_values(sba, oracle_mod):
+    """Block means of random bf16 bit patterns -- every exponent, subnormals, the largest
+    finite values, sums that cancel into the subnormal range -- equal the oracle's fp64
+    token-order sums bit for bit; blocks holding inf or NaN too (they take the
+    conversion-unit path)."""
+    rng = np.random.default_rng(7)
+    B, H, Np, D = 1, 2, 640, 64
+    bits = rng.integers(0, 1 << 16, size=(B, H, Np, D), dtype=np.uint16)
+    nonfinite = ((bits >> 7) & 0xFF) == 0xFF
+    bits[nonfinite] &= 0x807F              # exponent 0: those become subnormals or zeros
+    bits[0, 0, 64 * 3 + 5, 7] = 0x7F80     # +inf in block 3
+    bits[0, 1, 64 * 7 + 60, 2] = 0x7FC1    # NaN in block 7
+    bits[0, 1, 64 * 8:64 * 9, :] = bits[0, 1, 64 * 8, :]                       # block 8: one row repeated
+    bits[0, 1, 64 * 8 + 32:64 * 9, :] = bits[0, 1, 64 * 8, :] ^ 0x8000         # ... then negated: cancels
+    x = torch.from_numpy(bits.view(np.int16)).to(DEV).view(torch.bfloat16)
+    m = sba.block_means(x, None).cpu().numpy()
+    ref = oracle_mod.pool(bits, np.array([Np], dtype=np.int32))
+    np.testing.assert_array_equal(m, ref)
+
+
 def test_zero_queries_all_ties(sba, oracle_mod):
     """Every score is 0: the whole row is one tie band; the lowest indices win."""
     w = make_custom(1, 2, 128, (2, 16, 40), 0.7, seed=5)
