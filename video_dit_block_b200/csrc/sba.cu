@@ -14,7 +14,6 @@
 #include "attention2.cuh"
 #include "common.cuh"
 #include "select.cuh"
-#include "score_mma.cuh"
 #include "select_fused.cuh"
 #include "score_lse.cuh"
 #include "pair.cuh"

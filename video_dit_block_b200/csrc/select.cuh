@@ -11,12 +11,12 @@
 //
 // Exactness.  A block sum of 64 bf16 values is formed channel by channel in
 // token order in fp64; the mean is one correctly rounded division.  Scores are
-// first screened on the tensor cores (score_mma_kernel: bf16 hi/lo splits of the
+// first screened on the tensor cores (select_fused_kernel: bf16 hi/lo splits of the
 // means, fp32 accumulation in TMEM) with a proven bound delta on their error; only
-// candidates within 2*delta of the screened k-th value are re-scored in fp64, with
-// a fixed summation order and explicit round-to-nearest operations, and the
-// selection among them is made on those fp64 values.  Everything above the
-// band is kept, everything below is dropped.
+// candidates within 2*delta of the screened k-th value are re-scored in fp64, and
+// the selection among them is made on fp64 values computed with a fixed summation
+// order and explicit round-to-nearest operations.  Everything above the band is
+// kept, everything below is dropped.
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
@@ -521,16 +521,16 @@ __host__ __device__ inline size_t topk_smem(int warps, int ld) { return (size_t)
 
 // Top-k routing of one (b, h, I) row per warp, from the screened scores.
 //
-// Screen error.  The scores come from score_mma_kernel: S = qhi.khi + qhi.klo +
+// Screen error.  The scores come from select_fused_kernel: S = qhi.khi + qhi.klo +
 // qlo.khi in fp32, with hi = bf16(x), lo = bf16(x - hi) (each through fp32).  Per
 // term d the dropped parts (qlo.klo and the remainders of the split) are below
 // 4 * 2^-16 |qbar_d kbar_d|; the products are exact in fp32 and the accumulation
 // of the 3D products in fp32 adds at most 3D * 2^-22 of sum |qbar_d kbar_d| (two
 // units in the last place per addition, whatever the order).  With Cauchy-Schwarz,
 // |S - qbar.kbar| <= (4 * 2^-16 + 3D * 2^-22) |qbar_I| max_J |kbar_J|, doubled here
-// for margin, plus an absolute term for values in the subnormal range.  (The
-// screen now sums hi.hi apart from the two cross terms, which only lowers the
-// accumulation error; this bound is kept as it stands.)
+// for margin, plus an absolute term for values in the subnormal range.  (The fused
+// screen accumulates all 3D products in one fp32 TMEM accumulator, which is the case
+// this bound covers.)
 //
 // Log-sum-exp router (NSUB = 4).  The screen (score_lse_kernel) forms every
 // sub-block logit in log2 units, y' = fp32(acc * fp32(log2(e) / sqrt(D))), where acc
