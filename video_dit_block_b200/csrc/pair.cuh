@@ -115,37 +115,36 @@ __global__ void __launch_bounds__(256) pair_propose_kernel(PairWorkspace ws,
     }
     const uint32_t* ba = sbits + (size_t)(a - lo) * W;
     // lane l scores a - 64 + l, a - 32 + l, a + 1 + l, a + 33 + l.  Preference as one
-    // ordered key: larger overlap, then smaller distance, then lower index.
+    // ordered 32-bit key: larger overlap, then smaller distance, then the lower index
+    // (of the two candidates at one distance, the one before a); 0 = no candidate.
     constexpr int kSlots = 2 * kPairWindow / 32;
-    long long key[kSlots];
+    uint32_t key[kSlots];
 #pragma unroll
     for (int slot = 0; slot < kSlots; ++slot) {
         const int half = kPairWindow / 32;
         const int c = slot < half ? a - kPairWindow + 32 * slot + lane : a + 1 + 32 * (slot - half) + lane;
-        key[slot] = -1;
+        key[slot] = 0u;
         if (c < 0 || c >= nB) continue;
         const uint32_t* bc = sbits + (size_t)(c - lo) * W;
         int ov = 0;
         for (int w = 0; w < W; ++w) ov += __popc(ba[w] & bc[w]);
-        const int dist = c > a ? c - a : a - c;
-        key[slot] = ((long long)ov << 40) | ((long long)(0xFFFFF - dist) << 20) | (long long)(0xFFFFF - c);
+        const int dist = c > a ? c - a : a - c;  // 1 .. kPairWindow
+        key[slot] = ((uint32_t)(ov + 1) << 8) | ((uint32_t)(kPairWindow - dist) << 1) | (c < a ? 1u : 0u);
     }
     // the kPairCands best candidates, best first
     for (int r = 0; r < kPairCands; ++r) {
-        long long mine = key[0];
+        uint32_t mine = key[0];
 #pragma unroll
-        for (int slot = 1; slot < kSlots; ++slot) mine = key[slot] > mine ? key[slot] : mine;
-        long long best = mine;
+        for (int slot = 1; slot < kSlots; ++slot) mine = max(mine, key[slot]);
+        const uint32_t best = __reduce_max_sync(0xffffffffu, mine);
+        if (best != 0u && mine == best) {
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            const long long o = __shfl_xor_sync(0xffffffffu, best, off);
-            best = o > best ? o : best;
+            for (int slot = 0; slot < kSlots; ++slot) key[slot] = key[slot] == best ? 0u : key[slot];
         }
-        if (best >= 0 && mine == best) {
-#pragma unroll
-            for (int slot = 0; slot < kSlots; ++slot) key[slot] = key[slot] == best ? -1 : key[slot];
+        if (lane == 0) {
+            const int dist = kPairWindow - (int)((best >> 1) & 0x7Fu);
+            cand[r] = best == 0u ? -1 : ((best & 1u) ? a - dist : a + dist);
         }
-        if (lane == 0) cand[r] = best < 0 ? -1 : (int)(0xFFFFF - (best & 0xFFFFF));
     }
     if (lane == 0) ws.proposal[row] = cand[0];
 }

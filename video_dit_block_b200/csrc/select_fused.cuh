@@ -99,8 +99,27 @@ __device__ __forceinline__ int fused_bucket(float f, float vlo, float bscale) {
 
 // Smallest float x (over all non-NaN floats, in order) with fused_bucket(x) >= b, for
 // 1 <= b <= 255 and a finite bscale > 0 (then bucket(-inf) = 0 and bucket(+inf) = 255).
+// Starts from vlo + b / bscale, within a few units in the last place of the edge for
+// ranges that fp32 resolves, and steps float by float; a bisection over the whole
+// float order decides when that has not settled within 64 steps.
 __device__ float fused_bucket_edge(int b, float vlo, float bscale) {
-    uint32_t lo = f32_key(-INFINITY), hi = f32_key(INFINITY);
+    uint32_t g = f32_key(__fadd_rn(vlo, __fdiv_rn((float)b, bscale)));
+    const uint32_t kmin = f32_key(-INFINITY), kmax = f32_key(INFINITY);
+    if (g > kmin && g <= kmax) {
+        if (fused_bucket(key_to_f32(g), vlo, bscale) >= b) {
+            for (int step = 0; step < 64; ++step) {  // down while the float below is still in
+                if (g == kmin || fused_bucket(key_to_f32(g - 1u), vlo, bscale) < b) return key_to_f32(g);
+                --g;
+            }
+        } else {
+            for (int step = 0; step < 64; ++step) {  // up until in
+                ++g;
+                if (g > kmax) break;
+                if (fused_bucket(key_to_f32(g), vlo, bscale) >= b) return key_to_f32(g);
+            }
+        }
+    }
+    uint32_t lo = kmin, hi = kmax;
     while (hi - lo > 1u) {
         const uint32_t mid = lo + (hi - lo) / 2u;
         if (fused_bucket(key_to_f32(mid), vlo, bscale) >= b)
@@ -351,6 +370,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         for (int w = 32 * part; w < 32 * part + 32; ++w) hist[w * 128 + t] = 0u;
         rows_sync();
 
+        // the bound's inputs, fetched before pass A so that their latency is hidden
+        const double qn_row = part == 0 && active ? ws.qnorm[(size_t)rid] : 0.0;
+        const double kmx_bh = part == 0 && active ? ws.kmaxn[bh] : 0.0;
+
         // ---- pass A: 256-bucket histogram of the row's screened scores
         for (int ch = 0; ch < nC && ok; ++ch) {
             uint32_t v[32];
@@ -398,8 +421,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 }
             }
             ri.kk = k - cum;  // 1 <= kk <= the bucket's count
-            const double qn = ws.qnorm[(size_t)rid];
-            const double kmx = ws.kmaxn[bh];
+            const double qn = qn_row, kmx = kmx_bh;
             ri.delta = 2.0 * (4.0 * 0x1p-16 + 3.0 * D * 0x1p-22) * qn * kmx + 3.0 * D * 0x1p-120 * (1.0 + qn + kmx);
             // a bound that is not meaningful in fp32 goes to the row routine
             if (bstar < 0 || !(qn * kmx < 1.0e30) || !(ri.delta < 1.0e30)) {
@@ -530,13 +552,13 @@ __global__ void __launch_bounds__(32 * kFinishWarps) select_finish_kernel(Select
     using FS = FinishSmem<D>;
     extern __shared__ __align__(16) unsigned char fsm_raw[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const long long rid = (long long)blockIdx.x * kFinishWarps + warp;
+    const int rid = blockIdx.x * kFinishWarps + warp;  // rows < 2^28
     if (rid >= rows) return;
     unsigned char* wsm = fsm_raw + warp * FS::kWarp;
     const int nBmax = Npad / kBlock;
-    const long long bh = rid / nBmax;
-    const int I = (int)(rid % nBmax);
-    const int L = sample_len(valid_len, (int)(bh / H), Npad);
+    const int bh = rid / nBmax;
+    const int I = rid - bh * nBmax;
+    const int L = sample_len(valid_len, bh / H, Npad);
     const int nBb = (L + kBlock - 1) / kBlock;
     const int k = keep_count_budget(nBb, sparsity, budget);
     if (I >= nBb) {
@@ -550,7 +572,17 @@ __global__ void __launch_bounds__(32 * kFinishWarps) select_finish_kernel(Select
     const int cnt = min(h.cnt, kFusedList);
     const float2* ent = reinterpret_cast<const float2*>(rec + 32);
 
-    // ---- the window: lane holds entries lane and lane + 32
+    // ---- the window (lane holds entries lane and lane + 32), the row's mask (the
+    // blocks kept outright) and its query mean: all loads issued together
+    const int W = (nBb + 31) / 32;
+    const uint32_t* mw = reinterpret_cast<const uint32_t*>(rec + 32 + 8 * kFusedList);
+    uint32_t mwords[4];  // words lane + 32 i (W <= 128)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) mwords[i] = lane + 32 * i < W ? mw[lane + 32 * i] : 0u;
+    const double* qrow = ws.qmean64 + (size_t)rid * D;
+    double qd[D / 32];
+#pragma unroll
+    for (int i = 0; i < D / 32; ++i) qd[i] = qrow[lane + 32 * i];
     float f[2];
     int jb[2];
     bool has[2], mem[2];
@@ -600,15 +632,13 @@ __global__ void __launch_bounds__(32 * kFinishWarps) select_finish_kernel(Select
     }
     const uint32_t kb0 = __ballot_sync(0xffffffffu, keep[0]), kb1 = __ballot_sync(0xffffffffu, keep[1]);
     const uint32_t bb0 = __ballot_sync(0xffffffffu, band[0]), bb1 = __ballot_sync(0xffffffffu, band[1]);
-    // the row's mask (the blocks kept outright) into shared memory, and its count
+    // the row's mask into shared memory, and its count
     uint32_t* words = reinterpret_cast<uint32_t*>(wsm + FS::kW);
-    const int W = (nBb + 31) / 32;
-    const uint32_t* mw = reinterpret_cast<const uint32_t*>(rec + 32 + 8 * kFusedList);
     int n_sure = 0;
-    for (int w = lane; w < W; w += 32) {
-        const uint32_t x = mw[w];
-        words[w] = x;
-        n_sure += __popc(x);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        if (lane + 32 * i < W) words[lane + 32 * i] = mwords[i];
+        n_sure += __popc(mwords[i]);
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) n_sure += __shfl_xor_sync(0xffffffffu, n_sure, off);
@@ -648,30 +678,26 @@ __global__ void __launch_bounds__(32 * kFinishWarps) select_finish_kernel(Select
             if (band[q]) bj[base + __popc(bb & lanemask_lt())] = jb[q];
         }
         __syncwarp();
-        const double* qrow = ws.qmean64 + (size_t)rid * D;
         const double* kbase = ws.kmean64 + (size_t)bh * nBmax * D;
         const double inv = __ddiv_rn(1.0, __dsqrt_rn((double)D));
-        double qd[D / 32];
+        for (int m = 0; m < n_band; m += 4) {  // four members per step: their loads in flight together
+            double p[4];
+            double kv[4][D / 32];
 #pragma unroll
-        for (int i = 0; i < D / 32; ++i) qd[i] = qrow[lane + 32 * i];
-        for (int m = 0; m < n_band; m += 2) {  // two members per step: more loads in flight
-            const double* k0 = kbase + (size_t)bj[m] * D;
-            const double* k1 = kbase + (size_t)bj[m + 1 < n_band ? m + 1 : m] * D;
-            double p0 = 0.0, p1 = 0.0;
+            for (int u = 0; u < 4; ++u) {
+                const double* kr = kbase + (size_t)bj[m + u < n_band ? m + u : m] * D;
 #pragma unroll
-            for (int i = 0; i < D / 32; ++i) {
-                p0 = fma(qd[i], k0[lane + 32 * i], p0);
-                p1 = fma(qd[i], k1[lane + 32 * i], p1);
+                for (int i = 0; i < D / 32; ++i) kv[u][i] = kr[lane + 32 * i];
             }
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                p0 += __shfl_xor_sync(0xffffffffu, p0, off);
-                p1 += __shfl_xor_sync(0xffffffffu, p1, off);
+            for (int u = 0; u < 4; ++u) {
+                p[u] = 0.0;
+#pragma unroll
+                for (int i = 0; i < D / 32; ++i) p[u] = fma(qd[i], kv[u][i], p[u]);
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) p[u] += __shfl_xor_sync(0xffffffffu, p[u], off);
             }
-            if (lane == 0) {
-                rx[m] = p0 * inv;
-                if (m + 1 < n_band) rx[m + 1] = p1 * inv;
-            }
+            if (lane < 4 && m + lane < n_band) rx[m + lane] = (lane == 0 ? p[0] : lane == 1 ? p[1] : lane == 2 ? p[2] : p[3]) * inv;
         }
         __syncwarp();
         const double qn = ws.qnorm[(size_t)rid], kmx = ws.kmaxn[bh];
