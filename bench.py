@@ -665,14 +665,14 @@ def run_ours(args):
                                     f"{attn_ms:.1f} ms, well short of the seconds-long loop of the sustained figure",
                      "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
                      "traffic": traffic},
-        # per step: routing = 2 pooling + key-norm maximum + fused screen + finish + rest
-        # rows (the log-sum-exp router: 2 pooling + key-norm maximum + screen, only when
-        # blocks are dropped, + top-k); pairing = bitmaps + 4 x (propose, resolve) + emit
-        # (not with the CTA-pair kernel); 1 attention
+        # per step: routing = pooling (Q and K in one launch) + key-norm maximum + fused
+        # screen + finish + rest rows (the log-sum-exp router: the same pooling launch +
+        # key-norm maximum + screen, only when blocks are dropped, + top-k); pairing =
+        # bitmaps + 4 x (propose, resolve) + emit (not with the CTA-pair kernel); 1 attention
         # (--producer: 2 producer launches and 2 splits of the given means replace pooling)
         # (--compensate mean: 2 block-mean launches before the attention)
         # (--prune: norm + select + 3 gathers, and the positions' gather with --producer)
-        "gpu_launches": ((4 + (1 if w.sparsity > 0 else 0) if lse_router else 6) + (2 if args.producer else 0)
+        "gpu_launches": ((3 + (1 if w.sparsity > 0 else 0) if lse_router else 5) + (3 if args.producer else 0)
                          + (0 if pair_kernel else 10) + 1 + (2 if args.compensate == "mean" else 0)
                          + (5 + (1 if args.producer else 0) if args.prune is not None else 0)) * K,
         "clocks": clk,

@@ -249,10 +249,10 @@ sba_status run_select(const void* q, const void* k, int B, int H, int Npad, cons
         sba::split_means_kernel<D><<<pool_grid, 256, 0, s>>>(qmean, ws.qhi, ws.qlo, ws.qnorm, pgroups);
         sba::split_means_kernel<D><<<pool_grid, 256, 0, s>>>(kmean, ws.khi, ws.klo, ws.knorm, pgroups);
     } else {
-        sba::pool_kernel<D, BLK><<<pool_grid, 256, 0, s>>>(qb, valid_len, H, Npad, ws.qmean64, ws.qhi, ws.qlo,
-                                                           ws.qnorm, pgroups);
-        sba::pool_kernel<D, BLK><<<pool_grid, 256, 0, s>>>(kb, valid_len, H, Npad, ws.kmean64, ws.khi, ws.klo,
-                                                           ws.knorm, pgroups);
+        // Q and K in one launch: the CTAs past pool_grid pool K
+        const sba::PoolSecond kside{kb, ws.kmean64, ws.khi, ws.klo, ws.knorm, pool_grid};
+        sba::pool_kernel<D, BLK><<<2 * pool_grid, 256, 0, s>>>(qb, valid_len, H, Npad, ws.qmean64, ws.qhi, ws.qlo,
+                                                               ws.qnorm, pgroups, kside);
     }
     sba::kmax_kernel<<<(unsigned)((BH + 7) / 8), 256, 0, s>>>(ws, valid_len, H, Npad, (int)BH, BLK);
     if (NSUB == 1) {
@@ -433,10 +433,12 @@ sba_status sba_block_means(const void* x, int B, int H, int Npad, int D, const i
     const unsigned grid = (unsigned)((groups + gpc - 1) / gpc);
     if (D == 128)
         sba::pool_kernel<128><<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), valid_len, H,
-                                                   Npad, out, nullptr, nullptr, nullptr, groups);
+                                                   Npad, out, nullptr, nullptr, nullptr, groups,
+                                                   sba::PoolSecond{nullptr, nullptr, nullptr, nullptr, nullptr, grid});
     else
         sba::pool_kernel<64><<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), valid_len, H,
-                                                  Npad, out, nullptr, nullptr, nullptr, groups);
+                                                  Npad, out, nullptr, nullptr, nullptr, groups,
+                                                   sba::PoolSecond{nullptr, nullptr, nullptr, nullptr, nullptr, grid});
     return cudaGetLastError() == cudaSuccess ? SBA_OK : SBA_ERR_CUDA;
 }
 

@@ -147,17 +147,38 @@ __device__ __forceinline__ int sample_len(const int32_t* valid_len, int b, int N
 // the kBlock / BLK sub-blocks of a block are interleaved channel by channel,
 // [..][block][D][kBlock / BLK], so that the lanes re-scoring the sub-block pairs of
 // a block read adjacent words; hi/lo and the norms stay one row per pooled row.
+// The second tensor, pooled by CTAs blockIdx.x >= blocks0 of the same launch (the
+// router's Q and K in one grid); blocks0 = gridDim.x: one tensor.
+struct PoolSecond {
+    const __nv_bfloat16* x;
+    double* mean64;
+    __nv_bfloat16* hi16;
+    __nv_bfloat16* lo16;
+    double* norm;
+    unsigned blocks0;
+};
+
 template <int D, int BLK = kBlock>
 __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restrict__ x,
                                                    const int32_t* __restrict__ valid_len, int H,
                                                    int Npad, double* __restrict__ mean64,
                                                    __nv_bfloat16* __restrict__ hi16,
                                                    __nv_bfloat16* __restrict__ lo16,
-                                                   double* __restrict__ norm, long long n_groups) {
+                                                   double* __restrict__ norm, long long n_groups,
+                                                   PoolSecond second) {
     constexpr int LPB = D / 8;  // lanes per block group
     constexpr int UNROLL = 16;
     const int nB = Npad / BLK;
-    long long grp = (long long)blockIdx.x * (256 / LPB) + threadIdx.x / LPB;
+    unsigned bid = blockIdx.x;
+    if (bid >= second.blocks0) {
+        bid -= second.blocks0;
+        x = second.x;
+        mean64 = second.mean64;
+        hi16 = second.hi16;
+        lo16 = second.lo16;
+        norm = second.norm;
+    }
+    long long grp = (long long)bid * (256 / LPB) + threadIdx.x / LPB;
     const int g = threadIdx.x % LPB;
     const bool active = grp < n_groups;
     if (!active) grp = n_groups - 1;  // keep the shuffles below warp-uniform

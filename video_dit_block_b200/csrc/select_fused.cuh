@@ -600,19 +600,23 @@ __global__ void __launch_bounds__(32 * kFinishWarps) select_finish_kernel(Select
         if (lane == 0) raise_device_error(kErrBadRouting);
         return;
     }
-    // tau: the kk-th largest member of the bucket
+    // tau: the kk-th largest member of the bucket (the members' values gathered first)
+    float* mf = reinterpret_cast<float*>(wsm + FS::kX);  // free until the band needs it
+    const uint32_t mb0 = __ballot_sync(0xffffffffu, mem[0]), mb1 = __ballot_sync(0xffffffffu, mem[1]);
+    if (mem[0]) mf[__popc(mb0 & lanemask_lt())] = f[0];
+    if (mem[1]) mf[__popc(mb0) + __popc(mb1 & lanemask_lt())] = f[1];
+    const int n_mem = __popc(mb0) + __popc(mb1);
+    __syncwarp();
     int gt[2] = {0, 0}, ge[2] = {0, 0};
-    for (int u = 0; u < cnt; ++u) {
-        const float fu = __shfl_sync(0xffffffffu, u < 32 ? f[0] : f[1], u & 31);
-        const bool mu = __shfl_sync(0xffffffffu, u < 32 ? mem[0] : mem[1], u & 31);
-        if (mu) {
+    for (int u = 0; u < n_mem; ++u) {
+        const float fu = mf[u];
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                gt[q] += fu > f[q] ? 1 : 0;
-                ge[q] += fu >= f[q] ? 1 : 0;
-            }
+        for (int q = 0; q < 2; ++q) {
+            gt[q] += fu > f[q] ? 1 : 0;
+            ge[q] += fu >= f[q] ? 1 : 0;
         }
     }
+    __syncwarp();
     const bool hit0 = mem[0] && gt[0] < h.kk && h.kk <= ge[0];
     const bool hit1 = mem[1] && gt[1] < h.kk && h.kk <= ge[1];
     const uint32_t hb0 = __ballot_sync(0xffffffffu, hit0), hb1 = __ballot_sync(0xffffffffu, hit1);
