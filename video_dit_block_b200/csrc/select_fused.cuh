@@ -12,7 +12,7 @@
 // key blocks at a time (a "chunk": M128 N128, S = qhi.khi + qlo.khi + qhi.klo in one
 // fp32 TMEM buffer of 128 columns, two buffers), in this order:
 //   sample   one hi.hi product against 128 key blocks spread evenly over the head
-//            gives the row a value range [vlo, vhi];
+//            gives the row a value range [lo, hi];
 //   pass A   every chunk: a 256-bucket histogram of the screened scores over that
 //            range (the edge buckets open), which locates the bucket [A, Bv) holding
 //            the k-th largest screened value, and its rank kk inside;
@@ -90,39 +90,43 @@ struct FusedRowInfo {
     int32_t flags;  // 1: collect the window; 2: hand the row to topk_rest_kernel
 };
 
-// Bucket of a screened value: floor((f - vlo) * bscale) clamped to [0, 255], each
-// operation rounded to nearest, so the map is non-decreasing in f.
-__device__ __forceinline__ int fused_bucket(float f, float vlo, float bscale) {
-    const int b = __float2int_rd(__fmul_rn(__fsub_rn(f, vlo), bscale));
-    return min(255, max(0, b));
+// Bucket of a screened value: floor(f * bscale + boff) clamped to [0, 255] (one fused
+// multiply-add, rounded to nearest, then a floor conversion to an unsigned byte, which
+// clamps to [0, 255] by itself and sends NaN to 0), so the map is non-decreasing in f.
+// boff = -lo * bscale puts the row's smallest sampled value lo at the bottom of bucket 0,
+// up to rounding.
+__device__ __forceinline__ int fused_bucket(float f, float bscale, float boff) {
+    unsigned short b;
+    asm("cvt.rmi.u8.f32 %0, %1;" : "=h"(b) : "f"(__fmaf_rn(f, bscale, boff)));
+    return (int)b;
 }
 
 // Smallest float x (over all non-NaN floats, in order) with fused_bucket(x) >= b, for
 // 1 <= b <= 255 and a finite bscale > 0 (then bucket(-inf) = 0 and bucket(+inf) = 255).
-// Starts from vlo + b / bscale, within a few units in the last place of the edge for
+// Starts from (b - boff) / bscale, within a few units in the last place of the edge for
 // ranges that fp32 resolves, and steps float by float; a bisection over the whole
 // float order decides when that has not settled within 64 steps.
-__device__ float fused_bucket_edge(int b, float vlo, float bscale) {
-    uint32_t g = f32_key(__fadd_rn(vlo, __fdiv_rn((float)b, bscale)));
+__device__ float fused_bucket_edge(int b, float bscale, float boff) {
+    uint32_t g = f32_key(__fdiv_rn(__fsub_rn((float)b, boff), bscale));
     const uint32_t kmin = f32_key(-INFINITY), kmax = f32_key(INFINITY);
     if (g > kmin && g <= kmax) {
-        if (fused_bucket(key_to_f32(g), vlo, bscale) >= b) {
+        if (fused_bucket(key_to_f32(g), bscale, boff) >= b) {
             for (int step = 0; step < 64; ++step) {  // down while the float below is still in
-                if (g == kmin || fused_bucket(key_to_f32(g - 1u), vlo, bscale) < b) return key_to_f32(g);
+                if (g == kmin || fused_bucket(key_to_f32(g - 1u), bscale, boff) < b) return key_to_f32(g);
                 --g;
             }
         } else {
             for (int step = 0; step < 64; ++step) {  // up until in
                 ++g;
                 if (g > kmax) break;
-                if (fused_bucket(key_to_f32(g), vlo, bscale) >= b) return key_to_f32(g);
+                if (fused_bucket(key_to_f32(g), bscale, boff) >= b) return key_to_f32(g);
             }
         }
     }
     uint32_t lo = kmin, hi = kmax;
     while (hi - lo > 1u) {
         const uint32_t mid = lo + (hi - lo) / 2u;
-        if (fused_bucket(key_to_f32(mid), vlo, bscale) >= b)
+        if (fused_bucket(key_to_f32(mid), bscale, boff) >= b)
             hi = mid;
         else
             lo = mid;
@@ -331,7 +335,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             return true;
         };
 
-        // ---- sample: the row's value range [vlo, vlo + 256 / bscale]
+        // ---- sample: the row's value range [lo, hi], and the bucket map over it
         {
             float lo = INFINITY, hi = -INFINITY;
             uint32_t v[32];
@@ -348,7 +352,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             part_hi[part * 128 + t] = hi;
         }
         rows_sync();
-        float vlo = 0.f, bscale = 0.f;
+        float bscale = 0.f, boff = 0.f;
         {
             float lo = part_lo[t], hi = part_hi[t];
 #pragma unroll
@@ -359,9 +363,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             const float range = hi - lo;
             if (range > 0.f && range <= 3.0e38f) {
                 const float sc = 256.0f / range;
-                if (sc <= 3.0e38f) {
-                    vlo = lo;
+                if (sc <= 3.0e38f && fabsf(lo) * sc <= 3.0e38f) {
                     bscale = sc;
+                    boff = -lo * sc;
                 }
             }
         }
@@ -381,8 +385,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             const int lim = active ? nBb - ch * 128 - 32 * part : 0;  // columns i < lim are blocks
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-                const int b = fused_bucket(__uint_as_float(v[i]), vlo, bscale);
-                atomicAdd(&hist[(b >> 1) * 128 + t], i < lim ? 1u << ((b & 1) << 4) : 0u);
+                const uint32_t b = (uint32_t)fused_bucket(__uint_as_float(v[i]), bscale, boff);
+                atomicAdd(&hist[(b >> 1) * 128 + t], i < lim ? 1u + (b & 1u) * 0xFFFFu : 0u);
             }
         }
         rows_sync();
@@ -429,8 +433,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             } else {
                 ri.flags = 1;
                 if (bscale > 0.f) {
-                    if (bstar > 0) ri.A = fused_bucket_edge(bstar, vlo, bscale);
-                    if (bstar < 255) ri.Bv = fused_bucket_edge(bstar + 1, vlo, bscale);
+                    if (bstar > 0) ri.A = fused_bucket_edge(bstar, bscale, boff);
+                    if (bstar < 255) ri.Bv = fused_bucket_edge(bstar + 1, bscale, boff);
                 }
                 if (ri.Bv < INFINITY) ri.hiT = __double2float_ru((double)ri.Bv + 2.0 * ri.delta);
                 if (ri.A > -INFINITY) ri.loT = __double2float_rd((double)ri.A - 2.0 * ri.delta);
