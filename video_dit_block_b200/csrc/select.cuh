@@ -159,7 +159,7 @@ struct PoolSecond {
 };
 
 template <int D, int BLK = kBlock>
-__global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restrict__ x,
+__global__ void __launch_bounds__(256, 4) pool_kernel(const __nv_bfloat16* __restrict__ x,
                                                    const int32_t* __restrict__ valid_len, int H,
                                                    int Npad, double* __restrict__ mean64,
                                                    __nv_bfloat16* __restrict__ hi16,
@@ -167,7 +167,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
                                                    double* __restrict__ norm, long long n_groups,
                                                    PoolSecond second) {
     constexpr int LPB = D / 8;  // lanes per block group
-    constexpr int UNROLL = 16;
+    constexpr int UNROLL = 8;   // with four CTAs per SM: more rows in flight per SM than 16 with two
     const int nB = Npad / BLK;
     unsigned bid = blockIdx.x;
     if (bid >= second.blocks0) {
