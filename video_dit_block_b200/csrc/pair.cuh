@@ -86,22 +86,32 @@ __global__ void __launch_bounds__(256) pair_bitmap_kernel(PairWorkspace ws, cons
 constexpr int kPairWarps = 8;
 constexpr int kPairSpan = 2 * kPairWindow + kPairWarps;  // blocks staged per CTA
 
+// Words per staged bitmap row: W rounded up to a multiple of 4 (16-byte vector reads)
+// and, if that is a multiple of 8, 4 more, so that the rows read by 8 consecutive lanes
+// start in different banks.
+__host__ __device__ inline int pair_row_words(int W) {
+    int p = (W + 3) / 4 * 4;
+    if (p % 8 == 0) p += 4;
+    return p;
+}
+
 __global__ void __launch_bounds__(256) pair_propose_kernel(PairWorkspace ws,
                                                            const int32_t* __restrict__ kv_cnt,
                                                            const int32_t* __restrict__ valid_len,
                                                            int H, int nQ, int tiles_per_bh) {
-    extern __shared__ uint32_t sbits[];  // [kPairSpan][W]
+    extern __shared__ __align__(16) uint32_t sbits[];  // [kPairSpan][Wp], zero-padded
     const int bh = blockIdx.x / tiles_per_bh;
     const int a0 = (blockIdx.x % tiles_per_bh) * kPairWarps;
     const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
     const int L = valid_len ? valid_len[bh / H] : nQ * 64;
     const int nB = (L + 63) / 64;
     const int W = (nQ + 31) / 32;
+    const int Wp = pair_row_words(W);
     const uint32_t* gbits = ws.bits + (size_t)bh * nQ * W;
     const int lo = a0 - kPairWindow;
-    for (int i = threadIdx.x; i < kPairSpan * W; i += blockDim.x) {
-        const int c = lo + i / W;
-        sbits[i] = (c >= 0 && c < nB) ? gbits[(size_t)c * W + (i % W)] : 0u;
+    for (int i = threadIdx.x; i < kPairSpan * Wp; i += blockDim.x) {
+        const int c = lo + i / Wp, w = i % Wp;
+        sbits[i] = (c >= 0 && c < nB && w < W) ? gbits[(size_t)c * W + w] : 0u;
     }
     __syncthreads();
     const int a = a0 + warp;
@@ -113,7 +123,7 @@ __global__ void __launch_bounds__(256) pair_propose_kernel(PairWorkspace ws,
         if (lane == 0) ws.proposal[row] = -1;
         return;
     }
-    const uint32_t* ba = sbits + (size_t)(a - lo) * W;
+    const uint32_t* ba = sbits + (size_t)(a - lo) * Wp;
     // lane l scores a - 64 + l, a - 32 + l, a + 1 + l, a + 33 + l.  Preference as one
     // ordered 32-bit key: larger overlap, then smaller distance, then the lower index
     // (of the two candidates at one distance, the one before a); 0 = no candidate.
@@ -125,9 +135,13 @@ __global__ void __launch_bounds__(256) pair_propose_kernel(PairWorkspace ws,
         const int c = slot < half ? a - kPairWindow + 32 * slot + lane : a + 1 + 32 * (slot - half) + lane;
         key[slot] = 0u;
         if (c < 0 || c >= nB) continue;
-        const uint32_t* bc = sbits + (size_t)(c - lo) * W;
+        const uint32_t* bc = sbits + (size_t)(c - lo) * Wp;
         int ov = 0;
-        for (int w = 0; w < W; ++w) ov += __popc(ba[w] & bc[w]);
+        for (int w = 0; w < Wp; w += 4) {  // four words per read; the padding is zero
+            const uint4 x = *reinterpret_cast<const uint4*>(ba + w);
+            const uint4 y = *reinterpret_cast<const uint4*>(bc + w);
+            ov += __popc(x.x & y.x) + __popc(x.y & y.y) + __popc(x.z & y.z) + __popc(x.w & y.w);
+        }
         const int dist = c > a ? c - a : a - c;  // 1 .. kPairWindow
         key[slot] = ((uint32_t)(ov + 1) << 8) | ((uint32_t)(kPairWindow - dist) << 1) | (c < a ? 1u : 0u);
     }

@@ -713,7 +713,7 @@ extern "C" sba_status sba_pair_query_blocks(const int32_t* kv_idx, const int32_t
     sba::pair_bitmap_kernel<<<wgrid, 256, 8 * ((nQ + 31) / 32) * 4, s>>>(ws, kv_idx, kv_cnt, nQ, kmax, rows);
     const int W = (nQ + 31) / 32;
     const int tiles_per_bh = (nQ + sba::kPairWarps - 1) / sba::kPairWarps;
-    const size_t psmem = (size_t)sba::kPairSpan * W * 4;   // <= 136 x 128 x 4 = 68 KB
+    const size_t psmem = (size_t)sba::kPairSpan * sba::pair_row_words(W) * 4;  // <= 136 x 132 x 4 = 70 KB
     if (cudaFuncSetAttribute(sba::pair_propose_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)psmem) != cudaSuccess)
         return SBA_ERR_CUDA;
