@@ -173,3 +173,27 @@ def test_wide_windows_fall_back_to_the_row_routine(sba, oracle_mod):
     w.k = k
     for s in (0.5, 0.75, 0.9):
         check_routing(sba, oracle_mod, w, s)
+
+
+@pytest.mark.parametrize("n_blocks", [127, 128, 129, 255, 256, 257])
+def test_chunk_boundaries(sba, oracle_mod, n_blocks):
+    """Block counts just below, at and above one and two 128-block chunks of the fused
+    screen (the last chunk partial or full, one or two query tiles per head)."""
+    w = make_custom(1, 2, 128, (1, n_blocks, 64), 0.8, seed=50 + n_blocks)
+    assert w.Npad // 64 == n_blocks
+    check_routing(sba, oracle_mod, w)
+
+
+def test_d64_several_chunks(sba, oracle_mod):
+    """D = 64 (one 64-channel slice per operand tile) over three chunks, ragged."""
+    w = make_custom(2, 2, 64, (5, 32, 120), 0.75, seed=61, drop_rate=0.1)
+    assert w.Npad // 64 > 256
+    check_routing(sba, oracle_mod, w)
+
+
+def test_short_sample_beside_long_one(sba, oracle_mod):
+    """A sample far shorter than the padded length: the range sample strides over the
+    padded block count, so few of its 128 sampled blocks lie inside the short sample."""
+    w = make_custom(2, 2, 128, (4, 32, 192), 0.75, seed=62)      # 384 blocks
+    w.valid_len = np.array([w.Npad, 64 * 23 + 5], dtype=np.int32)  # 24 blocks in sample 1
+    check_routing(sba, oracle_mod, w)
