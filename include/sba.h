@@ -79,7 +79,10 @@ int32_t sba_keep_count(int32_t n_blocks, double sparsity);
 int32_t sba_keep_count_budget(int32_t n_blocks, double sparsity, int32_t budget);
 
 /* Bytes of device workspace sba_pool_select needs for this shape (0 on bad
- * arguments).  The workspace holds the pooled Q and K block means. */
+ * arguments).  The workspace holds the pooled Q and K block means, one record per
+ * routing row for the selection (its window around the k-th score and its keep mask),
+ * and room for the screened scores of rows the selection hands to its slower exact
+ * routine (none on typical inputs). */
 size_t sba_pool_select_workspace_size(int B, int H, int Npad, int D, int block);
 
 /* Routing step: pool Q and K per block, score every key block for every query

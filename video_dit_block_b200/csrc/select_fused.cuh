@@ -7,8 +7,9 @@
 // re-scoring of the band around the k-th value), but the screened scores live only in
 // TMEM and registers.
 //
-// select_fused_kernel.  A CTA owns 128 query blocks I = m0 + t of one (b, h): thread t
-// of warps 0-3 owns row t = TMEM lane t.  The tensor cores score the row against 128
+// select_fused_kernel.  A CTA owns 128 query blocks I = m0 + t of one (b, h): row t is
+// TMEM lane t, served by four threads (see the warp roles).  The tensor cores score the
+// row against 128
 // key blocks at a time (a "chunk": M128 N128, S = qhi.khi + qlo.khi + qhi.klo in one
 // fp32 TMEM buffer of 128 columns, two buffers), in this order:
 //   sample   one hi.hi product against 128 key blocks spread evenly over the head
@@ -21,8 +22,9 @@
 //            [A - 2 delta, hiT) -- the window -- go to a list of at most kFusedList
 //            (value, J) entries.
 // Each row then writes a record (header, window, mask) for select_finish_kernel.  A row
-// whose window overflows, or whose bound is not finite, gets a pass C instead: its screened scores go to ws.scores and
-// its index to ws.ovf_rows, and topk_rest_kernel finishes it with topk_kernel's routine.
+// whose window overflows, or whose bound is not finite, gets a pass C instead: its
+// screened scores go to ws.scores and its index to ws.ovf_rows, and topk_rest_kernel
+// finishes it with topk_kernel's routine.
 //
 // Warp roles (576 threads, one CTA per SM: 224 KB of shared memory for D = 128):
 //   warps 0-15 rows: warp w reads TMEM lanes 32 (w mod 4) .. + 31 and columns 32 (w / 4)
@@ -65,8 +67,9 @@ struct FusedSmem {
     static constexpr int kList = kK + kSlots * kTile;
     static constexpr int kListBytes = kFusedList * 128 * 8;
     static constexpr int kRegionBytes = 128 * 128 * 4;
-    static constexpr int kBars = kList + kRegionBytes;   // q_full, k_full[3], k_free[3], acc_full[2], acc_empty[2], drain
-    static constexpr int kCtl = kBars + 12 * 8;        // tmem base, abort flag
+    // q_full, k_full[3], k_free[3], acc_full[2], acc_empty[2], drain
+    static constexpr int kBars = kList + kRegionBytes;
+    static constexpr int kCtl = kBars + 12 * 8;  // tmem base, abort flag
     static constexpr int kTotal = kCtl + 16;
     static constexpr int kAlloc = kTotal + 1024;
     static_assert(kListBytes + 128 * 32 + 128 * 4 <= kRegionBytes, "lists, row info and counters share the region");
