@@ -62,6 +62,9 @@ def test_our_arm_line():
     assert p["max_abs"] <= 2e-2 and p["mean_abs"] <= 2e-3 and p["out_rows"] > 0
     m = d["median_ms"]
     assert m["step"] > 0 and m["attn"] > 0 and m["select"] > 0
+    r = m["rounds"]
+    assert r["n"] >= 1 and r["steps_each"] >= 1 and r["step"] > 0 and r["attn"] > 0
+    assert d["routing"]["pool_select_ms"] > 0 and d["routing"]["pair_ms"] > 0
 
 
 @pytest.mark.gpu
