@@ -64,6 +64,9 @@ def test_our_arm_line():
     assert m["step"] > 0 and m["attn"] > 0 and m["select"] > 0
     r = m["rounds"]
     assert r["n"] >= 1 and r["steps_each"] >= 1 and r["step"] > 0 and r["attn"] > 0
+    f = m["l2_flushed"]
+    assert f["n"] == r["n"] and f["flush_bytes"] >= 4 * 126 * 10**6
+    assert f["step"] > 0 and f["attn"] > 0 and f["routing_call"] > 0 and f["attn_tflops"] > 0
     assert d["routing"]["pool_select_ms"] > 0 and d["routing"]["pair_ms"] > 0
 
 
