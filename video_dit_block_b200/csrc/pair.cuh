@@ -85,6 +85,7 @@ __global__ void __launch_bounds__(256) pair_bitmap_kernel(PairWorkspace ws, cons
 // overlap with every candidate and proposes nothing, so it stays in order.
 constexpr int kPairWarps = 8;
 constexpr int kPairSpan = 2 * kPairWindow + kPairWarps;  // blocks staged per CTA
+static_assert(kPairSpan % kPairWarps == 0, "the staging gives each warp the same number of rows");
 
 // Words per staged bitmap row: W rounded up to a multiple of 4 (16-byte vector reads)
 // and, if that is a multiple of 8, 4 more, so that the rows read by 8 consecutive lanes
@@ -109,9 +110,21 @@ __global__ void __launch_bounds__(256) pair_propose_kernel(PairWorkspace ws,
     const int Wp = pair_row_words(W);
     const uint32_t* gbits = ws.bits + (size_t)bh * nQ * W;
     const int lo = a0 - kPairWindow;
-    for (int i = threadIdx.x; i < kPairSpan * Wp; i += blockDim.x) {
-        const int c = lo + i / Wp, w = i % Wp;
-        sbits[i] = (c >= 0 && c < nB && w < W) ? gbits[(size_t)c * W + w] : 0u;
+    // warp w stages rows w, w + 8, ...: six loads of a lane in flight before their stores
+    constexpr int kRowsPerWarp = kPairSpan / kPairWarps, kGroup = 6;
+    for (int w = lane; w < Wp; w += 32) {
+#pragma unroll 1
+        for (int i0 = 0; i0 < kRowsPerWarp; i0 += kGroup) {
+            uint32_t v[kGroup];
+#pragma unroll
+            for (int j = 0; j < kGroup; ++j) {
+                const int c = lo + warp + kPairWarps * (i0 + j);
+                v[j] = (i0 + j < kRowsPerWarp && c >= 0 && c < nB && w < W) ? gbits[(size_t)c * W + w] : 0u;
+            }
+#pragma unroll
+            for (int j = 0; j < kGroup; ++j)
+                if (i0 + j < kRowsPerWarp) sbits[(warp + kPairWarps * (i0 + j)) * Wp + w] = v[j];
+        }
     }
     __syncthreads();
     const int a = a0 + warp;

@@ -705,10 +705,20 @@ __global__ void __launch_bounds__(32 * kFinishWarps) select_finish_kernel(Select
                 p[u] = 0.0;
 #pragma unroll
                 for (int i = 0; i < D / 32; ++i) p[u] = fma(qd[i], kv[u][i], p[u]);
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1) p[u] += __shfl_xor_sync(0xffffffffu, p[u], off);
             }
-            if (lane < 4 && m + lane < n_band) rx[m + lane] = (lane == 0 ? p[0] : lane == 1 ? p[1] : lane == 2 ? p[2] : p[3]) * inv;
+            // a transposing butterfly: at distance 16 each lane keeps two of the four
+            // sums (members 0, 1 below lane 16, members 2, 3 from it) and sends the
+            // other two, at distance 8 one of those, then three plain steps; lanes
+            // 8u .. 8u + 7 end with member u's sum over all 32 lanes
+            const bool up16 = (lane & 16) != 0, up8 = (lane & 8) != 0;
+            double h0 = up16 ? p[2] : p[0], h1 = up16 ? p[3] : p[1];
+            h0 += __shfl_xor_sync(0xffffffffu, up16 ? p[0] : p[2], 16);
+            h1 += __shfl_xor_sync(0xffffffffu, up16 ? p[1] : p[3], 16);
+            double r = up8 ? h1 : h0;
+            r += __shfl_xor_sync(0xffffffffu, up8 ? h0 : h1, 8);
+#pragma unroll
+            for (int off = 4; off > 0; off >>= 1) r += __shfl_xor_sync(0xffffffffu, r, off);
+            if ((lane & 7) == 0 && m + (lane >> 3) < n_band) rx[m + (lane >> 3)] = r * inv;
         }
         __syncwarp();
         const double qn = ws.qnorm[(size_t)rid], kmx = ws.kmaxn[bh];
