@@ -714,12 +714,13 @@ def run_ours(args):
         # per step: routing = pooling (Q and K in one launch) + key-norm maximum + fused
         # screen + finish + rest rows (the log-sum-exp router: the same pooling launch +
         # key-norm maximum + screen, only when blocks are dropped, + top-k); pairing =
-        # bitmaps + 4 x (propose, resolve) + emit (not with the CTA-pair kernel); 1 attention
+        # bitmaps + proposals + the matching rounds and tile list in one launch (not with
+        # the CTA-pair kernel); 1 attention
         # (--producer: 2 producer launches and 2 splits of the given means replace pooling)
         # (--compensate mean: 2 block-mean launches before the attention)
         # (--prune: norm + select + 3 gathers, and the positions' gather with --producer)
         "gpu_launches": ((3 + (1 if w.sparsity > 0 else 0) if lse_router else 5) + (3 if args.producer else 0)
-                         + (0 if pair_kernel else 10) + 1 + (2 if args.compensate == "mean" else 0)
+                         + (0 if pair_kernel else 3) + 1 + (2 if args.compensate == "mean" else 0)
                          + (5 + (1 if args.producer else 0) if args.prune is not None else 0)) * K,
         "clocks": clk,
     }

@@ -9,7 +9,8 @@
 //   2. a few rounds of mutual-best matching: every unmatched query block proposes
 //      the unmatched block within +-64 positions whose kept set overlaps its own
 //      most (ties: nearer, then lower), and mutual proposals are matched.  Overlaps
-//      are computed once; later rounds walk each block's 16 best candidates.  The
+//      are computed once; later rounds walk each block's 16 best candidates, all
+//      rounds of a (b, h) in one CTA with its proposals in shared memory.  The
 //      window reaches the same position one frame later in the raster order of
 //      these latent grids (25-57 blocks per frame), where the kept sets are most
 //      alike;
@@ -26,6 +27,7 @@ constexpr int kPairWindow = 64;  // a multiple of 32
 constexpr int kPairRounds = 4;
 
 constexpr int kPairCands = 16;  // candidates kept per query block after the overlap pass
+static_assert(kPairCands % 4 == 0, "a row of candidates is read as 16-byte vectors");
 
 struct PairWorkspace {
     uint32_t* bits;     // [BH][nQ][W] kept-set bitmaps, W = ceil(nQ / 32)
@@ -54,7 +56,7 @@ __host__ __device__ inline PairWorkspace carve_pair_workspace(void* base, size_t
 }
 
 // One warp per routing row (bh, I): its kept-set bitmap (built in shared memory,
-// then written out word by word); partner reset to -1.
+// then written out word by word).
 __global__ void __launch_bounds__(256) pair_bitmap_kernel(PairWorkspace ws, const int32_t* __restrict__ kv_idx,
                                                           const int32_t* __restrict__ kv_cnt, int nQ, int kmax,
                                                           long long rows) {
@@ -69,14 +71,21 @@ __global__ void __launch_bounds__(256) pair_bitmap_kernel(PairWorkspace ws, cons
     int cnt = kv_cnt[row];
     cnt = cnt < 0 ? 0 : (cnt > kmax ? kmax : cnt);
     const int32_t* lst = kv_idx + (size_t)row * kmax;
-    for (int t = lane; t < cnt; t += 32) {
-        const int J = lst[t];
-        if (J >= 0 && J < nQ) atomicOr(&bm[J >> 5], 1u << (J & 31));
+    constexpr int kLoads = 8;  // entries of a lane loaded before their bits are set
+    for (int t0 = 0; t0 < cnt; t0 += 32 * kLoads) {
+        int J[kLoads];
+#pragma unroll
+        for (int u = 0; u < kLoads; ++u) {
+            const int t = t0 + 32 * u + lane;
+            J[u] = t < cnt ? lst[t] : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < kLoads; ++u)
+            if (J[u] >= 0 && J[u] < nQ) atomicOr(&bm[J[u] >> 5], 1u << (J[u] & 31));
     }
     __syncwarp();
     uint32_t* out = ws.bits + (size_t)row * W;
     for (int w = lane; w < W; w += 32) out[w] = bm[w];
-    if (lane == 0) ws.partner[row] = -1;
 }
 
 // A CTA of 8 warps proposes for 8 consecutive query blocks a0..a0+7 of one (b, h);
@@ -176,51 +185,73 @@ __global__ void __launch_bounds__(256) pair_propose_kernel(PairWorkspace ws,
     if (lane == 0) ws.proposal[row] = cand[0];
 }
 
-// Later rounds, one thread per (bh, a): propose the first still-unmatched cached candidate.
-__global__ void pair_repropose_kernel(PairWorkspace ws, int nQ, long long rows) {
-    const long long row = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (row >= rows) return;
-    const long long bh = row / nQ;
-    int prop = -1;
-    if (ws.partner[row] < 0) {
-        const int32_t* cand = ws.cand + row * kPairCands;
-        for (int r = 0; r < kPairCands; ++r) {
-            const int c = cand[r];
-            if (c >= 0 && ws.partner[bh * nQ + c] < 0) {
-                prop = c;
-                break;
-            }
-        }
-    }
-    ws.proposal[row] = prop;
-}
+// One CTA per (b, h) for the matching rounds and the tile list, with the head's
+// proposals and partners in shared memory and a block barrier between the steps of
+// a round (so every step sees the whole previous step, as separate launches would):
+//   resolve    a proposal returned by its target matches the two;
+//   repropose  (rounds after the first) every unmatched block proposes its first
+//              cached candidate that is still unmatched;
+// then warp 0 writes the tile list pair_order[bh][2 * nP] (nP = ceil(nQ / 2)).
+constexpr int kPairMatchThreads = 1024;
 
-// One thread per (bh, a): match mutual proposals.
-__global__ void pair_resolve_kernel(PairWorkspace ws, int nQ, long long rows) {
-    const long long row = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (row >= rows) return;
-    const long long bh = row / nQ;
-    const int c = ws.proposal[row];
-    if (c < 0 || ws.partner[row] >= 0) return;
-    if (ws.proposal[bh * nQ + c] == (int)(row % nQ)) ws.partner[row] = c;
-}
-
-// One warp per bh: the tile list pair_order[bh][2 * nP] (nP = ceil(nQ / 2)).
-__global__ void pair_emit_kernel(PairWorkspace ws, const int32_t* __restrict__ valid_len, int H, int nQ,
-                                 int32_t* __restrict__ pair_order, int BH) {
-    const int bh = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
-    const int lane = threadIdx.x & 31;
-    if (bh >= BH) return;
+__global__ void __launch_bounds__(kPairMatchThreads) pair_match_kernel(PairWorkspace ws,
+                                                                     const int32_t* __restrict__ valid_len,
+                                                                     int H, int nQ,
+                                                                     int32_t* __restrict__ pair_order) {
+    extern __shared__ int32_t pm_smem[];  // proposal [nQ], partner [nQ]
+    int32_t* prop = pm_smem;
+    int32_t* part = pm_smem + nQ;
+    const int bh = blockIdx.x;
     const int L = valid_len ? valid_len[bh / H] : nQ * 64;
     const int nB = (L + 63) / 64;
+    const size_t base = (size_t)bh * nQ;
+    for (int a = threadIdx.x; a < nQ; a += blockDim.x) {
+        prop[a] = ws.proposal[base + a];
+        part[a] = -1;
+    }
+    __syncthreads();
+    for (int r = 0; r < kPairRounds; ++r) {
+        if (r > 0) {
+            for (int a = threadIdx.x; a < nQ; a += blockDim.x) {
+                int p = -1;
+                if (part[a] < 0) {
+                    // the row's candidates in four 16-byte loads, then scanned in order
+                    const int4* c4 = reinterpret_cast<const int4*>(ws.cand + (base + a) * kPairCands);
+                    int cs[kPairCands];
+#pragma unroll
+                    for (int v = 0; v < kPairCands / 4; ++v) {
+                        const int4 x = c4[v];
+                        cs[4 * v] = x.x;
+                        cs[4 * v + 1] = x.y;
+                        cs[4 * v + 2] = x.z;
+                        cs[4 * v + 3] = x.w;
+                    }
+#pragma unroll
+                    for (int i = 0; i < kPairCands; ++i) {
+                        if (p < 0 && cs[i] >= 0 && cs[i] < nQ && part[cs[i]] < 0) p = cs[i];
+                    }
+                }
+                prop[a] = p;
+            }
+            __syncthreads();
+        }
+        for (int a = threadIdx.x; a < nQ; a += blockDim.x) {
+            const int c = prop[a];
+            if (c >= 0 && c < nQ && part[a] < 0 && prop[c] == a) part[a] = c;
+        }
+        __syncthreads();
+    }
+    for (int a = threadIdx.x; a < nQ; a += blockDim.x) ws.partner[base + a] = part[a];
+    if (threadIdx.x >= 32) return;
+
+    const int lane = threadIdx.x;
     const int nP = (nQ + 1) / 2;
-    const int32_t* partner = ws.partner + (size_t)bh * nQ;
     int32_t* out = pair_order + (size_t)bh * 2 * nP;
     int pos = 0;
     // matched pairs, by their lower block
     for (int a0 = 0; a0 < nQ; a0 += 32) {
         const int a = a0 + lane;
-        const int pa = a < nB ? partner[a] : -1;
+        const int pa = a < nB ? part[a] : -1;
         const bool lead = a < nB && pa > a;
         const uint32_t bal = __ballot_sync(0xffffffffu, lead);
         if (lead) {
@@ -234,7 +265,7 @@ __global__ void pair_emit_kernel(PairWorkspace ws, const int32_t* __restrict__ v
     for (int pass = 0; pass < 2; ++pass) {
         for (int a0 = 0; a0 < nQ; a0 += 32) {
             const int a = a0 + lane;
-            const bool take = pass == 0 ? (a < nB && partner[a] < 0) : (a >= nB && a < nQ);
+            const bool take = pass == 0 ? (a < nB && part[a] < 0) : (a >= nB && a < nQ);
             const uint32_t bal = __ballot_sync(0xffffffffu, take);
             if (take) out[pos + __popc(bal & ((1u << lane) - 1u))] = a;
             pos += __popc(bal);

@@ -713,19 +713,18 @@ extern "C" sba_status sba_pair_query_blocks(const int32_t* kv_idx, const int32_t
     sba::pair_bitmap_kernel<<<wgrid, 256, 8 * ((nQ + 31) / 32) * 4, s>>>(ws, kv_idx, kv_cnt, nQ, kmax, rows);
     const int W = (nQ + 31) / 32;
     const int tiles_per_bh = (nQ + sba::kPairWarps - 1) / sba::kPairWarps;
+    if (BH * tiles_per_bh > 0x7fffffffULL) return SBA_ERR_UNSUPPORTED;  // one grid dimension
     const size_t psmem = (size_t)sba::kPairSpan * sba::pair_row_words(W) * 4;  // <= 136 x 132 x 4 = 70 KB
     if (cudaFuncSetAttribute(sba::pair_propose_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)psmem) != cudaSuccess)
         return SBA_ERR_CUDA;
-    const unsigned tgrid = (unsigned)((rows + 255) / 256);
     sba::pair_propose_kernel<<<(unsigned)(BH * tiles_per_bh), 32 * sba::kPairWarps, psmem, s>>>(
         ws, kv_cnt, valid_len, H, nQ, tiles_per_bh);
-    sba::pair_resolve_kernel<<<tgrid, 256, 0, s>>>(ws, nQ, rows);
-    for (int r = 1; r < sba::kPairRounds; ++r) {
-        sba::pair_repropose_kernel<<<tgrid, 256, 0, s>>>(ws, nQ, rows);
-        sba::pair_resolve_kernel<<<tgrid, 256, 0, s>>>(ws, nQ, rows);
-    }
-    sba::pair_emit_kernel<<<(unsigned)((BH + 7) / 8), 256, 0, s>>>(ws, valid_len, H, nQ, pair_order, (int)BH);
+    const size_t msmem = (size_t)2 * nQ * 4;  // <= 2 x 4096 x 4 = 32 KB
+    if (cudaFuncSetAttribute(sba::pair_match_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)msmem) != cudaSuccess)
+        return SBA_ERR_CUDA;
+    sba::pair_match_kernel<<<(unsigned)BH, sba::kPairMatchThreads, msmem, s>>>(ws, valid_len, H, nQ, pair_order);
     return cudaGetLastError() == cudaSuccess ? SBA_OK : SBA_ERR_CUDA;
 }
 
