@@ -88,11 +88,11 @@ __global__ void __launch_bounds__(256) pair_bitmap_kernel(PairWorkspace ws, cons
     for (int w = lane; w < W; w += 32) out[w] = bm[w];
 }
 
-// A CTA of 8 warps proposes for 8 consecutive query blocks a0..a0+7 of one (b, h);
-// the bitmaps of their joint window [a0 - 64, a0 + 71] are staged in shared memory
+// A CTA of 16 warps proposes for 16 consecutive query blocks a0..a0+15 of one (b, h);
+// the bitmaps of their joint window [a0 - 64, a0 + 79] are staged in shared memory
 // once.  A query block that keeps every key block (dense routing) has the same
 // overlap with every candidate and proposes nothing, so it stays in order.
-constexpr int kPairWarps = 8;
+constexpr int kPairWarps = 16;
 constexpr int kPairSpan = 2 * kPairWindow + kPairWarps;  // blocks staged per CTA
 static_assert(kPairSpan % kPairWarps == 0, "the staging gives each warp the same number of rows");
 
@@ -105,7 +105,7 @@ __host__ __device__ inline int pair_row_words(int W) {
     return p;
 }
 
-__global__ void __launch_bounds__(256) pair_propose_kernel(PairWorkspace ws,
+__global__ void __launch_bounds__(32 * kPairWarps) pair_propose_kernel(PairWorkspace ws,
                                                            const int32_t* __restrict__ kv_cnt,
                                                            const int32_t* __restrict__ valid_len,
                                                            int H, int nQ, int tiles_per_bh) {
@@ -119,8 +119,8 @@ __global__ void __launch_bounds__(256) pair_propose_kernel(PairWorkspace ws,
     const int Wp = pair_row_words(W);
     const uint32_t* gbits = ws.bits + (size_t)bh * nQ * W;
     const int lo = a0 - kPairWindow;
-    // warp w stages rows w, w + 8, ...: six loads of a lane in flight before their stores
-    constexpr int kRowsPerWarp = kPairSpan / kPairWarps, kGroup = 6;
+    // warp w stages rows w, w + 16, ...: five loads of a lane in flight before their stores
+    constexpr int kRowsPerWarp = kPairSpan / kPairWarps, kGroup = 5;
     for (int w = lane; w < Wp; w += 32) {
 #pragma unroll 1
         for (int i0 = 0; i0 < kRowsPerWarp; i0 += kGroup) {

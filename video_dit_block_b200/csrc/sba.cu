@@ -714,7 +714,7 @@ extern "C" sba_status sba_pair_query_blocks(const int32_t* kv_idx, const int32_t
     const int W = (nQ + 31) / 32;
     const int tiles_per_bh = (nQ + sba::kPairWarps - 1) / sba::kPairWarps;
     if (BH * tiles_per_bh > 0x7fffffffULL) return SBA_ERR_UNSUPPORTED;  // one grid dimension
-    const size_t psmem = (size_t)sba::kPairSpan * sba::pair_row_words(W) * 4;  // <= 136 x 132 x 4 = 70 KB
+    const size_t psmem = (size_t)sba::kPairSpan * sba::pair_row_words(W) * 4;  // <= 144 x 132 x 4 = 76 KB
     if (cudaFuncSetAttribute(sba::pair_propose_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)psmem) != cudaSuccess)
         return SBA_ERR_CUDA;
