@@ -104,6 +104,8 @@ def test_pairing_rejects(lib):
     assert lib.sba_pair_query_blocks(A, A, 1, 2, 1024, 8, NULL, 64, A, A, 16, S) == 1
     assert lib.sba_pair_query_blocks(A, A, 1, 2, 1000, 8, NULL, 64, A, A, 1 << 30, S) == 1
     assert lib.sba_pair_query_blocks(A, A, 1, 2, 1024, 8, NULL, 64, A, MIS, 1 << 30, S) == 3
+    # more (b, h) rows than one grid dimension holds: refused before any launch
+    assert lib.sba_pair_query_blocks(A, A, 65535, 65535, 64, 8, NULL, 64, A, A, 1 << 62, S) == 2
     assert lib.sba_attention_paired(A, A, A, A, A, 1, 2, 1024, 64, NULL, 64, A, A, 8, NULL, 0.0, S) == 1
     assert lib.sba_attention_paired(A, A, A, A, A, 1, 2, 1024, 64, NULL, 64, A, A, 8,
                                     ctypes.c_void_p(0x10002), 0.0, S) == 3

@@ -706,14 +706,15 @@ extern "C" sba_status sba_pair_query_blocks(const int32_t* kv_idx, const int32_t
     if (!aligned16(workspace) || !aligned16(valid_len) || (reinterpret_cast<uintptr_t>(kv_idx) & 3u) ||
         (reinterpret_cast<uintptr_t>(kv_cnt) & 3u) || (reinterpret_cast<uintptr_t>(pair_order) & 3u))
         return SBA_ERR_ALIGNMENT;
+    const long long rows = (long long)BH * nQ;
+    const int tiles_per_bh = (nQ + sba::kPairWarps - 1) / sba::kPairWarps;
+    // every grid below is one dimension of at most 2^31 - 1 CTAs
+    if ((rows + 7) / 8 > 0x7fffffffLL || (long long)BH * tiles_per_bh > 0x7fffffffLL) return SBA_ERR_UNSUPPORTED;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     sba::PairWorkspace ws = sba::carve_pair_workspace(workspace, BH, nQ);
-    const long long rows = (long long)BH * nQ;
     const unsigned wgrid = (unsigned)((rows + 7) / 8);   // 8 warps per 256-thread CTA
     sba::pair_bitmap_kernel<<<wgrid, 256, 8 * ((nQ + 31) / 32) * 4, s>>>(ws, kv_idx, kv_cnt, nQ, kmax, rows);
     const int W = (nQ + 31) / 32;
-    const int tiles_per_bh = (nQ + sba::kPairWarps - 1) / sba::kPairWarps;
-    if (BH * tiles_per_bh > 0x7fffffffULL) return SBA_ERR_UNSUPPORTED;  // one grid dimension
     const size_t psmem = (size_t)sba::kPairSpan * sba::pair_row_words(W) * 4;  // <= 144 x 132 x 4 = 76 KB
     if (cudaFuncSetAttribute(sba::pair_propose_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)psmem) != cudaSuccess)
