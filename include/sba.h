@@ -86,7 +86,11 @@ int32_t sba_keep_count_budget(int32_t n_blocks, double sparsity, int32_t budget)
 size_t sba_pool_select_workspace_size(int B, int H, int Npad, int D, int block);
 
 /* Routing step: pool Q and K per block, score every key block for every query
- * block, keep the best keep(nB_b, sparsity) blocks per (b, h, I).
+ * block, keep the best keep(nB_b, sparsity) blocks per (b, h, I).  The page
+ * "MiniMax-H3 on 8xH200 benchmark" (news.paixiangai.cn), section "How SubBlock
+ * sparse attention works": the pooling and scoring step that picks the key blocks
+ * and hands their indices to the attention kernel, here with one sub-block per
+ * block (the mean-pooled score in the file comment).
  *   q, k        bf16 [B, H, Npad, D] (read only)
  *   valid_len   int32 [B] device, or NULL
  *   sparsity    in [0, 1)
@@ -228,7 +232,12 @@ sba_status sba_attention_mean_compensated(const void* q, const void* k, const vo
 sba_status sba_block_means(const void* x, int B, int H, int Npad, int D,
                            const int32_t* valid_len, int block, double* out, void* stream);
 
-/* Exact attention over the routed key blocks.
+/* Exact attention over the routed key blocks: the block-sparse attention kernel of
+ * the page "MiniMax-H3 on 8xH200 benchmark" (news.paixiangai.cn), section "How
+ * SubBlock sparse attention works", which takes the kept block indices and never
+ * forms the full attention matrix; it computes the softmax over the kept tokens
+ * exactly (the critical blocks of PISA, page "Sol Video Inference Engine",
+ * sjmshsh.github.io, section 4.2.2, without its approximation of the rest).
  *   o      bf16 [B, H, Npad, D] (written; padding rows written as 0)
  *   lse    fp32 [B, H, Npad] natural-log log-sum-exp of the scaled logits, or
  *          NULL; padding rows and rows with no kept token get -inf
@@ -330,7 +339,10 @@ sba_status sba_gather_tokens(const void* src, int B, int H, int N, int row_bytes
                              const int32_t* valid_len_out, int Npad_out, void* dst, void* stream);
 
 /* Dense attention over all valid tokens of each sample (the sparsity = 0 case
- * without a routing), same layouts as sba_attention. */
+ * without a routing), same layouts as sba_attention.  On the page "MiniMax-H3 on
+ * 8xH200 benchmark", section "How SubBlock sparse attention works", sparsity is the
+ * fraction of key blocks dropped, so sparsity 0 keeps every block: full attention,
+ * which this call computes directly. */
 sba_status sba_dense_attention(const void* q, const void* k, const void* v, void* o, float* lse,
                                int B, int H, int Npad, int D, const int32_t* valid_len,
                                float softmax_scale, void* stream);
